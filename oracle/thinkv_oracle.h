@@ -1,0 +1,102 @@
+/*
+ * thinkv_oracle.h -- CPU oracle for the ThinKV decode hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * CPU-baseline / reference legs of bench.py may build, load or call this
+ * code.  It shares nothing with the CUDA library (no headers, helpers or
+ * tables) and is written to be checked by eye against the method it follows:
+ *
+ *   "ThinKV: Thought-Adaptive KV Cache Compression for Efficient Reasoning
+ *   Models" -- arXiv abstract (kernel extending PagedAttention that reuses
+ *   evicted tokens' memory slots without compaction) and the explainer's
+ *   "Resume Technique / Methodologie" sections: TBQ (precision assigned by
+ *   thought type, R > E > T, group quantisation), TBE (eviction of tokens of
+ *   less important thoughts) and "Implementation Systeme: Pensee Continue
+ *   (CT)" (a modified block table tracking thought type, start index and
+ *   eviction mask; new tokens of the same thought type overwrite evicted
+ *   slots in place).
+ *
+ * Every place where the pages are silent is filled by one stated reading;
+ * the list is kept with the design notes of this repository.
+ *
+ * Layout of the oracle's own state is deliberately "natural": one code per
+ * (page, kv-head, K|V, slot, channel), one (scale, zero) pair per group.
+ */
+#ifndef THINKV_ORACLE_H
+#define THINKV_ORACLE_H
+#include <stdint.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { OR_OK = 0, OR_ERR_INVALID = 1, OR_ERR_OUT_OF_PAGES = 2, OR_ERR_OUT_OF_BLOCKS = 3 };
+enum { OR_R = 0, OR_E = 1, OR_T = 2 };
+#define OR_PAGE 16
+
+typedef struct {
+  int32_t num_q_heads, num_kv_heads, head_dim, page_size, group_size;
+  int32_t bits[3];
+  int32_t max_seqs, max_blocks_per_seq;
+  int32_t pool_pages[3];
+} or_layout;
+
+typedef struct or_state or_state;
+
+or_state* or_create(const or_layout* L);
+void or_destroy(or_state* S);
+const or_layout* or_get_layout(const or_state* S);
+
+/* ---- the three operations ------------------------------------------- */
+int or_append(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos,
+              const uint8_t* tag, const uint16_t* k_fp16, const uint16_t* v_fp16);
+int or_evict(or_state* S, int32_t n, const int32_t* seq, const int32_t* budget,
+             const uint8_t* order /* 3 classes, NULL = T,E,R */);
+int or_decode(const or_state* S, int32_t n, const int32_t* seq,
+              const uint16_t* q_fp16, double softmax_scale, int32_t topk,
+              double* out /* [n][Hq][d] */, double* mass /* [n][Hq] or NULL */,
+              int32_t threads);
+
+/* ---- building blocks, exposed for the pin tests ---------------------- */
+uint16_t or_f16_round_down(float x);
+uint16_t or_f16_round_up(float x);
+uint16_t or_f16_round_nearest(float x);
+float or_f16_to_f32(uint16_t h);
+void or_f16_round_array(const float* x, int64_t n, int32_t mode, uint16_t* out);
+void or_quantize_group(const uint16_t* x, int32_t G, int32_t bits,
+                       uint8_t* codes, uint16_t* scale, uint16_t* zero);
+
+/* ---- state export (for comparisons) ----------------------------------- */
+/* Natural layouts:
+ *   codes[c]   : [pool_pages[c]][Hkv][2][16][d]      uint8 codes (bits<=8)
+ *                or uint16 raw fp16 bits (bits==16)
+ *   params[c]  : [pool_pages[c]][Hkv][2][16][d/G][2] uint16 fp16 (scale, zero)
+ *   slot_pos[c]: [pool_pages[c]][16]                  int32, -1 when dead
+ *   table      : [max_seqs][max_blocks]               uint64 page|class<<32|mask<<48
+ *   num_blocks, live_count, num_live : [max_seqs]     int32
+ *   free_slots, fifo : [max_seqs][3][max_blocks*16]   int32 (entry*16+slot)
+ *   free_top, fifo_head, fifo_tail : [max_seqs][3]    int32
+ *   live_list, live_index : [max_seqs][max_blocks]    int32
+ *   page_bump : [3]                                   int32
+ */
+const void* or_codes(const or_state* S, int c);
+const uint16_t* or_params(const or_state* S, int c);
+const int32_t* or_slot_pos(const or_state* S, int c);
+const uint64_t* or_table(const or_state* S);
+const int32_t* or_num_blocks(const or_state* S);
+const int32_t* or_free_slots(const or_state* S);
+const int32_t* or_free_top(const or_state* S);
+const int32_t* or_fifo(const or_state* S);
+const int32_t* or_fifo_head(const or_state* S);
+const int32_t* or_fifo_tail(const or_state* S);
+const int32_t* or_live_count(const or_state* S);
+const int32_t* or_live_list(const or_state* S);
+const int32_t* or_live_index(const or_state* S);
+const int32_t* or_num_live(const or_state* S);
+const int32_t* or_page_bump(const or_state* S);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
