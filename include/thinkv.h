@@ -1,0 +1,252 @@
+/*
+ * thinkv.h -- C ABI of libthinkv.so: the ThinKV decode hot path on B200 (sm_100a).
+ *
+ * What the library computes follows "ThinKV: Thought-Adaptive KV Cache
+ * Compression for Efficient Reasoning Models":
+ *   - arXiv abstract: a kernel that extends PagedAttention so that evicted
+ *     tokens' memory slots are reused without compaction;
+ *   - explainer, Resume Technique > Methodologie > "Quantification Adaptative
+ *     a la Pensee (TBQ)": token precision set by thought type, R > E > T, by
+ *     group quantisation;
+ *   - explainer, Methodologie > "Eviction Adaptative a la Pensee (TBE)":
+ *     tokens of less important thoughts are evicted;
+ *   - explainer, Methodologie > "Implementation Systeme: Pensee Continue (CT)":
+ *     a modified block table tracking thought type, start index and eviction
+ *     mask; new tokens of the same thought type overwrite evicted slots.
+ * Where the pages leave a choice open (integer code format, rounding of the
+ * fp16 scale/zero, free-list discipline, eviction order, the attention-mass
+ * statistic) this header states the choice made.
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers owned by the caller, except the
+ *     ones documented as host arrays.  The library allocates nothing and keeps
+ *     no global state.  fp16 values travel as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous
+ *     on it.
+ *   - Host-checkable errors (bad layout, null pointers, sizes) return a
+ *     non-zero thinkv_status before anything is launched.
+ *   - Device-detected errors (bad token/sequence data, exhausted page pool,
+ *     full block table, a bounded wait that ran out) are written to the
+ *     cache's sticky `status` word: the first error wins and later errors do
+ *     not overwrite it.  While *status != 0, append and evict do nothing;
+ *     decode still runs (it only reads state that every operation leaves
+ *     consistent).  thinkv_get_status / thinkv_clear_status read and reset it.
+ *   - Nothing traps or spins without a bound.
+ */
+#ifndef THINKV_H
+#define THINKV_H
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define THINKV_API __attribute__((visibility("default")))
+#else
+#define THINKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  THINKV_OK = 0,
+  THINKV_ERR_INVALID = 1,        /* bad argument or token/sequence data           */
+  THINKV_ERR_OUT_OF_PAGES = 2,   /* a class page pool is exhausted                */
+  THINKV_ERR_OUT_OF_BLOCKS = 3,  /* a sequence's block table is full              */
+  THINKV_ERR_CUDA = 4,           /* a CUDA runtime call failed                    */
+  THINKV_ERR_TIMEOUT = 5,        /* a bounded wait inside a kernel ran out        */
+  THINKV_ERR_WORKSPACE = 6       /* workspace missing or too small                */
+} thinkv_status;
+
+/* thought types (classes) */
+enum { THINKV_R = 0, THINKV_E = 1, THINKV_T = 2 };
+#define THINKV_PAGE_SIZE 16
+
+/* Geometry of one cache (one attention layer); immutable after creation.
+ *   num_q_heads % num_kv_heads == 0 and num_q_heads / num_kv_heads <= 8
+ *   (query heads map contiguously onto kv-heads: q-head h uses kv-head
+ *   h / (num_q_heads / num_kv_heads));
+ *   head_dim in {64, 128}; group_size in {32, 64}, dividing head_dim;
+ *   page_size == 16; bits[c] in {2, 4, 8, 16} for c = R, E, T;
+ *   1 <= max_seqs <= 65536; 1 <= max_blocks_per_seq; pool_pages[c] >= 0. */
+typedef struct {
+  int32_t num_q_heads, num_kv_heads, head_dim, page_size, group_size;
+  int32_t bits[3];
+  int32_t max_seqs, max_blocks_per_seq;
+  int32_t pool_pages[3];
+} thinkv_layout;
+
+/* The cache: device buffers, all allocated and owned by the caller with the
+ * sizes thinkv_buffer_bytes() reports, and initialised by thinkv_cache_reset().
+ *
+ *   pool[c]       uint8 [pool_pages[c]][num_kv_heads][page_head_bytes(c)]
+ *                 One "page-head block" holds 16 token slots of one kv-head:
+ *                 K codes, V codes, K params, V params (layout below).
+ *   slot_pos[c]   int32 [pool_pages[c]][16]  position of the token in each slot
+ *                 (the block table's "start index"), -1 when the slot is dead.
+ *   block_table   uint64 [max_seqs][max_blocks_per_seq]
+ *                 entry = page | class << 32 | live_mask << 48
+ *                 (bit s of live_mask: slot s holds a live token; this is the
+ *                 eviction mask, inverted).
+ *   num_blocks    int32 [max_seqs]       entries in use per sequence
+ *   free_slots    int32 [max_seqs][3][max_blocks_per_seq*16]  per (sequence,
+ *                 class) LIFO stack of reusable slots; a slot id is
+ *                 entry*16 + slot.   free_top int32 [max_seqs][3].
+ *   fifo          int32 [max_seqs][3][max_blocks_per_seq*16]  per (sequence,
+ *                 class) ring of live slot ids in arrival order;
+ *                 fifo_head, fifo_tail int32 [max_seqs][3] monotone counters
+ *                 (ring index = counter mod capacity).
+ *   live_count    int32 [max_seqs]       live tokens per sequence
+ *   live_list     int32 [max_seqs][max_blocks_per_seq]  table entries with a
+ *                 non-zero live_mask (first num_live[s] valid); an entry joins
+ *                 at the end when it gains its first live token and leaves by
+ *                 swap-with-last when it loses its last one.
+ *   live_index    int32 [max_seqs][max_blocks_per_seq]  position of an entry
+ *                 in live_list, -1 if absent.    num_live int32 [max_seqs].
+ *   page_bump     int32 [3]              pages handed out per class pool
+ *   status        int32 [1]              sticky device status (thinkv_status)
+ *
+ * Page-head block of a class with b = bits[c] < 16 (d = head_dim, G =
+ * group_size, ng = d/G), byte offsets:
+ *   [0, 2db)          K codes      [2db, 4db)  V codes
+ *   [4db, 4db+64ng)   K params     [4db+64ng, 4db+128ng)  V params
+ * params: [slot 16][group ng][scale, zero] fp16.
+ * Codes of one block are "lane-major": 32 lanes x (d*b/16) bytes; lane
+ * l = 4*gid + tid (gid 0..7, tid 0..3).  Within 32-bit words (or a 16-bit
+ * piece) the codes of even channels sit in the low half and those of odd
+ * channels in the high half, each half little-endian.
+ *   K: lane l holds, for group gr = 0..ng-1 and r = 0..1, the codes of slot
+ *      gid + 8r, channels gr*G + tid*G/4 .. +G/4 (a piece of G*b/32 bytes),
+ *      pieces ordered (gr, r).
+ *   V: lane l holds words ordered (P = 0..1, q = 0..d*b/128-1); word (P, q)
+ *      has slot 2*tid + 8P in its low 16 bits and slot 2*tid + 8P + 1 in its
+ *      high 16 bits; each half holds 16/b codes, element k of chunk q being
+ *      channel 16*(e/2) + gid + 8*(e%2) with e = q*16/b + k.
+ * For b == 16 the block is K raw fp16 [2db) then V raw fp16 [2db), in the same
+ * lane-major orders, with no params.
+ *
+ * Quantiser (reading of TBQ's group quantisation): per token, per kv-head,
+ * per K|V, per group of G consecutive channels: zero = min rounded toward
+ * -inf to fp16; scale = fp32((max - zero)/(2^b - 1)) rounded toward +inf to
+ * fp16; code = clamp(rint_half_even(fp32(fp32(x - zero)/scale)), 0, 2^b-1),
+ * all fp32 operations rounded to nearest; scale 0 gives code 0.  Dequantised
+ * value: zero + code*scale.
+ */
+typedef struct {
+  thinkv_layout L;
+  uint8_t* pool[3];
+  int32_t* slot_pos[3];
+  uint64_t* block_table;
+  int32_t* num_blocks;
+  int32_t* free_slots;
+  int32_t* free_top;
+  int32_t* fifo;
+  int32_t* fifo_head;
+  int32_t* fifo_tail;
+  int32_t* live_count;
+  int32_t* live_list;
+  int32_t* live_index;
+  int32_t* num_live;
+  int32_t* page_bump;
+  int32_t* status;
+} thinkv_cache;
+
+/* buffer ids for thinkv_buffer_bytes */
+enum {
+  THINKV_BUF_POOL_R = 0, THINKV_BUF_POOL_E = 1, THINKV_BUF_POOL_T = 2,
+  THINKV_BUF_SLOT_POS_R = 3, THINKV_BUF_SLOT_POS_E = 4, THINKV_BUF_SLOT_POS_T = 5,
+  THINKV_BUF_BLOCK_TABLE = 6, THINKV_BUF_NUM_BLOCKS = 7,
+  THINKV_BUF_FREE_SLOTS = 8, THINKV_BUF_FREE_TOP = 9,
+  THINKV_BUF_FIFO = 10, THINKV_BUF_FIFO_HEAD = 11, THINKV_BUF_FIFO_TAIL = 12,
+  THINKV_BUF_LIVE_COUNT = 13, THINKV_BUF_LIVE_LIST = 14, THINKV_BUF_LIVE_INDEX = 15,
+  THINKV_BUF_NUM_LIVE = 16, THINKV_BUF_PAGE_BUMP = 17, THINKV_BUF_STATUS = 18,
+  THINKV_NUM_BUFFERS = 19
+};
+
+/* THINKV_OK if the layout is supported, else THINKV_ERR_INVALID. */
+THINKV_API int thinkv_layout_check(const thinkv_layout* L);
+
+/* Bytes of one page-head block of class c (0 for a bad layout or class). */
+THINKV_API size_t thinkv_page_head_bytes(const thinkv_layout* L, int32_t cls);
+
+/* Bytes of buffer `which` (THINKV_BUF_*); 0 for a bad layout or id. */
+THINKV_API size_t thinkv_buffer_bytes(const thinkv_layout* L, int32_t which);
+
+/* Empties the cache on `stream`: no pages granted, no live tokens, all
+ * slot_pos and live_index -1, status THINKV_OK.  Pool bytes are left as they
+ * are (a slot's bytes are only read while the slot is live). */
+THINKV_API int thinkv_cache_reset(const thinkv_cache* cache, void* stream);
+
+/* Workspace bytes thinkv_append_quantize needs for n_tokens tokens. */
+THINKV_API size_t thinkv_append_workspace_bytes(const thinkv_layout* L, int32_t n_tokens);
+
+/* Quantize-on-append (TBQ + CT write path).
+ * Appends n_tokens tokens: token i belongs to sequence seq[i] at position
+ * pos[i] with thought type tag[i] (0 = R, 1 = E, 2 = T); k and v are fp16
+ * [n_tokens][num_kv_heads][head_dim].  Tokens must come grouped by sequence
+ * (one contiguous run per sequence per call, positions strictly ascending
+ * within the run); positions should also grow across calls (they order the
+ * tokens of a sequence).
+ * Each token takes the top slot of its (sequence, class) free stack; when that
+ * stack is empty the class pool grants the next page (page_bump[c]), a table
+ * entry {page, class, mask 0} is appended, slots 15..1 are pushed (slot 1 on
+ * top) and slot 0 is used.  The token's K and V are quantised at bits[class]
+ * into the slot, its live bit and slot_pos are set, its slot id is pushed on
+ * the (sequence, class) FIFO and live_count grows.  Grants follow call order.
+ * The call is all-or-nothing: device-detected errors (seq out of range, tag >
+ * 2, negative or non-ascending positions, a sequence in two runs ->
+ * INVALID; pool exhausted -> OUT_OF_PAGES; table full -> OUT_OF_BLOCKS,
+ * checked in that order) set *status and change nothing.
+ * workspace: device, >= thinkv_append_workspace_bytes(L, n_tokens) bytes,
+ * caller-owned scratch; contents need not be initialised. */
+THINKV_API int thinkv_append_quantize(const thinkv_cache* cache, int32_t n_tokens,
+                           const int32_t* seq, const int32_t* pos, const uint8_t* tag,
+                           const uint16_t* k, const uint16_t* v,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Evict to budget (TBE + CT free path).
+ * For each i < n_seqs, sequence seq[i] (distinct, in range) keeps at most
+ * budget[i] >= 0 live tokens: n = max(0, live_count - budget) victims are the
+ * oldest live tokens of the first class in `order` whose FIFO is non-empty,
+ * then the next class, and so on.  Each victim's live bit is cleared, its
+ * slot_pos set to -1 and its slot pushed on its class's free stack, in victim
+ * order; entries that lose their last live token leave live_list.  Pages stay
+ * with their sequence (no compaction, no release).
+ * order: HOST array of 3 distinct classes, or NULL for {T, E, R}.
+ * Bad seq/budget data -> *status = INVALID and nothing changes. */
+THINKV_API int thinkv_evict(const thinkv_cache* cache, int32_t n_seqs, const int32_t* seq,
+                 const int32_t* budget, const uint8_t* order, void* stream);
+
+/* Workspace bytes thinkv_decode_attention needs on the CURRENT device. */
+THINKV_API size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t n_seqs, int32_t topk);
+
+/* Decode attention over the mixed-precision pages (the PagedAttention
+ * extension).  For each i < n_seqs (seq[i] distinct or not) and each q-head
+ * h: o = softmax(scale * q K^T) V over the live tokens of seq[i], with K, V
+ * dequantised from their class's codes (raw for 16-bit classes); kv-head
+ * h / (Hq/Hkv).  q: fp16 [n_seqs][num_q_heads][head_dim]; out: fp16, same
+ * shape (a sequence with no live token gives zeros).  softmax_scale <= 0
+ * means 1/sqrt(head_dim).
+ * topk_mass: NULL, or fp32 [n_seqs][num_q_heads]: the share of the softmax
+ * probability held by the topk (1..64) most probable live tokens (1 when the
+ * sequence has <= topk live tokens, 0 when it has none).
+ * workspace: device, >= thinkv_decode_workspace_bytes(L, n_seqs, topk) bytes,
+ * caller-owned scratch, no initialisation needed.  1 <= n_seqs <= 16384. */
+THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs, const int32_t* seq,
+                            const uint16_t* q, uint16_t* out, float* topk_mass,
+                            int32_t topk, float softmax_scale,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then copies *status to *out (host). */
+THINKV_API int thinkv_get_status(const thinkv_cache* cache, void* stream, int32_t* out);
+
+/* Sets *status back to THINKV_OK (asynchronously on `stream`). */
+THINKV_API int thinkv_clear_status(const thinkv_cache* cache, void* stream);
+
+/* Static description of a status code. */
+THINKV_API const char* thinkv_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* THINKV_H */

@@ -1,0 +1,474 @@
+// thinkv_append.cu -- quantize-on-append into reused slots (TBQ + CT write path).
+//
+// "ThinKV: Thought-Adaptive KV Cache Compression for Efficient Reasoning
+// Models", explainer, Methodologie: TBQ gives each token the precision of its
+// thought type (R > E > T) by group quantisation; "Implementation Systeme:
+// Pensee Continue (CT)" lets a new token of a thought type overwrite a slot
+// freed by eviction, so the cache is never compacted.
+//
+// Two launches:
+//   1. append_assign_kernel (one CTA): validates the call, counts per-(sequence,
+//      class) demand, grants pages in call order with block-wide exclusive
+//      scans, then one warp per sequence run pops free slots / opens pages,
+//      writes table entries, slot positions, FIFO pushes, live-list joins and
+//      the final free stacks.  It writes every token's pool slot id to the
+//      workspace, and a go/no-go flag (the call is all-or-nothing).
+//   2. append_scatter_kernel (grid): one warp per (token, kv-head, K|V):
+//      group min/max by warp shuffles, directed-rounded fp16 zero/scale,
+//      round-half-even codes, then scatter into the lane-major page-head block.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "thinkv_common.cuh"
+#include "thinkv_internal.h"
+
+namespace thinkv {
+
+namespace {
+
+constexpr int kAssignThreads = 1024;
+constexpr int kAssignWarps = kAssignThreads / 32;
+
+__device__ inline unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Block-wide exclusive scan of one int per thread (1024 threads); returns the
+// exclusive prefix, `total` gets the block sum.  Uses `sh` (>= 33 ints).
+__device__ int block_exclusive_scan(int v, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kAssignWarps ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    sh[lane] = w;  // inclusive warp prefix
+  }
+  __syncthreads();
+  int warp_excl = warp == 0 ? 0 : sh[warp - 1];
+  *total = sh[kAssignWarps - 1];
+  __syncthreads();
+  return warp_excl + x - v;
+}
+
+__global__ void __launch_bounds__(kAssignThreads, 1)
+    append_assign_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
+                         const int32_t* __restrict__ pos, const uint8_t* __restrict__ tag,
+                         AppendWorkspace ws) {
+  extern __shared__ uint32_t seen[];  // max_seqs bits
+  __shared__ int s_err;
+  __shared__ int s_blocks_bad;
+  __shared__ int sh[40];
+  __shared__ int s_nruns;
+  __shared__ int s_total[3];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int max_seqs = C.L.max_seqs, nb_max = C.L.max_blocks_per_seq;
+  const int64_t cap = (int64_t)nb_max * kPage;
+
+  if (tid == 0) {
+    s_err = (*C.status != 0) ? -1 : 0;
+    s_blocks_bad = 0;
+    *ws.ok = 0;
+  }
+  for (int i = tid; i < (max_seqs + 31) / 32; i += kAssignThreads) seen[i] = 0;
+  __syncthreads();
+  if (s_err != 0) return;
+
+  // ---- phase 1: validate, mark run starts --------------------------------
+  int nruns_base = 0;
+  for (int base = 0; base < n; base += kAssignThreads) {
+    int i = base + tid;
+    int start = 0;
+    if (i < n) {
+      int s = seq[i], c = tag[i], p = pos[i];
+      bool bad = s < 0 || s >= max_seqs || c > 2 || p < 0;
+      start = (i == 0) || seq[i - 1] != s;
+      if (!bad && !start && p <= pos[i - 1]) bad = true;
+      if (!bad && start) {
+        uint32_t old = atomicOr(&seen[s >> 5], 1u << (s & 31));
+        if (old & (1u << (s & 31))) bad = true;  // a sequence in two runs
+      }
+      if (bad) s_err = THINKV_ERR_INVALID;
+    }
+    int total;
+    int excl = block_exclusive_scan(start, sh, &total);
+    if (start) ws.runs[nruns_base + excl].start = i;
+    nruns_base += total;
+  }
+  if (tid == 0) s_nruns = nruns_base;
+  __syncthreads();
+  if (s_err != 0) {
+    if (tid == 0) set_status(C.status, s_err);
+    return;
+  }
+  const int R = s_nruns;
+
+  // ---- phase 2: per-run demand (warp per run) ------------------------------
+  for (int r = warp; r < R; r += kAssignWarps) {
+    int start = ws.runs[r].start;
+    int end = (r + 1 < R) ? ws.runs[r + 1].start : n;
+    int s = seq[start];
+    int cnt[3] = {0, 0, 0};
+    for (int i = start + lane; i - lane < end; i += 32) {
+      int c = (i < end) ? tag[i] : -1;
+#pragma unroll
+      for (int cc = 0; cc < 3; ++cc) cnt[cc] += __popc(__ballot_sync(0xFFFFFFFFu, c == cc));
+    }
+    if (lane == 0) {
+      int gs = 0;
+      RunInfo& ri = ws.runs[r];
+      ri.len = end - start;
+      ri.seq = s;
+#pragma unroll
+      for (int cc = 0; cc < 3; ++cc) {
+        int need = cnt[cc] - C.free_top[s * 3 + cc];
+        int g = need > 0 ? (need + kPage - 1) / kPage : 0;
+        ri.cnt[cc] = cnt[cc];
+        ri.grants[cc] = g;
+        gs += g;
+      }
+      if ((int64_t)C.num_blocks[s] + gs > nb_max) s_blocks_bad = 1;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 3: page grants in call order (exclusive scan per class) -------
+  for (int cc = 0; cc < 3; ++cc) {
+    int carry = 0;
+    for (int base = 0; base < R; base += kAssignThreads) {
+      int r = base + tid;
+      int g = r < R ? ws.runs[r].grants[cc] : 0;
+      int total;
+      int excl = block_exclusive_scan(g, sh, &total);
+      if (r < R) ws.runs[r].page_base[cc] = C.page_bump[cc] + carry + excl;
+      carry += total;
+    }
+    if (tid == 0) s_total[cc] = carry;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int err = 0;
+    if (s_blocks_bad) err = THINKV_ERR_OUT_OF_BLOCKS;
+    for (int cc = 0; cc < 3; ++cc)
+      if ((int64_t)C.page_bump[cc] + s_total[cc] > C.L.pool_pages[cc]) err = THINKV_ERR_OUT_OF_PAGES;
+    s_err = err;
+    if (err) set_status(C.status, err);
+  }
+  __syncthreads();
+  if (s_err != 0) return;
+
+  // ---- phase 4: slot assignment, warp per run ------------------------------
+  for (int r = warp; r < R; r += kAssignWarps) {
+    const RunInfo ri = ws.runs[r];
+    const int s = ri.seq;
+    uint64_t* table = C.block_table + (int64_t)s * nb_max;
+    int32_t* llist = C.live_list + (int64_t)s * nb_max;
+    int32_t* lidx = C.live_index + (int64_t)s * nb_max;
+    int F[3], tail[3], rank[3] = {0, 0, 0}, last_entry[3] = {-1, -1, -1};
+#pragma unroll
+    for (int cc = 0; cc < 3; ++cc) {
+      F[cc] = C.free_top[s * 3 + cc];
+      tail[cc] = C.fifo_tail[s * 3 + cc];
+    }
+    const int nb0 = C.num_blocks[s];
+    int grants = 0;
+    int nlive = C.num_live[s];
+    for (int base = ri.start; base < ri.start + ri.len; base += 32) {
+      const int i = base + lane;
+      const bool valid = i < ri.start + ri.len;
+      const int c = valid ? tag[i] : 0;
+      unsigned bal[3], gbal_c[3];
+#pragma unroll
+      for (int cc = 0; cc < 3; ++cc) bal[cc] = __ballot_sync(0xFFFFFFFFu, valid && c == cc);
+      const int k = rank[c] + __popc(bal[c] & lanemask_lt());
+      const bool is_pop = valid && k < F[c];
+      const int kp = k - F[c];
+      const int j = kp >> 4, slot_new = kp & 15;
+      const bool is_grant = valid && !is_pop && slot_new == 0;
+#pragma unroll
+      for (int cc = 0; cc < 3; ++cc) gbal_c[cc] = __ballot_sync(0xFFFFFFFFu, is_grant && c == cc);
+      const unsigned gbal = gbal_c[0] | gbal_c[1] | gbal_c[2];
+      const int entry_grant = nb0 + grants + __popc(gbal & lanemask_lt());
+      // the entry of my new page: the last grant of my class at or before me
+      const unsigned mine = gbal_c[c] & (lanemask_lt() | (1u << lane));
+      const int src = mine ? 31 - __clz(mine) : lane;
+      const int entry_from = __shfl_sync(0xFFFFFFFFu, entry_grant, src);
+      int entry = 0, slot = 0;
+      uint32_t page = 0;
+      if (valid) {
+        if (is_pop) {
+          int32_t ts = C.free_slots[((int64_t)s * 3 + c) * cap + (F[c] - 1 - k)];
+          entry = ts >> 4;
+          slot = ts & 15;
+          page = entry_page(table[entry]);
+        } else {
+          entry = mine ? entry_from : last_entry[c];
+          slot = slot_new;
+          page = (uint32_t)(ri.page_base[c] + j);
+        }
+      }
+      // live-list candidates: granted entries, and reused entries with no live token
+      bool cand = false;
+      if (valid) cand = is_grant || (is_pop && lidx[entry] == -1);
+      const int key = cand ? entry : -1 - lane;
+      const unsigned grp = __match_any_sync(0xFFFFFFFFu, key);
+      const bool adder = cand && (__ffs(grp) - 1) == lane;
+      const unsigned abal = __ballot_sync(0xFFFFFFFFu, adder);
+      if (adder) {
+        int at = nlive + __popc(abal & lanemask_lt());
+        llist[at] = entry;
+        lidx[entry] = at;
+      }
+      nlive += __popc(abal);
+      if (valid) {
+        const int64_t sp = (int64_t)page * kPage;
+        if (is_grant) {
+          int used = min(kPage, ri.cnt[c] - F[c] - (j << 4));
+          uint32_t mask = (used >= 16) ? 0xFFFFu : ((1u << used) - 1u);
+          table[entry] = make_entry(page, c, mask);
+          for (int sl = used; sl < kPage; ++sl) C.slot_pos[c][sp + sl] = -1;
+        } else if (is_pop) {
+          atomicOr(reinterpret_cast<unsigned long long*>(&table[entry]),
+                   (unsigned long long)(1ull << (48 + slot)));
+        }
+        C.slot_pos[c][sp + slot] = pos[i];
+        C.fifo[((int64_t)s * 3 + c) * cap + ((int64_t)tail[c] + k) % cap] = entry * kPage + slot;
+        ws.tok_slot[i] = (int32_t)(sp + slot);
+      }
+#pragma unroll
+      for (int cc = 0; cc < 3; ++cc) {
+        rank[cc] += __popc(bal[cc]);
+        if (gbal_c[cc]) last_entry[cc] = __shfl_sync(0xFFFFFFFFu, entry_grant, 31 - __clz(gbal_c[cc]));
+      }
+      grants += __popc(gbal);
+      __syncwarp();
+    }
+    // final free stacks, FIFO tails and counters
+#pragma unroll
+    for (int cc = 0; cc < 3; ++cc) {
+      int32_t* stack = C.free_slots + ((int64_t)s * 3 + cc) * cap;
+      int cnt = ri.cnt[cc];
+      int top;
+      if (cnt <= F[cc]) {
+        top = F[cc] - cnt;
+      } else {
+        int over = cnt - F[cc];
+        int u_last = over - (((over - 1) >> 4) << 4);  // slots used in the last new page
+        top = kPage - u_last;
+        for (int x = lane; x < top; x += 32) stack[x] = last_entry[cc] * kPage + (kPage - 1 - x);
+      }
+      if (lane == 0) {
+        C.free_top[s * 3 + cc] = top;
+        C.fifo_tail[s * 3 + cc] = tail[cc] + cnt;
+      }
+    }
+    if (lane == 0) {
+      C.num_blocks[s] = nb0 + grants;
+      C.num_live[s] = nlive;
+      C.live_count[s] += ri.len;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int cc = 0; cc < 3; ++cc) C.page_bump[cc] += s_total[cc];
+    __threadfence();
+    *ws.ok = 1;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// quantise + scatter: one warp per (token, kv-head, K|V)
+// ---------------------------------------------------------------------------
+template <int D>
+struct ScatterSmem {
+  uint16_t code[D];  // codes (b <= 8) or raw fp16 bits (b == 16)
+};
+
+template <int D, int G>
+__device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int h, int kv,
+                             const uint16_t* __restrict__ x, uint16_t* code_sm) {
+  constexpr int PER = D / 32;          // channels per lane
+  constexpr int LPG = G / PER;         // lanes per group
+  constexpr int NG = D / G;
+  const int lane = threadIdx.x & 31;
+  const int b = C.L.bits[c];
+  const uint32_t page = pool_slot >> 4, slot = pool_slot & 15;
+  const int64_t phb = page_head_bytes(D, G, b);
+  uint8_t* blk = C.pool[c] + ((int64_t)page * C.L.num_kv_heads + h) * phb;
+
+  // load this lane's channels
+  uint16_t raw[PER];
+  if constexpr (PER == 4) {
+    uint2 v = *reinterpret_cast<const uint2*>(x + lane * 4);
+    raw[0] = v.x & 0xFFFF; raw[1] = v.x >> 16; raw[2] = v.y & 0xFFFF; raw[3] = v.y >> 16;
+  } else {
+    uint32_t v = *reinterpret_cast<const uint32_t*>(x + lane * 2);
+    raw[0] = v & 0xFFFF; raw[1] = v >> 16;
+  }
+  if (b == 16) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) code_sm[lane * PER + e] = raw[e];
+  } else {
+    float xf[PER], mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      xf[e] = __half2float(__ushort_as_half(raw[e]));
+      mn = fminf(mn, xf[e]);
+      mx = fmaxf(mx, xf[e]);
+    }
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    }
+    const __half zh = __float2half_rd(mn);
+    const float zf = __half2float(zh);
+    const float levels = (float)((1 << b) - 1);
+    const float s32 = __fdiv_rn(__fsub_rn(mx, zf), levels);
+    const __half sh = __float2half_ru(s32);
+    const float sf = __half2float(sh);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      int cq = 0;
+      if (sf != 0.0f) {
+        float t = __fdiv_rn(__fsub_rn(xf[e], zf), sf);
+        float r = rintf(t);
+        r = fminf(fmaxf(r, 0.0f), levels);
+        cq = (int)r;
+      }
+      code_sm[lane * PER + e] = (uint16_t)cq;
+    }
+    const int grp = (lane * PER) / G;
+    if ((lane % LPG) == 0) {
+      uint16_t* prm = reinterpret_cast<uint16_t*>(blk + 4LL * D * b + (kv ? 64LL * NG : 0));
+      uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+      *reinterpret_cast<uint32_t*>(prm + (slot * NG + grp) * 2) = pair;
+    }
+  }
+  __syncwarp();
+
+  const int64_t lane_bytes = (int64_t)D * b / 16;
+  uint8_t* region = blk + (kv ? 2LL * D * b : 0);
+  if (kv == 0) {
+    // K: pieces (layout lane 4*(slot%8)+t, group gr, r = slot/8) of G/4 channels
+    const int pb = G * b / 32;                 // piece bytes (>= 2)
+    const int m = min(32 / b, G / 4);          // channels per word (or per 16-bit piece)
+    if (b == 16 && lane < 4 * NG) {
+      // raw fp16: the piece is G/4 channels in natural order
+      const int t = lane & 3, gr = lane >> 2;
+      const int l = 4 * (slot & 7) + t, r = slot >> 3;
+      uint8_t* dst = region + l * lane_bytes + (int64_t)(gr * 2 + r) * pb;
+      const uint16_t* src = code_sm + gr * G + t * (G / 4);
+      for (int e = 0; e < G / 4; e += 2)
+        *reinterpret_cast<uint32_t*>(dst + 2 * e) = (uint32_t)src[e] | ((uint32_t)src[e + 1] << 16);
+    } else if (lane < 4 * NG) {
+      const int t = lane & 3, gr = lane >> 2;
+      const int l = 4 * (slot & 7) + t, r = slot >> 3;
+      uint32_t words[4] = {0, 0, 0, 0};
+      for (int e = 0; e < G / 4; ++e) {
+        const uint32_t v = code_sm[gr * G + t * (G / 4) + e];
+        const int wi = e / m, el = e % m;
+        const int p = (el & 1) ? (m / 2 + el / 2) : (el / 2);
+        words[wi] |= v << (p * b);
+      }
+      uint8_t* dst = region + l * lane_bytes + (int64_t)(gr * 2 + r) * pb;
+      if (pb == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)words[0];
+      else if (pb == 4) *reinterpret_cast<uint32_t*>(dst) = words[0];
+      else if (pb == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+    }
+  } else {
+    // V: half-words (lane 4*g + t, P, q, half) holding 16/b codes each
+    const int t = (slot & 7) >> 1, P = slot >> 3, half = slot & 1;
+    const int Q = D * b / 128;                 // chunks per P
+    const int per = 16 / b;                    // codes per half-word
+    for (int u = lane; u < 8 * Q; u += 32) {
+      const int g = u / Q, q = u % Q;
+      uint32_t hw = 0;
+      for (int k = 0; k < per; ++k) {
+        const int e = q * per + k;
+        const int ch = 16 * (e >> 1) + g + 8 * (e & 1);
+        hw |= (uint32_t)code_sm[ch] << (b * k);
+      }
+      const int l = 4 * g + t;
+      uint8_t* dst = region + l * lane_bytes + (int64_t)(P * Q + q) * 4 + 2 * half;
+      *reinterpret_cast<uint16_t*>(dst) = (uint16_t)hw;
+    }
+  }
+  __syncwarp();
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(256)
+    append_scatter_kernel(CacheView C, int32_t n, const uint8_t* __restrict__ tag,
+                          const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+                          AppendWorkspace ws) {
+  __shared__ ScatterSmem<D> sm[8];
+  if (*ws.ok == 0) return;
+  const int warp = threadIdx.x >> 5;
+  const int H = C.L.num_kv_heads;
+  const int64_t units = (int64_t)n * H * 2;
+  for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += (int64_t)gridDim.x * 8) {
+    const int kv = (int)(u & 1);
+    const int64_t th = u >> 1;
+    const int h = (int)(th % H);
+    const int64_t i = th / H;
+    const int c = tag[i];
+    const uint16_t* x = (kv ? v : k) + (i * H + h) * D;
+    scatter_unit<D, G>(C, c, (uint32_t)ws.tok_slot[i], h, kv, x, sm[warp].code);
+  }
+}
+
+}  // namespace
+
+size_t append_workspace_bytes(int32_t n) {
+  size_t bytes = 256;                                   // ok flag
+  bytes += ((size_t)n * sizeof(int32_t) + 255) / 256 * 256;
+  bytes += ((size_t)(n > 0 ? n : 1) * sizeof(RunInfo) + 255) / 256 * 256;
+  return bytes;
+}
+
+AppendWorkspace carve_append_workspace(void* ws, int32_t n) {
+  AppendWorkspace w;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  w.ok = reinterpret_cast<int32_t*>(p);
+  p += 256;
+  w.tok_slot = reinterpret_cast<int32_t*>(p);
+  p += ((size_t)n * sizeof(int32_t) + 255) / 256 * 256;
+  w.runs = reinterpret_cast<RunInfo*>(p);
+  return w;
+}
+
+cudaError_t launch_append(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* pos,
+                          const uint8_t* tag, const uint16_t* k, const uint16_t* v,
+                          const AppendWorkspace& ws, cudaStream_t stream, int num_sms) {
+  const size_t seen_bytes = (size_t)((C.L.max_seqs + 31) / 32) * 4;
+  append_assign_kernel<<<1, kAssignThreads, seen_bytes, stream>>>(C, n, seq, pos, tag, ws);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t units = (int64_t)n * C.L.num_kv_heads * 2;
+  int64_t blocks = (units + 7) / 8;
+  const int64_t cap = (int64_t)num_sms * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const int D = C.L.head_dim, G = C.L.group_size;
+  if (D == 128 && G == 64) append_scatter_kernel<128, 64><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
+  else if (D == 128 && G == 32) append_scatter_kernel<128, 32><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
+  else if (D == 64 && G == 64) append_scatter_kernel<64, 64><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
+  else append_scatter_kernel<64, 32><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace thinkv

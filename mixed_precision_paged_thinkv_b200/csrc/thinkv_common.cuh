@@ -1,0 +1,147 @@
+// thinkv_common.cuh -- shared device helpers of libthinkv (sm_100a).
+//
+// Layout arithmetic for the page-head blocks declared in include/thinkv.h,
+// the sticky status word, and thin wrappers over the PTX this library uses:
+// mbarrier + cp.async.bulk (the TMA bulk-copy engine) and mma.sync m16n8k16.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "thinkv.h"
+
+namespace thinkv {
+
+constexpr int kPage = 16;
+
+// ---------------------------------------------------------------------------
+// geometry
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int64_t page_head_bytes(int d, int G, int b) {
+  // K codes + V codes (2*d*b each) + K/V params (64 bytes per group each)
+  if (b == 16) return 64LL * d;
+  return 4LL * d * b + 128LL * (d / G);
+}
+
+// Table entry fields.
+__host__ __device__ inline uint32_t entry_page(uint64_t e) { return (uint32_t)(e & 0xFFFFFFFFull); }
+__host__ __device__ inline int entry_class(uint64_t e) { return (int)((e >> 32) & 0xFF); }
+__host__ __device__ inline uint32_t entry_mask(uint64_t e) { return (uint32_t)(e >> 48); }
+__host__ __device__ inline uint64_t make_entry(uint32_t page, int cls, uint32_t mask) {
+  return (uint64_t)page | ((uint64_t)cls << 32) | ((uint64_t)mask << 48);
+}
+
+// ---------------------------------------------------------------------------
+// sticky status: the first error wins
+// ---------------------------------------------------------------------------
+__device__ inline void set_status(int32_t* status, int32_t code) {
+  atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ inline uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ inline void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ inline void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+// One bounded probe of phase `parity`; true once the phase has completed.
+__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` with an iteration bound; false if the bound ran out.
+constexpr uint32_t kWaitLimit = 1u << 22;
+__device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Bulk copy (TMA engine, no tensor map, no multicast) global -> shared,
+// completing `bytes` of transaction count on `bar`.  dst, src 16-byte
+// aligned; bytes a multiple of 16.
+__device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// D = A * B + C, m16n8k16, fp16 inputs, fp32 accumulate.
+__device__ inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 2^x on the SFU (PTX ex2.approx; relative error about 2^-22).
+__device__ inline float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// half2 bit pattern of (lo, hi) fp32 values, each rounded to nearest.
+__device__ inline uint32_t pack_half2_rn(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ inline uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// ---------------------------------------------------------------------------
+// code unpacking: element k of the low and of the high half-word of `w`
+// (b-bit codes, element k at bits [b*k, b*k+b) of its half) as the half2
+// (1024 + code_lo, 1024 + code_hi) -- exact, since fp16 has 10 mantissa bits.
+// ---------------------------------------------------------------------------
+template <int B>
+__device__ inline uint32_t unpack_pair(uint32_t w, int k) {
+  constexpr uint32_t m = (1u << B) - 1u;
+  return ((w >> (B * k)) & (m | (m << 16))) | 0x64006400u;
+}
+
+// fp16 pair (1024 + 2^(b-1), same): subtracting it centres a code pair.
+template <int B>
+__device__ inline uint32_t centre_bits() {
+  constexpr uint32_t h = 0x6400u + (1u << (B - 1));  // 1024 + 2^(b-1), exact in fp16
+  return h | (h << 16);
+}
+
+}  // namespace thinkv

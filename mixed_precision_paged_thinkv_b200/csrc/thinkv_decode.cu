@@ -1,0 +1,706 @@
+// thinkv_decode.cu -- decode attention over mixed-precision, slot-reusing pages.
+//
+// "ThinKV: Thought-Adaptive KV Cache Compression for Efficient Reasoning
+// Models": the arXiv abstract's kernel "that extends PagedAttention" to read a
+// cache whose tokens carry per-thought-type precision (explainer, Methodologie,
+// TBQ) and whose evicted slots are holes that are never compacted (explainer,
+// "Implementation Systeme: Pensee Continue (CT)").  The pages print no kernel
+// design; this one is written for sm_100a:
+//
+//   split kernel (stream-K): the live page-heads of all decoded sequences form
+//   one ordered list of units (sequence, kv-head, live page); every warp of the
+//   grid takes an equal contiguous share, so work is balanced by live pages no
+//   matter how lengths and budgets vary.  Per warp, lane 0 streams page-head
+//   blocks (K codes, V codes, params: one contiguous block per page and head)
+//   into a shared-memory ring with cp.async.bulk (TMA) + mbarriers; the warp
+//   unpacks codes straight into mma.sync m16n8k16 operands (fp16 magic-number
+//   conversion, codes centred by 2^(b-1) so products stay exact), computes
+//   q.k for the whole GQA group at once (tokens x heads), applies the per-group
+//   scale/zero in fp32, runs the online softmax, transposes p through a small
+//   shared buffer and accumulates p*scale (fp16, exponent-shifted) times the V
+//   codes on the tensor cores, with the zero terms summed in fp32.  Each warp
+//   writes one partial (m, l, o) per (sequence, kv-head) segment it touched.
+//   combine kernel: one warp per (sequence, q-head) merges the partials of its
+//   segment with the log-sum-exp rule, writes fp16 O and the top-k mass.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "thinkv_common.cuh"
+#include "thinkv_internal.h"
+
+namespace thinkv {
+
+namespace {
+
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kPbufStride = 12;                 // floats per row of the p transpose buffer
+constexpr int kPbufBytes = 16 * kPbufStride * 4;
+constexpr int kSigmaInit = 1 << 20;
+
+struct DecodeParams {
+  const uint8_t* pool[3];
+  int32_t phb[3];
+  int32_t bits[3];
+  const uint64_t* table;
+  const int32_t* live_list;
+  const int32_t* num_live;
+  int32_t max_blocks, max_seqs;
+  int32_t Hkv, Hq, Gq;
+  const int32_t* seq;
+  int32_t n;
+  const uint16_t* q;
+  float scale_log2;
+  float* part_o;   // [pieces][Gq][D]
+  float* part_ml;  // [pieces][Gq][2]   (m in log2 units, l)
+  int32_t* plan;   // [n + 1] exclusive prefix of live pages per decoded sequence
+  int32_t* status;
+  int32_t nstage, stage_bytes, warp_smem, plan_smem;
+};
+
+__device__ inline float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// Per-warp state of the (sequence, kv-head) segment being processed.
+template <int D, int G>
+struct SegState {
+  static constexpr int NG = D / G;
+  static constexpr int KS = G / 16;   // k-steps per group
+  static constexpr int MT = D / 16;   // m-tiles (16 channels) of the PV product
+  uint32_t qf[NG][KS][2];             // Q^T B-fragments (head = gid)
+  float qsum[NG][2];                  // per-group sum of q for heads 2t, 2t+1
+  float m[2], lp[2];                  // running max (log2 units), partial row sums
+  float z[NG][2];                     // zero-term accumulators (heads 2t, 2t+1)
+  float acc[MT][4];                   // PV accumulators, units of 2^-sigma[group]
+  int sigma[NG];
+};
+
+template <int D, int G>
+__device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i, int h) {
+  constexpr int NG = SegState<D, G>::NG, KS = SegState<D, G>::KS, MT = SegState<D, G>::MT;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const bool has = g < p.Gq;
+  const uint16_t* qrow = p.q + ((int64_t)i * p.Hq + h * p.Gq + (has ? g : 0)) * D;
+  float qs[NG];
+#pragma unroll
+  for (int gr = 0; gr < NG; ++gr) {
+    qs[gr] = 0.f;
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+      const uint16_t* qp = qrow + gr * G + t * (G / 4) + 4 * s;
+      uint2 v = has ? *reinterpret_cast<const uint2*>(qp) : make_uint2(0, 0);
+      S.qf[gr][s][0] = v.x;
+      S.qf[gr][s][1] = v.y;
+      __half2 a = *reinterpret_cast<__half2*>(&v.x), b = *reinterpret_cast<__half2*>(&v.y);
+      float2 fa = __half22float2(a), fb = __half22float2(b);
+      qs[gr] += (fa.x + fa.y) + (fb.x + fb.y);
+    }
+    qs[gr] += __shfl_xor_sync(0xFFFFFFFFu, qs[gr], 1);
+    qs[gr] += __shfl_xor_sync(0xFFFFFFFFu, qs[gr], 2);
+    S.qsum[gr][0] = __shfl_sync(0xFFFFFFFFu, qs[gr], 8 * t);
+    S.qsum[gr][1] = __shfl_sync(0xFFFFFFFFu, qs[gr], 8 * t + 4);
+    S.z[gr][0] = S.z[gr][1] = 0.f;
+    S.sigma[gr] = kSigmaInit;
+  }
+  S.m[0] = S.m[1] = -INFINITY;
+  S.lp[0] = S.lp[1] = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) S.acc[mt][0] = S.acc[mt][1] = S.acc[mt][2] = S.acc[mt][3] = 0.f;
+}
+
+template <int D, int G>
+__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t piece) {
+  constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    S.lp[0] += __shfl_xor_sync(0xFFFFFFFFu, S.lp[0], o);
+    S.lp[1] += __shfl_xor_sync(0xFFFFFFFFu, S.lp[1], o);
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr) {
+      S.z[gr][0] += __shfl_xor_sync(0xFFFFFFFFu, S.z[gr][0], o);
+      S.z[gr][1] += __shfl_xor_sync(0xFFFFFFFFu, S.z[gr][1], o);
+    }
+  }
+  const int Gq = p.Gq;
+  float* po = p.part_o + piece * Gq * D;
+  if (g == 0) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int hd = 2 * t + c;
+      if (hd < Gq) {
+        p.part_ml[(piece * Gq + hd) * 2 + 0] = S.m[c];
+        p.part_ml[(piece * Gq + hd) * 2 + 1] = S.lp[c];
+      }
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int gr = (mt * 16) / G;
+    const float inv = pow2i(-S.sigma[gr]);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int c = x & 1, ch = mt * 16 + g + 8 * (x >> 1), hd = 2 * t + c;
+      if (hd < Gq) po[hd * D + ch] = S.acc[mt][x] * inv + S.z[gr][c];
+    }
+  }
+}
+
+// One live page-head block (in shared memory) of a class with B-bit codes.
+template <int D, int G, int B>
+__device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
+                                 float scale_log2, float* pbuf) {
+  constexpr int NG = D / G, KS = G / 16, MT = D / 16;
+  constexpr int LANE_BYTES = D * B / 16;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const bool live0 = (mask >> g) & 1, live1 = (mask >> (g + 8)) & 1;
+
+  // ---------------- logits: S^T = K(codes) x Q^T, per group ----------------
+  float lg[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const uint8_t* kl = blk + lane * LANE_BYTES;
+    constexpr int PB = G * B / 32 > 0 ? G * B / 32 : 1;  // piece bytes
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr) {
+      // the two pieces (rows gid and gid+8) of this group
+      uint32_t w[2][PB >= 4 ? PB / 4 : 1];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint8_t* src = kl + (gr * 2 + r) * PB;
+        if constexpr (PB == 2) {
+          uint32_t h16 = *reinterpret_cast<const uint16_t*>(src);
+          w[r][0] = (h16 & 0xFFu) | ((h16 & 0xFF00u) << 8);  // bytes -> half-words
+        } else if constexpr (PB == 4) {
+          w[r][0] = *reinterpret_cast<const uint32_t*>(src);
+        } else if constexpr (PB == 8) {
+          uint2 v = *reinterpret_cast<const uint2*>(src);
+          w[r][0] = v.x; w[r][1] = v.y;
+        } else {
+#pragma unroll
+          for (int x = 0; x < PB / 16; ++x) {
+            uint4 v = *reinterpret_cast<const uint4*>(src + 16 * x);
+            w[r][4 * x] = v.x; w[r][4 * x + 1] = v.y; w[r][4 * x + 2] = v.z; w[r][4 * x + 3] = v.w;
+          }
+        }
+      }
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        uint32_t a[4];
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int u = 2 * s + hi;  // pair index inside the piece
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            uint32_t reg;
+            if constexpr (B == 16) {
+              reg = w[r][u];
+            } else {
+              constexpr int PAIRS = (PB == 2 ? 4 : 16 / B);  // pairs per (spread) word
+              reg = hsub2_bits(unpack_pair<B>(w[r][u / PAIRS], u % PAIRS), centre_bits<B>());
+            }
+            a[hi * 2 + r] = reg;
+          }
+        }
+        mma_16816(c, a, S.qf[gr][s][0], S.qf[gr][s][1]);
+      }
+      if constexpr (B == 16) {
+        lg[0] += c[0]; lg[1] += c[1]; lg[2] += c[2]; lg[3] += c[3];
+      } else {
+        const uint16_t* kp = reinterpret_cast<const uint16_t*>(blk + 4 * D * B);
+        const uint32_t p0 = *reinterpret_cast<const uint32_t*>(kp + (g * NG + gr) * 2);
+        const uint32_t p1 = *reinterpret_cast<const uint32_t*>(kp + ((g + 8) * NG + gr) * 2);
+        const float s0 = __half2float(__ushort_as_half(p0 & 0xFFFF));
+        const float z0 = __half2float(__ushort_as_half(p0 >> 16));
+        const float s1 = __half2float(__ushort_as_half(p1 & 0xFFFF));
+        const float z1 = __half2float(__ushort_as_half(p1 >> 16));
+        const float zc0 = fmaf((float)(1 << (B - 1)), s0, z0);
+        const float zc1 = fmaf((float)(1 << (B - 1)), s1, z1);
+        lg[0] += fmaf(s0, c[0], zc0 * S.qsum[gr][0]);
+        lg[1] += fmaf(s0, c[1], zc0 * S.qsum[gr][1]);
+        lg[2] += fmaf(s1, c[2], zc1 * S.qsum[gr][0]);
+        lg[3] += fmaf(s1, c[3], zc1 * S.qsum[gr][1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < 4; ++x) lg[x] *= scale_log2;
+  if (!live0) lg[0] = lg[1] = -INFINITY;
+  if (!live1) lg[2] = lg[3] = -INFINITY;
+
+  // ---------------- online softmax (heads 2t, 2t+1) ----------------
+  float pm0 = fmaxf(lg[0], lg[2]), pm1 = fmaxf(lg[1], lg[3]);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    pm0 = fmaxf(pm0, __shfl_xor_sync(0xFFFFFFFFu, pm0, o));
+    pm1 = fmaxf(pm1, __shfl_xor_sync(0xFFFFFFFFu, pm1, o));
+  }
+  const float mn0 = fmaxf(S.m[0], pm0), mn1 = fmaxf(S.m[1], pm1);
+  const float a0 = exp2_approx(S.m[0] - mn0), a1 = exp2_approx(S.m[1] - mn1);
+  S.m[0] = mn0;
+  S.m[1] = mn1;
+  float pr[4];
+  pr[0] = exp2_approx(lg[0] - mn0);
+  pr[1] = exp2_approx(lg[1] - mn1);
+  pr[2] = exp2_approx(lg[2] - mn0);
+  pr[3] = exp2_approx(lg[3] - mn1);
+  S.lp[0] = fmaf(S.lp[0], a0, pr[0] + pr[2]);
+  S.lp[1] = fmaf(S.lp[1], a1, pr[1] + pr[3]);
+
+  const uint16_t* vpar = reinterpret_cast<const uint16_t*>(blk + 4 * D * B + 64 * NG);
+  if constexpr (B != 16) {
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr) {
+      const uint32_t p0 = *reinterpret_cast<const uint32_t*>(vpar + (g * NG + gr) * 2);
+      const uint32_t p1 = *reinterpret_cast<const uint32_t*>(vpar + ((g + 8) * NG + gr) * 2);
+      float zv0 = fmaf((float)(1 << (B - 1)), __half2float(__ushort_as_half(p0 & 0xFFFF)),
+                       __half2float(__ushort_as_half(p0 >> 16)));
+      float zv1 = fmaf((float)(1 << (B - 1)), __half2float(__ushort_as_half(p1 & 0xFFFF)),
+                       __half2float(__ushort_as_half(p1 >> 16)));
+      zv0 = live0 ? zv0 : 0.f;
+      zv1 = live1 ? zv1 : 0.f;
+      S.z[gr][0] = fmaf(S.z[gr][0], a0, fmaf(pr[0], zv0, pr[2] * zv1));
+      S.z[gr][1] = fmaf(S.z[gr][1], a1, fmaf(pr[1], zv0, pr[3] * zv1));
+    }
+  }
+
+  // ---------------- p transpose: (tokens gid, gid+8 ; heads 2t, 2t+1) ->
+  //                  (tokens 2t, 2t+1, 2t+8, 2t+9 ; head gid) ----------------
+  *reinterpret_cast<float2*>(pbuf + g * kPbufStride + 2 * t) = make_float2(pr[0], pr[1]);
+  *reinterpret_cast<float2*>(pbuf + (g + 8) * kPbufStride + 2 * t) = make_float2(pr[2], pr[3]);
+  __syncwarp();
+  float pt[4];
+  pt[0] = pbuf[(2 * t) * kPbufStride + g];
+  pt[1] = pbuf[(2 * t + 1) * kPbufStride + g];
+  pt[2] = pbuf[(2 * t + 8) * kPbufStride + g];
+  pt[3] = pbuf[(2 * t + 9) * kPbufStride + g];
+  const int tok[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+  bool tl[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) tl[j] = (mask >> tok[j]) & 1;
+
+  // ---------------- per-group B fragments W = p * s_V * 2^sigma ----------------
+  uint32_t wf[NG][2];
+  float fac[NG];
+  bool rescale = (a0 != 1.f) || (a1 != 1.f);
+#pragma unroll
+  for (int gr = 0; gr < NG; ++gr) {
+    float sv[4];
+    int e5 = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if constexpr (B == 16) {
+        sv[j] = 1.f;
+        e5 = 15;
+      } else {
+        const uint16_t sb = vpar[(tok[j] * NG + gr) * 2];
+        sv[j] = __half2float(__ushort_as_half(sb));
+        const int ef = max((int)((sb >> 10) & 31), 1);
+        e5 = tl[j] ? max(e5, ef) : e5;
+      }
+    }
+    if constexpr (B != 16) {
+      e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 1));
+      e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 2));
+    }
+    const int sp = 29 - e5;  // s * 2^sp < 2^15, so p * s * 2^sigma fits in fp16
+    fac[gr] = 1.f;
+    if (sp < S.sigma[gr]) {
+      if (S.sigma[gr] != kSigmaInit) {
+        fac[gr] = pow2i(sp - S.sigma[gr]);
+        rescale = true;
+      }
+      S.sigma[gr] = sp;
+    }
+    const float f = pow2i(S.sigma[gr]);
+    float wv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wv[j] = tl[j] ? pt[j] * sv[j] * f : 0.f;
+    wf[gr][0] = pack_half2_rn(wv[0], wv[1]);
+    wf[gr][1] = pack_half2_rn(wv[2], wv[3]);
+  }
+  if (__any_sync(0xFFFFFFFFu, rescale)) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const float f = fac[(mt * 16) / G];
+      S.acc[mt][0] *= a0 * f;
+      S.acc[mt][1] *= a1 * f;
+      S.acc[mt][2] *= a0 * f;
+      S.acc[mt][3] *= a1 * f;
+    }
+  }
+
+  // ---------------- O^T += V^T(codes) x W ----------------
+  {
+    constexpr int Q = D * B / 128 > 0 ? D * B / 128 : 1;  // words per token pair
+    constexpr int PER = 16 / B;                          // codes per half-word
+    const uint32_t* vw = reinterpret_cast<const uint32_t*>(blk + 2 * D * B + lane * LANE_BYTES);
+    uint32_t vr[2 * Q];
+#pragma unroll
+    for (int x = 0; x < (2 * Q) / 4; ++x) {
+      uint4 v = reinterpret_cast<const uint4*>(vw)[x];
+      vr[4 * x] = v.x; vr[4 * x + 1] = v.y; vr[4 * x + 2] = v.z; vr[4 * x + 3] = v.w;
+    }
+    if constexpr ((2 * Q) % 4 == 2) {
+      uint2 v = reinterpret_cast<const uint2*>(vw)[(2 * Q) / 2 - 1];
+      vr[2 * Q - 2] = v.x; vr[2 * Q - 1] = v.y;
+    }
+    uint32_t dead_mask[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+    if constexpr (B == 16) {
+      dead_mask[0] = (tl[0] ? 0xFFFFu : 0u) | (tl[1] ? 0xFFFF0000u : 0u);
+      dead_mask[1] = (tl[2] ? 0xFFFFu : 0u) | (tl[3] ? 0xFFFF0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int gr = (mt * 16) / G;
+      uint32_t a[4];
+#pragma unroll
+      for (int P = 0; P < 2; ++P) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int e = 2 * mt + r;
+          uint32_t reg;
+          if constexpr (B == 16) {
+            reg = vr[P * Q + e] & dead_mask[P];
+          } else {
+            reg = hsub2_bits(unpack_pair<B>(vr[P * Q + e / PER], e % PER), centre_bits<B>());
+          }
+          a[P * 2 + r] = reg;
+        }
+      }
+      mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
+    }
+  }
+}
+
+template <int D, int G>
+__device__ inline void page_dispatch(SegState<D, G>& S, const uint8_t* blk, int bits, uint32_t mask,
+                                     float scale_log2, float* pbuf) {
+  switch (bits) {
+    case 8: page_step<D, G, 8>(S, blk, mask, scale_log2, pbuf); break;
+    case 4: page_step<D, G, 4>(S, blk, mask, scale_log2, pbuf); break;
+    case 2: page_step<D, G, 2>(S, blk, mask, scale_log2, pbuf); break;
+    default: page_step<D, G, 16>(S, blk, mask, scale_log2, pbuf); break;
+  }
+}
+
+// Everything a lane needs to know about one unit (sequence, kv-head, live page).
+struct UnitMeta {
+  const uint8_t* src;
+  int32_t seg;       // i * Hkv + h
+  int32_t i;         // index into the call's sequences
+  int32_t h;
+  uint32_t cls_mask; // class << 16 | live mask
+};
+
+__device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P, int64_t u,
+                                        int64_t U1) {
+  UnitMeta m;
+  m.src = nullptr;
+  m.seg = -1;
+  m.i = 0;
+  m.h = 0;
+  m.cls_mask = 0;
+  if (u >= U1) return m;
+  int lo = 0, hi = p.n;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)P[mid] * p.Hkv <= u) lo = mid; else hi = mid;
+  }
+  const int i = lo;
+  const int nl = P[i + 1] - P[i];
+  const int64_t rel = u - (int64_t)P[i] * p.Hkv;
+  const int h = (int)(rel / nl), j = (int)(rel % nl);
+  const int s = p.seq[i];
+  const int e = p.live_list[(int64_t)s * p.max_blocks + j];
+  const uint64_t ent = p.table[(int64_t)s * p.max_blocks + e];
+  const int cls = entry_class(ent);
+  m.src = p.pool[cls] + ((int64_t)entry_page(ent) * p.Hkv + h) * p.phb[cls];
+  m.seg = i * p.Hkv + h;
+  m.i = i;
+  m.h = h;
+  m.cls_mask = ((uint32_t)cls << 16) | entry_mask(ent);
+  return m;
+}
+
+__device__ inline UnitMeta shfl_meta(const UnitMeta& m, int src) {
+  UnitMeta r;
+  r.src = reinterpret_cast<const uint8_t*>(
+      __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(m.src), src));
+  r.seg = __shfl_sync(0xFFFFFFFFu, m.seg, src);
+  r.i = __shfl_sync(0xFFFFFFFFu, m.i, src);
+  r.h = __shfl_sync(0xFFFFFFFFu, m.h, src);
+  r.cls_mask = __shfl_sync(0xFFFFFFFFu, m.cls_mask, src);
+  return r;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecThreads)
+    decode_split_kernel(DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int32_t* P = reinterpret_cast<int32_t*>(smem);
+
+  // ---- prefix of live pages over the call's sequences (per CTA) ----
+  {
+    __shared__ int wsum[kDecWarps];
+    int carry = 0;
+    for (int base = 0; base < p.n; base += kDecThreads) {
+      const int i = base + tid;
+      int v = 0;
+      if (i < p.n) {
+        const int s = p.seq[i];
+        if (s >= 0 && s < p.max_seqs) v = p.num_live[s];
+        else if (blockIdx.x == 0) set_status(p.status, THINKV_ERR_INVALID);  // decoded as empty
+      }
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) wsum[warp] = x;
+      __syncthreads();
+      int before = carry;
+      for (int w = 0; w < warp; ++w) before += wsum[w];
+      if (i < p.n) P[i] = before + x - v;
+      int tot = 0;
+      for (int w = 0; w < kDecWarps; ++w) tot += wsum[w];
+      carry += tot;
+      __syncthreads();
+    }
+    if (tid == 0) P[p.n] = carry;
+    __syncthreads();
+    if (blockIdx.x == 0)
+      for (int i = tid; i <= p.n; i += kDecThreads) p.plan[i] = P[i];
+  }
+
+  const int64_t T = (int64_t)P[p.n] * p.Hkv;
+  const int64_t W = (int64_t)gridDim.x * kDecWarps;
+  const int64_t w = (int64_t)blockIdx.x * kDecWarps + warp;
+  const int64_t U0 = w * T / W, U1 = (w + 1) * T / W;
+  if (U0 >= U1) return;
+
+  uint8_t* wsm = smem + p.plan_smem + warp * p.warp_smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + p.nstage * p.stage_bytes);
+  float* pbuf = reinterpret_cast<float*>(wsm + p.nstage * p.stage_bytes + 64);
+  if (lane == 0) {
+    for (int s = 0; s < p.nstage; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  UnitMeta cur = resolve_unit(p, P, U0 + lane, U1);
+  UnitMeta nxt = resolve_unit(p, P, U0 + 32 + lane, U1);
+
+  // prologue: fill the ring
+  const int64_t nunits = U1 - U0;
+  for (int s = 0; s < p.nstage && s < nunits; ++s) {
+    const UnitMeta m = shfl_meta(cur, s);  // nstage <= 8 < 32
+    if (lane == 0) {
+      const uint32_t bytes = (uint32_t)p.phb[m.cls_mask >> 16];
+      mbar_arrive_expect_tx(&bars[s], bytes);
+      bulk_g2s(wsm + s * p.stage_bytes, m.src, bytes, &bars[s]);
+    }
+  }
+
+  SegState<D, G> S;
+  int seg = -1;
+  for (int64_t k = 0; k < nunits; ++k) {
+    const int kk = (int)(k & 31);
+    if (kk == 0 && k > 0) {
+      cur = nxt;
+      nxt = resolve_unit(p, P, U0 + k + 32 + lane, U1);
+    }
+    const UnitMeta m = shfl_meta(cur, kk);
+    if (m.seg != seg) {
+      if (seg >= 0) seg_end<D, G>(S, p, w + seg);
+      seg = m.seg;
+      seg_begin<D, G>(S, p, m.i, m.h);
+    }
+    const int stage = (int)(k % p.nstage);
+    const uint32_t parity = (uint32_t)((k / p.nstage) & 1);
+    if (!mbar_wait_bounded(&bars[stage], parity)) {
+      if (lane == 0) set_status(p.status, THINKV_ERR_TIMEOUT);
+      // drain the copies still in flight (bounded), then leave
+      for (int64_t k2 = k + 1; k2 < nunits && k2 < k + p.nstage; ++k2)
+        mbar_wait_bounded(&bars[k2 % p.nstage], (uint32_t)((k2 / p.nstage) & 1));
+      return;
+    }
+    const int cls = (int)(m.cls_mask >> 16);
+    page_dispatch<D, G>(S, wsm + stage * p.stage_bytes, p.bits[cls], m.cls_mask & 0xFFFFu,
+                        p.scale_log2, pbuf);
+    __syncwarp();
+    // refill this stage with unit k + nstage
+    const int64_t kn = k + p.nstage;
+    const int srcl = (int)(kn & 31);
+    const UnitMeta ma = shfl_meta(cur, srcl);
+    const UnitMeta mb = shfl_meta(nxt, srcl);
+    const UnitMeta& mn = ((kn >> 5) == (k >> 5)) ? ma : mb;
+    if (lane == 0 && kn < nunits) {
+      fence_proxy_async_smem();
+      const uint32_t bytes = (uint32_t)p.phb[mn.cls_mask >> 16];
+      mbar_arrive_expect_tx(&bars[stage], bytes);
+      bulk_g2s(wsm + stage * p.stage_bytes, mn.src, bytes, &bars[stage]);
+    }
+  }
+  if (seg >= 0) seg_end<D, G>(S, p, w + seg);
+}
+
+// ---------------------------------------------------------------------------
+// combine: one warp per (sequence, q-head)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128)
+    decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                          const int32_t* __restrict__ plan, int32_t n, int32_t Hq, int32_t Hkv,
+                          int32_t Gq, int64_t W, uint16_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (gw >= (int64_t)n * Hq) return;
+  const int i = (int)(gw / Hq), hq = (int)(gw % Hq), h = hq / Gq, r = hq % Gq;
+  constexpr int PER = D / 32;
+  uint16_t* o = out + gw * D + lane * PER;
+  const int Pi = plan[i], nl = plan[i + 1] - Pi;
+  if (nl == 0) {
+#pragma unroll
+    for (int x = 0; x < PER; ++x) o[x] = 0;
+    return;
+  }
+  const int64_t T = (int64_t)plan[n] * Hkv;
+  const int64_t Us = (int64_t)Pi * Hkv + (int64_t)h * nl, Ue = Us + nl;
+  const int64_t w0 = ((Us + 1) * W - 1) / T, w1 = (Ue * W - 1) / T;
+  const int64_t seg = (int64_t)i * Hkv + h;
+  float M = -INFINITY;
+  for (int64_t w = w0; w <= w1; ++w) M = fmaxf(M, part_ml[((w + seg) * Gq + r) * 2]);
+  float L = 0.f, acc[PER];
+#pragma unroll
+  for (int x = 0; x < PER; ++x) acc[x] = 0.f;
+  for (int64_t w = w0; w <= w1; ++w) {
+    const int64_t pc = (w + seg) * Gq + r;
+    const float f = exp2_approx(part_ml[pc * 2] - M);
+    L = fmaf(part_ml[pc * 2 + 1], f, L);
+    const float* po = part_o + pc * D + lane * PER;
+#pragma unroll
+    for (int x = 0; x < PER; ++x) acc[x] = fmaf(po[x], f, acc[x]);
+  }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int x = 0; x < PER; ++x) o[x] = __half_as_ushort(__float2half_rn(acc[x] * inv));
+}
+
+template <int D, int G>
+cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  decode_split_kernel<D, G><<<dl.grid, kDecThreads, dl.smem_bytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+int plan_smem_bytes(int32_t n) { return ((n + 1) * 4 + 127) / 128 * 128; }
+
+}  // namespace
+
+bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, DecodeLaunch* out) {
+  const int D = L.head_dim, G = L.group_size;
+  int64_t maxphb = 0;
+  for (int c = 0; c < 3; ++c) {
+    int64_t b = page_head_bytes(D, G, L.bits[c]);
+    if (b > maxphb) maxphb = b;
+  }
+  const int stage_bytes = (int)((maxphb + 127) / 128 * 128);
+  int nstage = (int)(18432 / stage_bytes);
+  if (nstage < 2) nstage = 2;
+  if (nstage > 8) nstage = 8;
+  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes;
+  const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)kDecWarps * warp_smem;
+  if (smem > 227 * 1024) return false;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return false;
+  int smem_per_sm = 0;
+  if (cudaDeviceGetAttribute(&smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
+      cudaSuccess)
+    return false;
+  // CTAs per SM limited by shared memory (1 KB reserved per CTA) and threads
+  int per_sm = smem_per_sm / (int)(smem + 1024);
+  if (per_sm > 16) per_sm = 16;
+  if (per_sm < 1) per_sm = 1;
+  out->grid = sms * per_sm;
+  out->warps_per_cta = kDecWarps;
+  out->nstage = nstage;
+  out->stage_bytes = stage_bytes;
+  out->smem_bytes = smem;
+  out->pieces = (int64_t)out->grid * kDecWarps + (int64_t)n_seqs * L.num_kv_heads;
+  return true;
+}
+
+size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
+                              const DecodeLaunch& dl) {
+  (void)topk;
+  const int Gq = L.num_q_heads / L.num_kv_heads;
+  size_t b = ((size_t)(n_seqs + 1) * 4 + 255) / 256 * 256;
+  b += ((size_t)dl.pieces * Gq * 2 * 4 + 255) / 256 * 256;
+  b += ((size_t)dl.pieces * Gq * L.head_dim * 4 + 255) / 256 * 256;
+  return b;
+}
+
+cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, const uint16_t* q,
+                          uint16_t* out, float* mass, int32_t topk, float softmax_scale,
+                          void* ws, const DecodeLaunch& dl, cudaStream_t stream) {
+  (void)mass;
+  (void)topk;
+  const thinkv_layout& L = C.L;
+  const int D = L.head_dim, G = L.group_size;
+  DecodeParams p;
+  for (int c = 0; c < 3; ++c) {
+    p.pool[c] = C.pool[c];
+    p.phb[c] = (int32_t)page_head_bytes(D, G, L.bits[c]);
+    p.bits[c] = L.bits[c];
+  }
+  p.table = C.block_table;
+  p.live_list = C.live_list;
+  p.num_live = C.num_live;
+  p.max_blocks = L.max_blocks_per_seq;
+  p.max_seqs = L.max_seqs;
+  p.Hkv = L.num_kv_heads;
+  p.Hq = L.num_q_heads;
+  p.Gq = L.num_q_heads / L.num_kv_heads;
+  p.seq = seq;
+  p.n = n;
+  p.q = q;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.plan = reinterpret_cast<int32_t*>(w);
+  w += ((size_t)(n + 1) * 4 + 255) / 256 * 256;
+  p.part_ml = reinterpret_cast<float*>(w);
+  w += ((size_t)dl.pieces * p.Gq * 2 * 4 + 255) / 256 * 256;
+  p.part_o = reinterpret_cast<float*>(w);
+  p.status = C.status;
+  p.nstage = dl.nstage;
+  p.stage_bytes = dl.stage_bytes;
+  p.warp_smem = dl.nstage * dl.stage_bytes + 64 + kPbufBytes;
+  p.plan_smem = plan_smem_bytes(n);
+  cudaError_t e;
+  if (D == 128 && G == 64) e = launch_split<128, 64>(p, dl, stream);
+  else if (D == 128 && G == 32) e = launch_split<128, 32>(p, dl, stream);
+  else if (D == 64 && G == 64) e = launch_split<64, 64>(p, dl, stream);
+  else e = launch_split<64, 32>(p, dl, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t warps = (int64_t)n * L.num_q_heads;
+  const int blocks = (int)((warps + 3) / 4);
+  const int64_t W = (int64_t)dl.grid * kDecWarps;
+  if (D == 128)
+    decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(p.part_o, p.part_ml, p.plan, n, p.Hq,
+                                                          p.Hkv, p.Gq, W, out);
+  else
+    decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(p.part_o, p.part_ml, p.plan, n, p.Hq,
+                                                         p.Hkv, p.Gq, W, out);
+  return cudaGetLastError();
+}
+
+}  // namespace thinkv

@@ -1,0 +1,72 @@
+// thinkv_internal.h -- host/device structures shared by the libthinkv sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "thinkv.h"
+
+namespace thinkv {
+
+// The cache as kernels see it (passed by value).
+struct CacheView {
+  thinkv_layout L;
+  uint8_t* pool[3];
+  int32_t* slot_pos[3];
+  uint64_t* block_table;
+  int32_t* num_blocks;
+  int32_t* free_slots;
+  int32_t* free_top;
+  int32_t* fifo;
+  int32_t* fifo_head;
+  int32_t* fifo_tail;
+  int32_t* live_count;
+  int32_t* live_list;
+  int32_t* live_index;
+  int32_t* num_live;
+  int32_t* page_bump;
+  int32_t* status;
+};
+
+// One sequence run of an append call (slot-assignment scratch).
+struct RunInfo {
+  int32_t start, len, seq, pad;
+  int32_t cnt[3];
+  int32_t grants[3];
+  int32_t page_base[3];
+  int32_t pad2;
+};
+
+struct AppendWorkspace {
+  int32_t* ok;        // 1 once the slot assignment succeeded
+  int32_t* tok_slot;  // [n] pool slot id (page*16 + slot) of every token
+  RunInfo* runs;      // [n] sequence runs
+};
+
+size_t append_workspace_bytes(int32_t n);
+AppendWorkspace carve_append_workspace(void* ws, int32_t n);
+cudaError_t launch_append(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* pos,
+                          const uint8_t* tag, const uint16_t* k, const uint16_t* v,
+                          const AppendWorkspace& ws, cudaStream_t stream, int num_sms);
+
+cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
+                         const uint8_t order[3], cudaStream_t stream);
+
+// decode
+struct DecodeLaunch {
+  int grid;            // CTAs of the split kernel
+  int warps_per_cta;
+  int nstage;          // pipeline stages per warp
+  int stage_bytes;     // bytes per stage
+  size_t smem_bytes;   // dynamic shared memory of the split kernel
+  int64_t pieces;      // partial slots
+};
+bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, DecodeLaunch* out);
+size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
+                              const DecodeLaunch& dl);
+cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, const uint16_t* q,
+                          uint16_t* out, float* mass, int32_t topk, float softmax_scale,
+                          void* ws, const DecodeLaunch& dl, cudaStream_t stream);
+
+}  // namespace thinkv

@@ -1,0 +1,92 @@
+"""Drive a synthetic workload's schedule on a ThinKVCache (GPU).
+
+The schedule (prefill appends in calls of <= 4096 positions per sequence, one
+evict to budget, optional appends and churn steps) comes from ``workloads``;
+this module only turns it into library calls.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import workloads as W
+from .binding import ThinKVCache
+
+
+def geometry(w: W.Workload, sched: W.Schedule) -> dict:
+    """Pool and table sizes that can never run out for this schedule.
+
+    Pages are never released, so (sequence, class) needs at most
+    ceil(tokens of that class ever appended / 16) pages.
+    """
+    pool = [0, 0, 0]
+    max_blocks = 1
+    for s in range(w.batch):
+        tags = sched.tags(s)
+        cnt = np.bincount(tags, minlength=3)
+        pages = [int(math.ceil(int(cnt[c]) / 16)) for c in range(3)]
+        for c in range(3):
+            pool[c] += pages[c]
+        max_blocks = max(max_blocks, sum(pages))
+    return {"pool_pages": [max(1, p) for p in pool], "max_blocks_per_seq": max_blocks,
+            "max_seqs": w.batch}
+
+
+def to_dev(a, dtype, device):
+    return torch.as_tensor(np.ascontiguousarray(a)).to(device=device, dtype=dtype)
+
+
+class WorkloadRun:
+    """A cache plus the bookkeeping of how many tokens each sequence generated."""
+
+    def __init__(self, w: W.Workload, extra: int = 0, device: str = "cuda",
+                 bits: Optional[tuple] = None):
+        self.w = w
+        self.sched = W.Schedule(w, extra)
+        self.geom = geometry(w, self.sched)
+        self.device = torch.device(device)
+        self.cache = ThinKVCache(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size,
+                                 bits or w.bits, self.geom["max_seqs"],
+                                 self.geom["max_blocks_per_seq"], self.geom["pool_pages"],
+                                 device=device)
+        self.generated = self.sched.lengths.astype(np.int64).copy()
+        self.all_seqs = torch.arange(w.batch, dtype=torch.int32, device=self.device)
+
+    # -- single operations --
+    def append_call(self, call: W.AppendCall):
+        k, v = W.call_kv(self.w, call, device=self.device)
+        self.cache.append(to_dev(call.seqs, torch.int32, self.device),
+                          to_dev(call.pos, torch.int32, self.device),
+                          to_dev(call.tags, torch.uint8, self.device), k, v)
+
+    def evict_all(self):
+        b = self.sched.budgets(self.generated)
+        self.cache.evict(self.all_seqs, to_dev(b, torch.int32, self.device))
+
+    def decode(self, step: int, topk: Optional[int] = None):
+        q = W.q_values(self.w, step, device=self.device)
+        return self.cache.decode(self.all_seqs, q, topk=topk)
+
+    # -- schedule --
+    def setup(self):
+        for call in self.sched.prefill_calls():
+            self.append_call(call)
+        self.evict_all()
+        post = self.sched.post_evict_call()
+        if post is not None:
+            self.append_call(post)
+            self.generated += self.w.post_evict_append
+        for _ in range(self.w.churn_steps):
+            self.churn_step(decode=False)
+
+    def churn_step(self, decode: bool = False, step: int = 0, topk: Optional[int] = None):
+        call = self.sched.one_token_call(self.generated)
+        self.append_call(call)
+        self.generated += 1
+        self.evict_all()
+        if decode:
+            return self.decode(step, topk)
+        return None

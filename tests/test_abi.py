@@ -1,0 +1,118 @@
+"""The C ABI library loads, exports every entry point include/thinkv.h
+declares, and its host-only functions behave (no GPU needed)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixed_precision_paged_thinkv_b200 import build, binding
+    build.build()
+    return binding.lib()
+
+
+def _declared():
+    hdr = open(os.path.join(ROOT, "include", "thinkv.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    return sorted(set(re.findall(r"\b(thinkv_[a-z_]+)\s*\(", hdr)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from mixed_precision_paged_thinkv_b200 import binding
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert set(declared) == set(binding.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (thinkv_\w+)", out))
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    # nothing else leaks out of the library under the thinkv_ prefix
+    assert exported == set(declared)
+
+
+def _layout(**kw):
+    from mixed_precision_paged_thinkv_b200 import binding
+    a = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, group_size=64, bits=(8, 4, 2),
+             max_seqs=16, max_blocks_per_seq=100, pool_pages=(10, 20, 30))
+    a.update(kw)
+    return binding.make_layout(**a)
+
+
+def test_layout_check_and_sizes(lib):
+    L = _layout()
+    assert lib.thinkv_layout_check(C.byref(L)) == 0
+    d, G = 128, 64
+    for c, b in enumerate((8, 4, 2)):
+        assert lib.thinkv_page_head_bytes(C.byref(L), c) == 4 * d * b + 128 * (d // G)
+    assert lib.thinkv_page_head_bytes(C.byref(L), 0) == 4352
+    assert lib.thinkv_buffer_bytes(C.byref(L), 0) == 10 * 8 * 4352
+    assert lib.thinkv_buffer_bytes(C.byref(L), 6) == 16 * 100 * 8      # block table
+    assert lib.thinkv_buffer_bytes(C.byref(L), 8) == 16 * 3 * 1600 * 4  # free slots
+    assert lib.thinkv_buffer_bytes(C.byref(L), 18) == 4
+    assert lib.thinkv_buffer_bytes(C.byref(L), 19) == 0
+    L16 = _layout(bits=(16, 16, 16))
+    assert lib.thinkv_page_head_bytes(C.byref(L16), 2) == 64 * d
+    for bad in (dict(head_dim=96), dict(group_size=16), dict(bits=(8, 3, 2)),
+                dict(num_q_heads=36), dict(num_q_heads=72, num_kv_heads=8),
+                dict(max_seqs=0), dict(max_seqs=70000), dict(pool_pages=(-1, 0, 0))):
+        Lb = _layout(**bad)
+        assert lib.thinkv_layout_check(C.byref(Lb)) == 1, bad
+        assert lib.thinkv_buffer_bytes(C.byref(Lb), 0) == 0
+
+
+def test_host_validation_without_launch(lib):
+    """Bad arguments are rejected before anything reaches the GPU."""
+    from mixed_precision_paged_thinkv_b200 import binding
+    cs = binding.CacheStruct()
+    cs.L = _layout()
+    # null buffers -> invalid, no CUDA call made
+    assert lib.thinkv_cache_reset(C.byref(cs), None) == 1
+    assert lib.thinkv_append_quantize(C.byref(cs), 4, None, None, None, None, None, None, 0, None) == 1
+    assert lib.thinkv_evict(C.byref(cs), 1, None, None, None, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, None, None, None, None, 0, 0.0, None, 0, None) == 1
+    # a cache struct whose pointers are non-null but bad sizes/orders
+    fake = C.c_void_p(16)
+    for name, _ in binding.CacheStruct._fields_[1:]:
+        v = getattr(cs, name)
+        if isinstance(v, C.Array):
+            for i in range(3):
+                v[i] = 16
+        else:
+            setattr(cs, name, 16)
+    assert lib.thinkv_append_quantize(C.byref(cs), -1, fake, fake, fake, fake, fake, fake, 10 ** 6, None) == 1
+    assert lib.thinkv_append_quantize(C.byref(cs), 0, None, None, None, None, None, None, 0, None) == 0
+    assert lib.thinkv_append_quantize(C.byref(cs), 8, fake, fake, fake, fake, fake, fake, 8, None) == 6
+    bad_order = (C.c_uint8 * 3)(2, 2, 0)
+    assert lib.thinkv_evict(C.byref(cs), 1, fake, fake, C.cast(bad_order, C.c_void_p), None) == 1
+    assert lib.thinkv_evict(C.byref(cs), 0, None, None, None, None) == 0
+    assert lib.thinkv_decode_attention(C.byref(cs), 0, fake, fake, fake, None, 0, 0.0, fake, 1, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, fake, fake, fake, fake, 65, 0.0, fake, 1, None) == 1
+    assert lib.thinkv_append_workspace_bytes(C.byref(cs.L), 1000) >= 1000 * 4
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.thinkv_status_string(code)
+    assert lib.thinkv_status_string(99) == b"unknown status"
+
+
+def test_layout_decoder_is_a_bijection():
+    """The test-side layout decoder maps every (slot, channel) to its own bits."""
+    from layout_decode import _maps
+    for d, G in ((64, 32), (128, 64), (128, 32), (64, 64)):
+        for b in (2, 4, 8, 16):
+            kb, ks, vb, vs = _maps(d, G, b)
+            w = 16 if b == 16 else b
+            for bo, sh, lo in ((kb, ks, 0), (vb, vs, 2 * d * b if b < 16 else 32 * d)):
+                bits = (bo - lo) * 8 + sh
+                assert bits.min() == 0 and bits.max() == 16 * d * w - w
+                assert len(np.unique(bits)) == 16 * d
+                assert np.all(bits % w == 0)
