@@ -5,6 +5,8 @@
 // thinkv_evict.cu and thinkv_decode.cu.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "thinkv.h"
@@ -79,7 +81,11 @@ int num_sms_current() {
   return cached[dev];
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? THINKV_OK : THINKV_ERR_CUDA; }
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return THINKV_OK;
+  if (getenv("THINKV_VERBOSE")) fprintf(stderr, "libthinkv: %s\n", cudaGetErrorString(e));
+  return THINKV_ERR_CUDA;
+}
 
 }  // namespace
 

@@ -570,12 +570,18 @@ __global__ void __launch_bounds__(128)
   const int64_t Us = (int64_t)Pi * Hkv + (int64_t)h * nl, Ue = Us + nl;
   const int64_t w0 = ((Us + 1) * W - 1) / T, w1 = (Ue * W - 1) / T;
   const int64_t seg = (int64_t)i * Hkv + h;
+  // warps whose unit range is empty (possible when there are fewer units than
+  // warps) wrote no partial
   float M = -INFINITY;
-  for (int64_t w = w0; w <= w1; ++w) M = fmaxf(M, part_ml[((w + seg) * Gq + r) * 2]);
+  for (int64_t w = w0; w <= w1; ++w) {
+    if (w * T / W == (w + 1) * T / W) continue;
+    M = fmaxf(M, part_ml[((w + seg) * Gq + r) * 2]);
+  }
   float L = 0.f, acc[PER];
 #pragma unroll
   for (int x = 0; x < PER; ++x) acc[x] = 0.f;
   for (int64_t w = w0; w <= w1; ++w) {
+    if (w * T / W == (w + 1) * T / W) continue;
     const int64_t pc = (w + seg) * Gq + r;
     const float f = exp2_approx(part_ml[pc * 2] - M);
     L = fmaf(part_ml[pc * 2 + 1], f, L);
@@ -590,12 +596,17 @@ __global__ void __launch_bounds__(128)
 
 template <int D, int G>
 cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  // raise the dynamic shared-memory limit of this instantiation once per device
+  static size_t configured[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (dl.smem_bytes > configured[dev]) {
+    e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dl.smem_bytes);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev] = dl.smem_bytes;
   }
   decode_split_kernel<D, G><<<dl.grid, kDecThreads, dl.smem_bytes, stream>>>(p);
   return cudaGetLastError();
@@ -618,7 +629,10 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, Deco
   if (nstage > 8) nstage = 8;
   const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes;
   const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)kDecWarps * warp_smem;
-  if (smem > 227 * 1024) return false;
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
+    return false;
+  if (smem + 1024 > (size_t)optin) return false;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return false;
   int smem_per_sm = 0;
