@@ -199,7 +199,7 @@ size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t n_seqs, int
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   DecodeLaunch dl;
-  if (!plan_decode_launch(*L, n_seqs, dev, &dl)) return 0;
+  if (!plan_decode_launch(*L, n_seqs, topk, dev, &dl)) return 0;
   return decode_workspace_bytes(*L, n_seqs, topk, dl);
 }
 
@@ -213,7 +213,7 @@ int thinkv_decode_attention(const thinkv_cache* C, int32_t n, const int32_t* seq
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return THINKV_ERR_CUDA;
   DecodeLaunch dl;
-  if (!plan_decode_launch(C->L, n, dev, &dl)) return THINKV_ERR_INVALID;
+  if (!plan_decode_launch(C->L, n, topk_mass ? topk : 0, dev, &dl)) return THINKV_ERR_INVALID;
   if (!workspace || workspace_bytes < decode_workspace_bytes(C->L, n, topk_mass ? topk : 0, dl))
     return THINKV_ERR_WORKSPACE;
   return cuda_status(launch_decode(view_of(C), n, seq, q, out, topk_mass, topk_mass ? topk : 0,

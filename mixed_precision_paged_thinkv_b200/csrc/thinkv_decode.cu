@@ -37,6 +37,8 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kPbufStride = 12;                 // floats per row of the p transpose buffer
 constexpr int kPbufBytes = 16 * kPbufStride * 4;
 constexpr int kSigmaInit = 1 << 20;
+constexpr int kCandCap = 128;                   // top-k candidate slots per head
+constexpr int kTopkHdrBytes = 64;               // per-head counts and thresholds
 
 struct DecodeParams {
   const uint8_t* pool[3];
@@ -54,11 +56,79 @@ struct DecodeParams {
   float* part_o;   // [pieces][Gq][D]
   float* part_ml;  // [pieces][Gq][2]   (m in log2 units, l)
   int32_t* plan;   // [n + 1] exclusive prefix of live pages per decoded sequence
+  float* part_topk;  // [pieces][Gq][topk] largest logits (log2 units), -inf padded
+  int32_t topk;
   int32_t* status;
   int32_t nstage, stage_bytes, warp_smem, plan_smem;
 };
 
 __device__ inline float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// ---------------------------------------------------------------------------
+// top-k attention mass: candidate buffers
+// ---------------------------------------------------------------------------
+// Sorts 128 values held 4 per lane (element lane*4 + j) into descending order
+// (bitonic network; exchanges across lanes use shuffles).
+__device__ inline void bitonic128_desc(float (&v)[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 128; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = lane * 4 + j;
+          const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], stride >> 2);
+          const bool desc = (i & size) == 0, lower = (i & stride) == 0;
+          v[j] = (lower == desc) ? fmaxf(v[j], o) : fminf(v[j], o);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j & stride) continue;
+          const int i = lane * 4 + j;
+          const bool desc = (i & size) == 0;
+          const float a = v[j], b = v[j | stride];
+          v[j] = desc ? fmaxf(a, b) : fminf(a, b);
+          v[j | stride] = desc ? fminf(a, b) : fmaxf(a, b);
+        }
+      }
+    }
+  }
+}
+
+struct TopkCtx {
+  float* cand;    // [Gq][kCandCap]
+  int* cnt;       // [Gq]
+  float* theta;   // [Gq]  values <= theta cannot enter the top-k any more
+  int topk;
+};
+
+// Keeps the topk largest candidates of head h and raises its threshold.
+__device__ inline void cand_compact(const TopkCtx& tk, int h) {
+  const int lane = threadIdx.x & 31;
+  float* c = tk.cand + h * kCandCap;
+  const int n = tk.cnt[h];
+  float v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = (lane * 4 + j < n) ? c[lane * 4 + j] : -INFINITY;
+  bitonic128_desc(v);
+  __syncwarp();
+  const int keep = min(n, tk.topk);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (lane * 4 + j < keep) c[lane * 4 + j] = v[j];
+  const int kl = tk.topk - 1;
+  const float sel = (kl & 3) == 0 ? v[0] : (kl & 3) == 1 ? v[1] : (kl & 3) == 2 ? v[2] : v[3];
+  const float kth = __shfl_sync(0xFFFFFFFFu, sel, kl >> 2);
+  __syncwarp();
+  if (lane == 0) {
+    tk.cnt[h] = keep;
+    if (n >= tk.topk) tk.theta[h] = kth;
+  }
+  __syncwarp();
+}
 
 // Per-warp state of the (sequence, kv-head) segment being processed.
 template <int D, int G>
@@ -75,7 +145,8 @@ struct SegState {
 };
 
 template <int D, int G>
-__device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i, int h) {
+__device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i, int h,
+                                 const TopkCtx& tk) {
   constexpr int NG = SegState<D, G>::NG, KS = SegState<D, G>::KS, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const bool has = g < p.Gq;
@@ -105,10 +176,18 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i
   S.lp[0] = S.lp[1] = 0.f;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) S.acc[mt][0] = S.acc[mt][1] = S.acc[mt][2] = S.acc[mt][3] = 0.f;
+  if (tk.topk > 0) {
+    if (lane < p.Gq) {
+      tk.cnt[lane] = 0;
+      tk.theta[lane] = -INFINITY;
+    }
+    __syncwarp();
+  }
 }
 
 template <int D, int G>
-__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t piece) {
+__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t piece,
+                               const TopkCtx& tk) {
   constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -143,12 +222,21 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
       if (hd < Gq) po[hd * D + ch] = S.acc[mt][x] * inv + S.z[gr][c];
     }
   }
+  if (tk.topk > 0) {
+    for (int hd = 0; hd < Gq; ++hd) {
+      if (tk.cnt[hd] > tk.topk) cand_compact(tk, hd);
+      const int n = tk.cnt[hd];
+      float* dst = p.part_topk + (piece * Gq + hd) * tk.topk;
+      for (int j = lane; j < tk.topk; j += 32) dst[j] = j < n ? tk.cand[hd * kCandCap + j] : -INFINITY;
+    }
+    __syncwarp();
+  }
 }
 
 // One live page-head block (in shared memory) of a class with B-bit codes.
 template <int D, int G, int B>
 __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
-                                 float scale_log2, float* pbuf) {
+                                 float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
   constexpr int NG = D / G, KS = G / 16, MT = D / 16;
   constexpr int LANE_BYTES = D * B / 16;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -226,6 +314,25 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   for (int x = 0; x < 4; ++x) lg[x] *= scale_log2;
   if (!live0) lg[0] = lg[1] = -INFINITY;
   if (!live1) lg[2] = lg[3] = -INFINITY;
+
+  // ---------------- top-k candidates (logits above the head's threshold) ----------------
+  if (tk.topk > 0) {
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int hd = 2 * t + (x & 1);
+      if (hd < Gq && lg[x] > tk.theta[hd]) {
+        const int at = atomicAdd(&tk.cnt[hd], 1);
+        tk.cand[hd * kCandCap + at] = lg[x];
+      }
+    }
+    __syncwarp();
+    // a head whose buffer could overflow on the next page is cut back to its top-k
+    unsigned full = __ballot_sync(0xFFFFFFFFu, lane < Gq && tk.cnt[lane] > kCandCap - 16);
+    while (full) {
+      cand_compact(tk, __ffs(full) - 1);
+      full &= full - 1;
+    }
+  }
 
   // ---------------- online softmax (heads 2t, 2t+1) ----------------
   float pm0 = fmaxf(lg[0], lg[2]), pm1 = fmaxf(lg[1], lg[3]);
@@ -374,12 +481,12 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
 
 template <int D, int G>
 __device__ inline void page_dispatch(SegState<D, G>& S, const uint8_t* blk, int bits, uint32_t mask,
-                                     float scale_log2, float* pbuf) {
+                                     float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
   switch (bits) {
-    case 8: page_step<D, G, 8>(S, blk, mask, scale_log2, pbuf); break;
-    case 4: page_step<D, G, 4>(S, blk, mask, scale_log2, pbuf); break;
-    case 2: page_step<D, G, 2>(S, blk, mask, scale_log2, pbuf); break;
-    default: page_step<D, G, 16>(S, blk, mask, scale_log2, pbuf); break;
+    case 8: page_step<D, G, 8>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 4: page_step<D, G, 4>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 2: page_step<D, G, 2>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    default: page_step<D, G, 16>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
   }
 }
 
@@ -483,6 +590,14 @@ __global__ void __launch_bounds__(kDecThreads)
   uint8_t* wsm = smem + p.plan_smem + warp * p.warp_smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + p.nstage * p.stage_bytes);
   float* pbuf = reinterpret_cast<float*>(wsm + p.nstage * p.stage_bytes + 64);
+  TopkCtx tk;
+  {
+    uint8_t* tb = wsm + p.nstage * p.stage_bytes + 64 + kPbufBytes;
+    tk.cnt = reinterpret_cast<int*>(tb);
+    tk.theta = reinterpret_cast<float*>(tb + 32);
+    tk.cand = reinterpret_cast<float*>(tb + kTopkHdrBytes);
+    tk.topk = p.topk;
+  }
   if (lane == 0) {
     for (int s = 0; s < p.nstage; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
@@ -513,9 +628,9 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     const UnitMeta m = shfl_meta(cur, kk);
     if (m.seg != seg) {
-      if (seg >= 0) seg_end<D, G>(S, p, w + seg);
+      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk);
       seg = m.seg;
-      seg_begin<D, G>(S, p, m.i, m.h);
+      seg_begin<D, G>(S, p, m.i, m.h, tk);
     }
     const int stage = (int)(k % p.nstage);
     const uint32_t parity = (uint32_t)((k / p.nstage) & 1);
@@ -528,7 +643,7 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     const int cls = (int)(m.cls_mask >> 16);
     page_dispatch<D, G>(S, wsm + stage * p.stage_bytes, p.bits[cls], m.cls_mask & 0xFFFFu,
-                        p.scale_log2, pbuf);
+                        p.scale_log2, pbuf, tk, p.Gq);
     __syncwarp();
     // refill this stage with unit k + nstage
     const int64_t kn = k + p.nstage;
@@ -543,30 +658,43 @@ __global__ void __launch_bounds__(kDecThreads)
       bulk_g2s(wsm + stage * p.stage_bytes, mn.src, bytes, &bars[stage]);
     }
   }
-  if (seg >= 0) seg_end<D, G>(S, p, w + seg);
+  if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk);
 }
 
 // ---------------------------------------------------------------------------
 // combine: one warp per (sequence, q-head)
 // ---------------------------------------------------------------------------
+struct CombineParams {
+  const float* part_o;
+  const float* part_ml;
+  const float* part_topk;
+  const int32_t* plan;
+  const int32_t* seq;
+  const int32_t* live_count;
+  int32_t n, Hq, Hkv, Gq, topk;
+  int64_t W;
+  uint16_t* out;
+  float* mass;
+};
+
 template <int D>
-__global__ void __launch_bounds__(128)
-    decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                          const int32_t* __restrict__ plan, int32_t n, int32_t Hq, int32_t Hkv,
-                          int32_t Gq, int64_t W, uint16_t* __restrict__ out) {
+__global__ void __launch_bounds__(128) decode_combine_kernel(CombineParams c) {
   const int lane = threadIdx.x & 31;
   const int64_t gw = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (gw >= (int64_t)n * Hq) return;
-  const int i = (int)(gw / Hq), hq = (int)(gw % Hq), h = hq / Gq, r = hq % Gq;
+  if (gw >= (int64_t)c.n * c.Hq) return;
+  const int Hkv = c.Hkv, Gq = c.Gq;
+  const int i = (int)(gw / c.Hq), hq = (int)(gw % c.Hq), h = hq / Gq, r = hq % Gq;
   constexpr int PER = D / 32;
-  uint16_t* o = out + gw * D + lane * PER;
-  const int Pi = plan[i], nl = plan[i + 1] - Pi;
+  uint16_t* o = c.out + gw * D + lane * PER;
+  const int Pi = c.plan[i], nl = c.plan[i + 1] - Pi;
   if (nl == 0) {
 #pragma unroll
     for (int x = 0; x < PER; ++x) o[x] = 0;
+    if (c.mass && lane == 0) c.mass[gw] = 0.f;
     return;
   }
-  const int64_t T = (int64_t)plan[n] * Hkv;
+  const int64_t W = c.W;
+  const int64_t T = (int64_t)c.plan[c.n] * Hkv;
   const int64_t Us = (int64_t)Pi * Hkv + (int64_t)h * nl, Ue = Us + nl;
   const int64_t w0 = ((Us + 1) * W - 1) / T, w1 = (Ue * W - 1) / T;
   const int64_t seg = (int64_t)i * Hkv + h;
@@ -575,7 +703,7 @@ __global__ void __launch_bounds__(128)
   float M = -INFINITY;
   for (int64_t w = w0; w <= w1; ++w) {
     if (w * T / W == (w + 1) * T / W) continue;
-    M = fmaxf(M, part_ml[((w + seg) * Gq + r) * 2]);
+    M = fmaxf(M, c.part_ml[((w + seg) * Gq + r) * 2]);
   }
   float L = 0.f, acc[PER];
 #pragma unroll
@@ -583,15 +711,45 @@ __global__ void __launch_bounds__(128)
   for (int64_t w = w0; w <= w1; ++w) {
     if (w * T / W == (w + 1) * T / W) continue;
     const int64_t pc = (w + seg) * Gq + r;
-    const float f = exp2_approx(part_ml[pc * 2] - M);
-    L = fmaf(part_ml[pc * 2 + 1], f, L);
-    const float* po = part_o + pc * D + lane * PER;
+    const float f = exp2_approx(c.part_ml[pc * 2] - M);
+    L = fmaf(c.part_ml[pc * 2 + 1], f, L);
+    const float* po = c.part_o + pc * D + lane * PER;
 #pragma unroll
     for (int x = 0; x < PER; ++x) acc[x] = fmaf(po[x], f, acc[x]);
   }
   const float inv = 1.f / L;
 #pragma unroll
   for (int x = 0; x < PER; ++x) o[x] = __half_as_ushort(__float2half_rn(acc[x] * inv));
+
+  if (c.mass) {
+    const int k = c.topk;
+    const int nlive = c.live_count[c.seq[i]];
+    if (nlive <= k) {
+      if (lane == 0) c.mass[gw] = 1.f;
+      return;
+    }
+    // top-k of the union of the pieces' top-k lists: merge piece by piece
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = -INFINITY;
+    for (int64_t w = w0; w <= w1; ++w) {
+      if (w * T / W == (w + 1) * T / W) continue;
+      const float* src = c.part_topk + ((w + seg) * Gq + r) * k;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = lane * 4 + j;
+        if (e >= k) v[j] = (e < 2 * k) ? src[e - k] : -INFINITY;
+      }
+      bitonic128_desc(v);
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (lane * 4 + j < k) sum += exp2_approx(v[j] - M);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+    if (lane == 0) c.mass[gw] = sum * inv;
+  }
 }
 
 template <int D, int G>
@@ -616,7 +774,8 @@ int plan_smem_bytes(int32_t n) { return ((n + 1) * 4 + 127) / 128 * 128; }
 
 }  // namespace
 
-bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, DecodeLaunch* out) {
+bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, int device,
+                        DecodeLaunch* out) {
   const int D = L.head_dim, G = L.group_size;
   int64_t maxphb = 0;
   for (int c = 0; c < 3; ++c) {
@@ -627,7 +786,9 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, Deco
   int nstage = (int)(18432 / stage_bytes);
   if (nstage < 2) nstage = 2;
   if (nstage > 8) nstage = 8;
-  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes;
+  const int Gq = L.num_q_heads / L.num_kv_heads;
+  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes +
+                        (topk > 0 ? kTopkHdrBytes + Gq * kCandCap * 4 : 0);
   const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)kDecWarps * warp_smem;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
@@ -648,25 +809,24 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, Deco
   out->nstage = nstage;
   out->stage_bytes = stage_bytes;
   out->smem_bytes = smem;
+  out->warp_smem = warp_smem;
   out->pieces = (int64_t)out->grid * kDecWarps + (int64_t)n_seqs * L.num_kv_heads;
   return true;
 }
 
 size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
                               const DecodeLaunch& dl) {
-  (void)topk;
   const int Gq = L.num_q_heads / L.num_kv_heads;
   size_t b = ((size_t)(n_seqs + 1) * 4 + 255) / 256 * 256;
   b += ((size_t)dl.pieces * Gq * 2 * 4 + 255) / 256 * 256;
   b += ((size_t)dl.pieces * Gq * L.head_dim * 4 + 255) / 256 * 256;
+  b += ((size_t)dl.pieces * Gq * (topk > 0 ? topk : 0) * 4 + 255) / 256 * 256;
   return b;
 }
 
 cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, const uint16_t* q,
                           uint16_t* out, float* mass, int32_t topk, float softmax_scale,
                           void* ws, const DecodeLaunch& dl, cudaStream_t stream) {
-  (void)mass;
-  (void)topk;
   const thinkv_layout& L = C.L;
   const int D = L.head_dim, G = L.group_size;
   DecodeParams p;
@@ -694,10 +854,13 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   p.part_ml = reinterpret_cast<float*>(w);
   w += ((size_t)dl.pieces * p.Gq * 2 * 4 + 255) / 256 * 256;
   p.part_o = reinterpret_cast<float*>(w);
+  w += ((size_t)dl.pieces * p.Gq * D * 4 + 255) / 256 * 256;
+  p.part_topk = reinterpret_cast<float*>(w);
+  p.topk = mass ? topk : 0;
   p.status = C.status;
   p.nstage = dl.nstage;
   p.stage_bytes = dl.stage_bytes;
-  p.warp_smem = dl.nstage * dl.stage_bytes + 64 + kPbufBytes;
+  p.warp_smem = dl.warp_smem;
   p.plan_smem = plan_smem_bytes(n);
   cudaError_t e;
   if (D == 128 && G == 64) e = launch_split<128, 64>(p, dl, stream);
@@ -707,13 +870,23 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   if (e != cudaSuccess) return e;
   const int64_t warps = (int64_t)n * L.num_q_heads;
   const int blocks = (int)((warps + 3) / 4);
-  const int64_t W = (int64_t)dl.grid * kDecWarps;
-  if (D == 128)
-    decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(p.part_o, p.part_ml, p.plan, n, p.Hq,
-                                                          p.Hkv, p.Gq, W, out);
-  else
-    decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(p.part_o, p.part_ml, p.plan, n, p.Hq,
-                                                         p.Hkv, p.Gq, W, out);
+  CombineParams cp;
+  cp.part_o = p.part_o;
+  cp.part_ml = p.part_ml;
+  cp.part_topk = p.part_topk;
+  cp.plan = p.plan;
+  cp.seq = seq;
+  cp.live_count = C.live_count;
+  cp.n = n;
+  cp.Hq = p.Hq;
+  cp.Hkv = p.Hkv;
+  cp.Gq = p.Gq;
+  cp.topk = p.topk;
+  cp.W = (int64_t)dl.grid * kDecWarps;
+  cp.out = out;
+  cp.mass = p.topk > 0 ? mass : nullptr;
+  if (D == 128) decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(cp);
+  else decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(cp);
   return cudaGetLastError();
 }
 

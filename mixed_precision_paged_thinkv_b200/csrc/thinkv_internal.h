@@ -60,9 +60,11 @@ struct DecodeLaunch {
   int nstage;          // pipeline stages per warp
   int stage_bytes;     // bytes per stage
   size_t smem_bytes;   // dynamic shared memory of the split kernel
+  int warp_smem;       // bytes of shared memory per warp
   int64_t pieces;      // partial slots
 };
-bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int device, DecodeLaunch* out);
+bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, int device,
+                        DecodeLaunch* out);
 size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
                               const DecodeLaunch& dl);
 cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, const uint16_t* q,

@@ -54,7 +54,7 @@ def test_tiny_workload():
     g, o = _pair(w)
     g.setup()
     o.setup()
-    _check_all(g, o)
+    _check_all(g, o, topk=8)
 
 
 @pytest.mark.parametrize("name,batch,length", [
@@ -78,11 +78,12 @@ def test_reduced_configs(name, batch, length):
     g, o = _pair(w, extra=40)
     g.setup()
     o.setup()
-    _check_all(g, o, step=0)
+    k = w.topk or 16
+    _check_all(g, o, step=0, topk=k)
     for step in range(1, 4):
         g.churn_step()
         o.churn_step()
-        _check_all(g, o, step=step, codes=(step == 3))
+        _check_all(g, o, step=step, topk=k, codes=(step == 3))
 
 
 @pytest.mark.parametrize("bits", [(16, 16, 16), (8, 8, 8), (2, 4, 8), (16, 4, 2), (4, 2, 16)])
@@ -94,10 +95,10 @@ def test_bit_widths_and_shapes(bits, d, G):
     g, o = _pair(w, extra=10, bits=bits)
     g.setup()
     o.setup()
-    _check_all(g, o)
+    _check_all(g, o, topk=5)
     g.churn_step()
     o.churn_step()
-    _check_all(g, o, step=1)
+    _check_all(g, o, step=1, topk=64)
 
 
 @pytest.mark.parametrize("hq,hkv", [(1, 1), (2, 2), (5, 1), (8, 1), (40, 8), (6, 3)])
@@ -107,7 +108,7 @@ def test_gqa_groups(hq, hkv):
     g, o = _pair(w)
     g.setup()
     o.setup()
-    _check_all(g, o)
+    _check_all(g, o, topk=3)
 
 
 def test_no_eviction_dense_16bit():
@@ -126,6 +127,17 @@ def test_empty_and_fully_evicted_sequences():
     g, o = _pair(w)
     g.setup()
     o.setup()
-    out, _ = g.decode(0)
-    assert torch.count_nonzero(out) == 0
-    _check_all(g, o)
+    out, mass = g.decode(0, topk=4)
+    assert torch.count_nonzero(out) == 0 and torch.count_nonzero(mass) == 0
+    _check_all(g, o, topk=4)
+
+
+@pytest.mark.parametrize("k", [1, 2, 31, 32, 33, 64])
+def test_topk_mass_values_of_k(k):
+    """k around the candidate-buffer boundaries; long segments force compactions."""
+    w = W.Workload(name="x", batch=2, num_q_heads=16, num_kv_heads=2, head_dim=64, group_size=32,
+                   lengths=("fixed", 3000), budget=("frac", 0.5), seed=7)
+    g, o = _pair(w)
+    g.setup()
+    o.setup()
+    _check_all(g, o, topk=k, codes=False)
