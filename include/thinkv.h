@@ -231,7 +231,12 @@ THINKV_API size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t 
  * probability held by the topk (1..64) most probable live tokens (1 when the
  * sequence has <= topk live tokens, 0 when it has none).
  * workspace: device, >= thinkv_decode_workspace_bytes(L, n_seqs, topk) bytes,
- * caller-owned scratch, no initialisation needed.  1 <= n_seqs <= 16384. */
+ * caller-owned scratch.  Its first n_seqs*num_kv_heads 32-bit words are the
+ * per-(sequence, kv-head) arrival counters of the split-K merge: zero-fill the
+ * workspace once before its first use; every call that completes leaves them
+ * zero again (after a call that stopped on a device error, zero them again).
+ * Calls that share a workspace must not overlap on the GPU.
+ * 1 <= n_seqs <= 16384. */
 THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs, const int32_t* seq,
                             const uint16_t* q, uint16_t* out, float* topk_mass,
                             int32_t topk, float softmax_scale,

@@ -19,9 +19,10 @@
 //   scale/zero in fp32, runs the online softmax, transposes p through a small
 //   shared buffer and accumulates p*scale (fp16, exponent-shifted) times the V
 //   codes on the tensor cores, with the zero terms summed in fp32.  Each warp
-//   writes one partial (m, l, o) per (sequence, kv-head) segment it touched.
-//   combine kernel: one warp per (sequence, q-head) merges the partials of its
-//   segment with the log-sum-exp rule, writes fp16 O and the top-k mass.
+//   writes one partial (m, l, o, top-k logits) per (sequence, kv-head) segment
+//   it touched and counts itself in on the segment's arrival counter; the
+//   last warp to arrive merges the segment's partials with the log-sum-exp
+//   rule and writes fp16 O and the top-k mass -- one launch per decode.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -55,8 +56,11 @@ struct DecodeParams {
   float scale_log2;
   float* part_o;   // [pieces][Gq][D]
   float* part_ml;  // [pieces][Gq][2]   (m in log2 units, l)
-  int32_t* plan;   // [n + 1] exclusive prefix of live pages per decoded sequence
   float* part_topk;  // [pieces][Gq][topk] largest logits (log2 units), -inf padded
+  uint32_t* ctr;     // [n * Hkv] arrival counters of the segments (zero between calls)
+  const int32_t* live_count;
+  uint16_t* out;     // [n][Hq][D]
+  float* mass;       // [n][Hq] or null
   int32_t topk;
   int32_t* status;
   int32_t nstage, stage_bytes, warp_smem, plan_smem;
@@ -130,6 +134,93 @@ __device__ inline void cand_compact(const TopkCtx& tk, int h) {
   __syncwarp();
 }
 
+// Merges the partials (m, l, o, top-k logits) of segment (i, h) -- pieces
+// w0..w1, skipping warps with an empty unit range -- into fp16 O and the
+// top-k mass of its Gq query heads.  Run by the last warp to finish a piece of
+// the segment; partials are read through L2 (ld.global.cg).
+template <int D>
+__device__ void merge_segment(const DecodeParams& p, int i, int h, int64_t w0, int64_t w1,
+                              int64_t T, int64_t W) {
+  const int lane = threadIdx.x & 31;
+  constexpr int PER = D / 32;
+  const int Gq = p.Gq;
+  const int64_t seg = (int64_t)i * p.Hkv + h;
+  for (int r = 0; r < Gq; ++r) {
+    const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
+    float M = -INFINITY;
+    for (int64_t w = w0; w <= w1; ++w) {
+      if (w * T / W == (w + 1) * T / W) continue;
+      M = fmaxf(M, __ldcg(&p.part_ml[((w + seg) * Gq + r) * 2]));
+    }
+    float L = 0.f, acc[PER];
+#pragma unroll
+    for (int x = 0; x < PER; ++x) acc[x] = 0.f;
+    for (int64_t w = w0; w <= w1; ++w) {
+      if (w * T / W == (w + 1) * T / W) continue;
+      const int64_t pc = (w + seg) * Gq + r;
+      const float f = exp2_approx(__ldcg(&p.part_ml[pc * 2]) - M);
+      L = fmaf(__ldcg(&p.part_ml[pc * 2 + 1]), f, L);
+      const float* po = p.part_o + pc * D + lane * PER;
+#pragma unroll
+      for (int x = 0; x < PER; ++x) acc[x] = fmaf(__ldcg(po + x), f, acc[x]);
+    }
+    const float inv = 1.f / L;
+    uint16_t* o = p.out + row * D + lane * PER;
+    if constexpr (PER == 4) {
+      const uint32_t a = (uint32_t)__half_as_ushort(__float2half_rn(acc[0] * inv)) |
+                         ((uint32_t)__half_as_ushort(__float2half_rn(acc[1] * inv)) << 16);
+      const uint32_t b = (uint32_t)__half_as_ushort(__float2half_rn(acc[2] * inv)) |
+                         ((uint32_t)__half_as_ushort(__float2half_rn(acc[3] * inv)) << 16);
+      *reinterpret_cast<uint2*>(o) = make_uint2(a, b);
+    } else {
+      *reinterpret_cast<uint32_t*>(o) =
+          (uint32_t)__half_as_ushort(__float2half_rn(acc[0] * inv)) |
+          ((uint32_t)__half_as_ushort(__float2half_rn(acc[1] * inv)) << 16);
+    }
+    if (p.mass) {
+      const int k = p.topk;
+      if (p.live_count[p.seq[i]] <= k) {
+        if (lane == 0) p.mass[row] = 1.f;
+        continue;
+      }
+      // top-k of the union of the pieces' top-k lists, merged piece by piece
+      float v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = -INFINITY;
+      for (int64_t w = w0; w <= w1; ++w) {
+        if (w * T / W == (w + 1) * T / W) continue;
+        const float* src = p.part_topk + ((w + seg) * Gq + r) * k;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = lane * 4 + j;
+          if (e >= k) v[j] = (e < 2 * k) ? __ldcg(src + e - k) : -INFINITY;
+        }
+        bitonic128_desc(v);
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (lane * 4 + j < k) sum += exp2_approx(v[j] - M);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+      if (lane == 0) p.mass[row] = sum * inv;
+    }
+  }
+}
+
+// Sequences with no live token: zeros (and mass 0), written by the grid.
+__device__ void write_empty_outputs(const DecodeParams& p, const int32_t* P, int D) {
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t x = tid; x < (int64_t)p.n * p.Hq; x += nthreads) {
+    const int i = (int)(x / p.Hq);
+    if (P[i + 1] != P[i]) continue;
+    uint16_t* o = p.out + x * D;
+    for (int c = 0; c < D; ++c) o[c] = 0;
+    if (p.mass) p.mass[x] = 0.f;
+  }
+}
+
 // Per-warp state of the (sequence, kv-head) segment being processed.
 template <int D, int G>
 struct SegState {
@@ -187,7 +278,8 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i
 
 template <int D, int G>
 __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t piece,
-                               const TopkCtx& tk) {
+                               const TopkCtx& tk, const int32_t* P, int i, int h, int64_t T,
+                               int64_t W) {
   constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -230,6 +322,21 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
       for (int j = lane; j < tk.topk; j += 32) dst[j] = j < n ? tk.cand[hd * kCandCap + j] : -INFINITY;
     }
     __syncwarp();
+  }
+  // arrival: the last warp to finish a piece of this segment merges all pieces
+  const int nl = P[i + 1] - P[i];
+  const int64_t Us = (int64_t)P[i] * p.Hkv + (int64_t)h * nl, Ue = Us + nl;
+  const int64_t w0 = ((Us + 1) * W - 1) / T, w1 = (Ue * W - 1) / T;
+  // with T <= W every non-empty warp holds exactly one unit; otherwise none is empty
+  const uint32_t npieces = (uint32_t)(T <= W ? (int64_t)nl : w1 - w0 + 1);
+  __threadfence();
+  __syncwarp();
+  uint32_t old = 0;
+  if (lane == 0) old = atomicInc(&p.ctr[(int64_t)i * p.Hkv + h], npieces - 1);
+  old = __shfl_sync(0xFFFFFFFFu, old, 0);
+  if (old == npieces - 1) {
+    __threadfence();
+    merge_segment<D>(p, i, h, w0, w1, T, W);
   }
 }
 
@@ -577,9 +684,8 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     if (tid == 0) P[p.n] = carry;
     __syncthreads();
-    if (blockIdx.x == 0)
-      for (int i = tid; i <= p.n; i += kDecThreads) p.plan[i] = P[i];
   }
+  write_empty_outputs(p, P, D);
 
   const int64_t T = (int64_t)P[p.n] * p.Hkv;
   const int64_t W = (int64_t)gridDim.x * kDecWarps;
@@ -619,7 +725,7 @@ __global__ void __launch_bounds__(kDecThreads)
   }
 
   SegState<D, G> S;
-  int seg = -1;
+  int seg = -1, cur_i = 0, cur_h = 0;
   for (int64_t k = 0; k < nunits; ++k) {
     const int kk = (int)(k & 31);
     if (kk == 0 && k > 0) {
@@ -628,8 +734,10 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     const UnitMeta m = shfl_meta(cur, kk);
     if (m.seg != seg) {
-      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk);
+      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, cur_i, cur_h, T, W);
       seg = m.seg;
+      cur_i = m.i;
+      cur_h = m.h;
       seg_begin<D, G>(S, p, m.i, m.h, tk);
     }
     const int stage = (int)(k % p.nstage);
@@ -658,98 +766,7 @@ __global__ void __launch_bounds__(kDecThreads)
       bulk_g2s(wsm + stage * p.stage_bytes, mn.src, bytes, &bars[stage]);
     }
   }
-  if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk);
-}
-
-// ---------------------------------------------------------------------------
-// combine: one warp per (sequence, q-head)
-// ---------------------------------------------------------------------------
-struct CombineParams {
-  const float* part_o;
-  const float* part_ml;
-  const float* part_topk;
-  const int32_t* plan;
-  const int32_t* seq;
-  const int32_t* live_count;
-  int32_t n, Hq, Hkv, Gq, topk;
-  int64_t W;
-  uint16_t* out;
-  float* mass;
-};
-
-template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(CombineParams c) {
-  const int lane = threadIdx.x & 31;
-  const int64_t gw = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (gw >= (int64_t)c.n * c.Hq) return;
-  const int Hkv = c.Hkv, Gq = c.Gq;
-  const int i = (int)(gw / c.Hq), hq = (int)(gw % c.Hq), h = hq / Gq, r = hq % Gq;
-  constexpr int PER = D / 32;
-  uint16_t* o = c.out + gw * D + lane * PER;
-  const int Pi = c.plan[i], nl = c.plan[i + 1] - Pi;
-  if (nl == 0) {
-#pragma unroll
-    for (int x = 0; x < PER; ++x) o[x] = 0;
-    if (c.mass && lane == 0) c.mass[gw] = 0.f;
-    return;
-  }
-  const int64_t W = c.W;
-  const int64_t T = (int64_t)c.plan[c.n] * Hkv;
-  const int64_t Us = (int64_t)Pi * Hkv + (int64_t)h * nl, Ue = Us + nl;
-  const int64_t w0 = ((Us + 1) * W - 1) / T, w1 = (Ue * W - 1) / T;
-  const int64_t seg = (int64_t)i * Hkv + h;
-  // warps whose unit range is empty (possible when there are fewer units than
-  // warps) wrote no partial
-  float M = -INFINITY;
-  for (int64_t w = w0; w <= w1; ++w) {
-    if (w * T / W == (w + 1) * T / W) continue;
-    M = fmaxf(M, c.part_ml[((w + seg) * Gq + r) * 2]);
-  }
-  float L = 0.f, acc[PER];
-#pragma unroll
-  for (int x = 0; x < PER; ++x) acc[x] = 0.f;
-  for (int64_t w = w0; w <= w1; ++w) {
-    if (w * T / W == (w + 1) * T / W) continue;
-    const int64_t pc = (w + seg) * Gq + r;
-    const float f = exp2_approx(c.part_ml[pc * 2] - M);
-    L = fmaf(c.part_ml[pc * 2 + 1], f, L);
-    const float* po = c.part_o + pc * D + lane * PER;
-#pragma unroll
-    for (int x = 0; x < PER; ++x) acc[x] = fmaf(po[x], f, acc[x]);
-  }
-  const float inv = 1.f / L;
-#pragma unroll
-  for (int x = 0; x < PER; ++x) o[x] = __half_as_ushort(__float2half_rn(acc[x] * inv));
-
-  if (c.mass) {
-    const int k = c.topk;
-    const int nlive = c.live_count[c.seq[i]];
-    if (nlive <= k) {
-      if (lane == 0) c.mass[gw] = 1.f;
-      return;
-    }
-    // top-k of the union of the pieces' top-k lists: merge piece by piece
-    float v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = -INFINITY;
-    for (int64_t w = w0; w <= w1; ++w) {
-      if (w * T / W == (w + 1) * T / W) continue;
-      const float* src = c.part_topk + ((w + seg) * Gq + r) * k;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int e = lane * 4 + j;
-        if (e >= k) v[j] = (e < 2 * k) ? src[e - k] : -INFINITY;
-      }
-      bitonic128_desc(v);
-    }
-    float sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (lane * 4 + j < k) sum += exp2_approx(v[j] - M);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
-    if (lane == 0) c.mass[gw] = sum * inv;
-  }
+  if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, cur_i, cur_h, T, W);
 }
 
 template <int D, int G>
@@ -817,7 +834,7 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
 size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
                               const DecodeLaunch& dl) {
   const int Gq = L.num_q_heads / L.num_kv_heads;
-  size_t b = ((size_t)(n_seqs + 1) * 4 + 255) / 256 * 256;
+  size_t b = ((size_t)n_seqs * L.num_kv_heads * 4 + 255) / 256 * 256;  // arrival counters
   b += ((size_t)dl.pieces * Gq * 2 * 4 + 255) / 256 * 256;
   b += ((size_t)dl.pieces * Gq * L.head_dim * 4 + 255) / 256 * 256;
   b += ((size_t)dl.pieces * Gq * (topk > 0 ? topk : 0) * 4 + 255) / 256 * 256;
@@ -849,14 +866,17 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
   uint8_t* w = static_cast<uint8_t*>(ws);
-  p.plan = reinterpret_cast<int32_t*>(w);
-  w += ((size_t)(n + 1) * 4 + 255) / 256 * 256;
+  p.ctr = reinterpret_cast<uint32_t*>(w);
+  w += ((size_t)n * L.num_kv_heads * 4 + 255) / 256 * 256;
   p.part_ml = reinterpret_cast<float*>(w);
   w += ((size_t)dl.pieces * p.Gq * 2 * 4 + 255) / 256 * 256;
   p.part_o = reinterpret_cast<float*>(w);
   w += ((size_t)dl.pieces * p.Gq * D * 4 + 255) / 256 * 256;
   p.part_topk = reinterpret_cast<float*>(w);
   p.topk = mass ? topk : 0;
+  p.live_count = C.live_count;
+  p.out = out;
+  p.mass = p.topk > 0 ? mass : nullptr;
   p.status = C.status;
   p.nstage = dl.nstage;
   p.stage_bytes = dl.stage_bytes;
@@ -867,27 +887,7 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   else if (D == 128 && G == 32) e = launch_split<128, 32>(p, dl, stream);
   else if (D == 64 && G == 64) e = launch_split<64, 64>(p, dl, stream);
   else e = launch_split<64, 32>(p, dl, stream);
-  if (e != cudaSuccess) return e;
-  const int64_t warps = (int64_t)n * L.num_q_heads;
-  const int blocks = (int)((warps + 3) / 4);
-  CombineParams cp;
-  cp.part_o = p.part_o;
-  cp.part_ml = p.part_ml;
-  cp.part_topk = p.part_topk;
-  cp.plan = p.plan;
-  cp.seq = seq;
-  cp.live_count = C.live_count;
-  cp.n = n;
-  cp.Hq = p.Hq;
-  cp.Hkv = p.Hkv;
-  cp.Gq = p.Gq;
-  cp.topk = p.topk;
-  cp.W = (int64_t)dl.grid * kDecWarps;
-  cp.out = out;
-  cp.mass = p.topk > 0 ? mass : nullptr;
-  if (D == 128) decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(cp);
-  else decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(cp);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace thinkv
