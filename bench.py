@@ -1,0 +1,447 @@
+"""Benchmark of the ThinKV decode hot path (append -> evict -> decode per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl thinkv|reference]
+
+One step = one token appended (quantised) per sequence, eviction back to the
+budget, and decode attention (+ the top-k mass when the workload asks for
+it) over every sequence -- the whole hot path over one batch.  The workload
+defaults to the R1-Distill-Llama-8B-shaped layer (16 sequences x 16384
+generated tokens, 32/8 heads, head_dim 128, 8/4/2-bit R/E/T codes, group 64,
+5% budget).  Inputs are synthetic and seeded; the per-step inputs are
+resident on the GPU before timing; L2 is flushed (512 MiB write) between
+steps, outside the timed events.
+
+The metric is decode tokens/s (one token per sequence per step); the
+roofline block reports the decode kernel's achieved HBM bandwidth from its
+algorithmic bytes.  `--impl reference` times the CPU oracle (oracle/) on the
+same workload.  Multi-GPU: replicas only (each rank runs its own copy of the
+workload; no data-path collective); value = tokens of all ranks / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
+DEFAULT_WORKLOAD = "r1-llama-8b"
+FLUSH_BYTES = 512 << 20
+DECODE_SRC = os.path.join(ROOT, "mixed_precision_paged_thinkv_b200", "csrc", "thinkv_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------- #
+# small host-side helpers (unit-tested on CPU)
+# --------------------------------------------------------------------------- #
+def aggregate(per_rank):
+    """per_rank: [(tokens, seconds)] -> (total tokens / max seconds, max seconds)."""
+    tokens = sum(t for t, _ in per_rank)
+    worst = max(s for _, s in per_rank)
+    return tokens / worst, worst
+
+
+def parse_clocks(csv_text: str, index: int = None):
+    """Summary of `nvidia-smi --query-gpu=index,clocks.sm,clocks.max.sm,power.draw,
+    clocks_event_reasons.active,...hw_slowdown,hw_thermal_slowdown,sw_thermal_slowdown,
+    sw_power_cap --format=csv` samples taken during the timed region."""
+    rows = []
+    for line in csv_text.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9 or not parts[0].isdigit():
+            continue
+        if index is not None and int(parts[0]) != index:
+            continue
+        try:
+            sm = float(parts[1].split()[0])
+            smax = float(parts[2].split()[0])
+        except ValueError:
+            continue
+        rows.append((sm, smax, parts[5:9]))
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[k] for (_, _, flags) in rows for k, f in enumerate(flags)
+                      if f.lower().startswith("active")})
+    sm = sorted(r[0] for r in rows)
+    return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows),
+            "reasons": reasons, "samples": len(rows)}
+
+
+def peak_hbm_gbs():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    with open(DECODE_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_per_launch(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode source for this workload; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        e = rec.get(workload)
+        if e and e.get("source_sha") == decode_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def algorithmic_decode_bytes(w, snap) -> int:
+    """Bytes one decode call must move: codes + params of every live token for
+    every kv-head, the table entry and live-list entry of every live page, Q,
+    O and (if asked) the fp32 top-k mass."""
+    H, d, G = w.num_kv_heads, w.head_dim, w.group_size
+
+    def entry_class(e):  # block-table entry: page | class << 32 | live_mask << 48
+        return (int(e) >> 32) & 0xFF
+
+    def entry_mask(e):
+        return (int(e) >> 48) & 0xFFFF
+
+    live_by_class = [0, 0, 0]
+    pages = 0
+    for s in range(w.batch):
+        nl = int(snap["num_live"][s])
+        ents = snap["table"][s, snap["live_list"][s, :nl]]
+        pages += nl
+        for e in ents:
+            live_by_class[int(entry_class(e))] += bin(int(entry_mask(e))).count("1")
+    total = 0
+    for c in range(3):
+        b = w.bits[c]
+        per = 2 * d * b // 8 + (2 * (d // G) * 4 if b < 16 else 0)
+        total += live_by_class[c] * H * per
+    total += pages * (8 + 4)
+    total += 2 * w.batch * w.num_q_heads * d * 2
+    if w.topk:
+        total += w.batch * w.num_q_heads * 4
+    return total, live_by_class, pages
+
+
+class ClockSampler:
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, out_path):
+        self.out_path = out_path
+        self.proc = None
+
+    def start(self):
+        try:
+            self.f = open(self.out_path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}",
+                                          "--format=csv", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, uuid: str):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        text = open(self.out_path).read()
+        # drop the uuid column after selecting our GPU's rows
+        keep = []
+        for line in text.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 10 and parts[0].isdigit():
+                u = parts[1].replace("GPU-", "")
+                if uuid and u != uuid.replace("GPU-", ""):
+                    continue
+                keep.append(",".join([parts[0]] + parts[2:]))
+        return parse_clocks("\n".join(keep))
+
+
+# --------------------------------------------------------------------------- #
+# distributed plumbing (replicas only)
+# --------------------------------------------------------------------------- #
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if os.environ.get("THINKV_BENCH_BACKEND", "nccl") == "nccl" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def dist_max_sum(seconds: float, tokens: float, world: int, device):
+    if world == 1:
+        return seconds, tokens
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    n = torch.tensor([tokens], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- #
+# oracle timing (CPU baseline and the reference arm)
+# --------------------------------------------------------------------------- #
+def time_oracle(w, steps: int, warmup: int, budget_s: float, gen_device: str):
+    """Replays the workload's setup in the oracle (untimed), then times oracle
+    steps (append + evict + decode over every sequence).  Returns a dict."""
+    import torch
+    from mixed_precision_paged_thinkv_b200 import workloads as W
+    from mixed_precision_paged_thinkv_b200.runner import geometry
+    from oracle import oracle as O
+
+    sched = W.Schedule(w, extra=warmup + steps + 2)
+    geom = geometry(w, sched)
+    o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
+                 geom["max_seqs"], geom["max_blocks_per_seq"], geom["pool_pages"])
+    t0 = time.time()
+    for call in sched.prefill_calls():
+        k, v = W.call_kv(w, call, device=gen_device)
+        assert o.append(call.seqs, call.pos, call.tags, k.cpu(), v.cpu()) == O.OK
+    gen = sched.lengths.astype(np.int64).copy()
+    allseq = np.arange(w.batch, dtype=np.int32)
+    assert o.evict(allseq, sched.budgets(gen)) == O.OK
+    setup_s = time.time() - t0
+    threads = os.cpu_count() or 1
+    times = []
+    for k in range(warmup + steps):
+        call = sched.one_token_call(gen)
+        kk, vv = W.call_kv(w, call, device=gen_device)
+        kk, vv = kk.cpu(), vv.cpu()
+        q = W.q_values(w, k, device=gen_device).cpu()
+        gen = gen + 1
+        b = sched.budgets(gen)
+        t = time.perf_counter()
+        assert o.append(call.seqs, call.pos, call.tags, kk, vv) == O.OK
+        assert o.evict(allseq, b) == O.OK
+        o.decode(allseq, q, topk=w.topk, threads=threads)
+        dt = time.perf_counter() - t
+        if k >= warmup:
+            times.append(dt)
+        if k >= warmup and sum(times) > budget_s:
+            break
+    total = sum(times)
+    return {"seconds": total, "steps": len(times), "tokens": w.batch * len(times),
+            "value": w.batch * len(times) / total, "cores": threads, "setup_s": setup_s}
+
+
+def reference_arm(args, w, world, rank):
+    if rank != 0:
+        return 0
+    gen_device = "cuda" if _cuda_ok() else "cpu"
+    r = time_oracle(w, args.steps, args.warmup, budget_s=120.0, gen_device=gen_device)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": r["steps"], "warmup": args.warmup,
+        "ms_per_step": 1000.0 * r["seconds"] / max(1, r["steps"]), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (attention), f32 (quantiser)",
+        "data": "synthetic", "config": workload_config(w, None),
+        "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": r["cores"],
+                         "kind": "oracle",
+                         "sample": f"oracle replays the setup untimed, then {r['steps']} steps "
+                                   f"(append 1 token/seq + evict + decode over all {w.batch} seqs)"},
+        "e2e": {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _cuda_ok():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+def workload_config(w, live):
+    cfg = {"workload": f"{w.name}: layer {w.num_q_heads}q/{w.num_kv_heads}kv heads, "
+                       f"head_dim {w.head_dim}, batch {w.batch}, lengths {w.lengths}, "
+                       f"R/E/T {w.bits[0]}/{w.bits[1]}/{w.bits[2]}-bit, group {w.group_size}, "
+                       f"budget {w.budget}",
+           "batch": w.batch, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
+           "head_dim": w.head_dim, "group_size": w.group_size, "page_size": w.page_size,
+           "bits_RET": list(w.bits), "topk": w.topk,
+           "l2": "flushed between steps (512 MiB write, outside the timed events)",
+           "parallelism": "replicas"}
+    if live is not None:
+        cfg["live_tokens_by_class"] = live
+    return cfg
+
+
+# --------------------------------------------------------------------------- #
+# the library arm
+# --------------------------------------------------------------------------- #
+def thinkv_arm(args, w, world, rank, local):
+    import torch
+    from mixed_precision_paged_thinkv_b200 import build as B
+    from mixed_precision_paged_thinkv_b200.runner import (WorkloadRun, make_steps, run_step,
+                                                          run_step_from_host)
+    B.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    K, Wm = args.steps, args.warmup
+    e2e_steps = max(3, min(K, 20))
+    run = WorkloadRun(w, extra=Wm + K + e2e_steps + 2, device=str(dev))
+    run.setup()
+    torch.cuda.synchronize()
+    steps = make_steps(run, Wm + K + e2e_steps, device=dev)
+    out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float16, device=dev)
+    mass = torch.empty(w.batch, w.num_q_heads, dtype=torch.float32, device=dev) if w.topk else None
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for k in range(Wm):
+        flush.zero_()
+        run_step(run.cache, steps[k], out, topk=w.topk, mass=mass)
+    torch.cuda.synchronize()
+    assert run.cache.status() == 0, "device status after warm-up"
+    snap = run.cache.snapshot()
+    alg_bytes, live, pages = algorithmic_decode_bytes(w, snap)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/clocks{rank}.csv")
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.4)
+    t_wall = time.time()
+    for k in range(K):
+        flush.zero_()
+        inp = steps[Wm + k]
+        ev[k][0].record()
+        run.cache.append(inp.seqs, inp.pos, inp.tags, inp.k, inp.v)
+        run.cache.evict(inp.seqs, inp.budgets)
+        ev[k][1].record()
+        run.cache.decode(inp.seqs, inp.q, topk=w.topk, out=out, mass=mass)
+        ev[k][2].record()
+    torch.cuda.synchronize()
+    t_wall = time.time() - t_wall
+    barrier(world)
+    clk = clocks.stop(str(torch.cuda.get_device_properties(dev).uuid))
+    assert run.cache.status() == 0, "device status after the timed steps"
+    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    step_s = sum(step_ms) / 1000.0
+    max_s, tokens = dist_max_sum(step_s, float(w.batch * K), world, dev)
+    value = tokens / max_s
+
+    # end to end through host buffers (pinned), copies inside the timed region
+    host = [steps[Wm + K + k].to("cpu", pin=True) for k in range(e2e_steps)]
+    dbuf = steps[Wm + K]  # device staging tensors, overwritten by the copies
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    mass_h = torch.empty(mass.shape, dtype=mass.dtype).pin_memory() if w.topk else None
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(e2e_steps)]
+    torch.cuda.synchronize()
+    for k in range(e2e_steps):
+        flush.zero_()
+        e2e_ev[k][0].record()
+        run_step_from_host(run.cache, host[k], dbuf, out, out_h, topk=w.topk,
+                           mass_dev=mass, mass_host=mass_h)
+        e2e_ev[k][1].record()
+    torch.cuda.synchronize()
+    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1000.0
+    e2e_max, e2e_tok = dist_max_sum(e2e_s, float(w.batch * e2e_steps), world, dev)
+    h2d = host[0].nbytes()
+    d2h = out_h.numel() * 2 + (mass_h.numel() * 4 if w.topk else 0)
+
+    # roofline of the decode kernel (one launch per decode call)
+    dec_avg_s = sum(dec_ms) / len(dec_ms) / 1000.0
+    achieved = alg_bytes / dec_avg_s / 1e9
+    peak, peak_kind = peak_hbm_gbs()
+    traffic = traffic_per_launch(w.name)
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            r = time_oracle(w, steps=200, warmup=1, budget_s=15.0, gen_device=str(dev))
+            cpu = {"value": r["value"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+                   "sample": f"oracle (C, fp64 attention) replays the setup untimed, then "
+                             f"{r['steps']} steps of append 1 token/seq + evict + decode over all "
+                             f"{w.batch} seqs (~15 s cap); decode on {r['cores']} OpenMP threads"}
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": Wm, "ms_per_step": 1000.0 * max_s / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8/4/2 codes, f16 mma, f32 accumulate",
+            "data": "synthetic (seeded counter-hash normals, segment tags)",
+            "config": workload_config(w, live),
+            "decode_ms": sum(dec_ms) / len(dec_ms),
+            "decode_hbm_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                         "kernel": "decode_split_kernel (one launch per decode call)",
+                         "algorithmic_bytes_per_launch": alg_bytes, "live_pages": pages},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_tok / e2e_max, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": 4 * K,
+            "clocks": clk,
+            "wall_s_timed_loop": t_wall,
+        }
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="thinkv", choices=["thinkv", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from mixed_precision_paged_thinkv_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    world, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            return reference_arm(args, w, world, rank)
+        res = thinkv_arm(args, w, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

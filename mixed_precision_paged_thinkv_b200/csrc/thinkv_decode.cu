@@ -134,77 +134,159 @@ __device__ inline void cand_compact(const TopkCtx& tk, int h) {
   __syncwarp();
 }
 
-// Merges the partials (m, l, o, top-k logits) of segment (i, h) -- pieces
-// w0..w1, skipping warps with an empty unit range -- into fp16 O and the
-// top-k mass of its Gq query heads.  Run by the last warp to finish a piece of
-// the segment; partials are read through L2 (ld.global.cg).
+// Merges the partials (m, l, o, top-k logits) of segment (i, h) into fp16 O
+// and the top-k mass of its Gq query heads.  Run by the last warp to finish a
+// piece of the segment.  Pieces are the non-empty warps from w0 on: with
+// T <= W every unit has its own warp, otherwise all of w0..w1 hold units.
+// Loads are issued lane-parallel or in independent batches (a loop of
+// dependent loads would put one L2 round trip per piece on the kernel tail);
+// partials are read through L2 (ld.global.cg).
+__device__ inline int64_t piece_warp(int j, int64_t Us, int64_t w0, int64_t T, int64_t W) {
+  return T <= W ? ((Us + j + 1) * W - 1) / T : w0 + j;
+}
+
 template <int D>
-__device__ void merge_segment(const DecodeParams& p, int i, int h, int64_t w0, int64_t w1,
-                              int64_t T, int64_t W) {
+__device__ void merge_segment(const DecodeParams& p, int i, int h, int64_t Us, int64_t w0,
+                              int np, int64_t T, int64_t W, const TopkCtx& tk) {
   const int lane = threadIdx.x & 31;
   constexpr int PER = D / 32;
+  constexpr int BATCH = 8;
   const int Gq = p.Gq;
   const int64_t seg = (int64_t)i * p.Hkv + h;
   for (int r = 0; r < Gq; ++r) {
     const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
-    float M = -INFINITY;
-    for (int64_t w = w0; w <= w1; ++w) {
-      if (w * T / W == (w + 1) * T / W) continue;
-      M = fmaxf(M, __ldcg(&p.part_ml[((w + seg) * Gq + r) * 2]));
-    }
-    float L = 0.f, acc[PER];
+    // ---- running max and row sum: pieces across lanes ----
+    float mloc = -INFINITY;
+    for (int j = lane; j < np; j += 32)
+      mloc = fmaxf(mloc, __ldcg(&p.part_ml[((piece_warp(j, Us, w0, T, W) + seg) * Gq + r) * 2]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xFFFFFFFFu, mloc, o));
+    const float M = mloc;
+    float lloc = 0.f;
+    float acc[PER];
 #pragma unroll
     for (int x = 0; x < PER; ++x) acc[x] = 0.f;
-    for (int64_t w = w0; w <= w1; ++w) {
-      if (w * T / W == (w + 1) * T / W) continue;
-      const int64_t pc = (w + seg) * Gq + r;
-      const float f = exp2_approx(__ldcg(&p.part_ml[pc * 2]) - M);
-      L = fmaf(__ldcg(&p.part_ml[pc * 2 + 1]), f, L);
-      const float* po = p.part_o + pc * D + lane * PER;
+    for (int jb = 0; jb < np; jb += 32) {
+      // this lane's piece of the chunk: weight f = 2^(m - M)
+      float f = 0.f;
+      if (jb + lane < np) {
+        const int64_t pc = (piece_warp(jb + lane, Us, w0, T, W) + seg) * Gq + r;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + pc * 2));
+        f = exp2_approx(ml.x - M);
+        lloc = fmaf(ml.y, f, lloc);
+      }
+      const int cnt = min(32, np - jb);
+      for (int jj = 0; jj < cnt; jj += BATCH) {
+        float vals[BATCH][PER];
 #pragma unroll
-      for (int x = 0; x < PER; ++x) acc[x] = fmaf(__ldcg(po + x), f, acc[x]);
+        for (int b = 0; b < BATCH; ++b) {
+          if (jj + b < cnt) {
+            const int64_t pc = (piece_warp(jb + jj + b, Us, w0, T, W) + seg) * Gq + r;
+            const float* po = p.part_o + pc * D + lane * PER;
+            if constexpr (PER == 4) {
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(po));
+              vals[b][0] = v.x; vals[b][1] = v.y; vals[b][2] = v.z; vals[b][3] = v.w;
+            } else {
+              const float2 v = __ldcg(reinterpret_cast<const float2*>(po));
+              vals[b][0] = v.x; vals[b][1] = v.y;
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+          const float fb = __shfl_sync(0xFFFFFFFFu, f, (jj + b) & 31);
+          if (jj + b < cnt) {
+#pragma unroll
+            for (int x = 0; x < PER; ++x) acc[x] = fmaf(vals[b][x], fb, acc[x]);
+          }
+        }
+      }
     }
-    const float inv = 1.f / L;
-    uint16_t* o = p.out + row * D + lane * PER;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lloc += __shfl_xor_sync(0xFFFFFFFFu, lloc, o);
+    const float inv = 1.f / lloc;
+    uint16_t* out = p.out + row * D + lane * PER;
     if constexpr (PER == 4) {
       const uint32_t a = (uint32_t)__half_as_ushort(__float2half_rn(acc[0] * inv)) |
                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[1] * inv)) << 16);
       const uint32_t b = (uint32_t)__half_as_ushort(__float2half_rn(acc[2] * inv)) |
                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[3] * inv)) << 16);
-      *reinterpret_cast<uint2*>(o) = make_uint2(a, b);
+      *reinterpret_cast<uint2*>(out) = make_uint2(a, b);
     } else {
-      *reinterpret_cast<uint32_t*>(o) =
+      *reinterpret_cast<uint32_t*>(out) =
           (uint32_t)__half_as_ushort(__float2half_rn(acc[0] * inv)) |
           ((uint32_t)__half_as_ushort(__float2half_rn(acc[1] * inv)) << 16);
     }
-    if (p.mass) {
-      const int k = p.topk;
-      if (p.live_count[p.seq[i]] <= k) {
-        if (lane == 0) p.mass[row] = 1.f;
-        continue;
+
+    if (!p.mass) continue;
+    const int k = p.topk;
+    if (p.live_count[p.seq[i]] <= k) {
+      if (lane == 0) p.mass[row] = 1.f;
+      continue;
+    }
+    // ---- top-k of the union of the pieces' top-k lists ----
+    // Each list holds its piece's k largest logits (-inf padded), so the
+    // union's k-th largest is >= theta = max over pieces of min(list): only
+    // values >= theta can be in the top-k, and at least k of them exist.
+    float v[4];
+    bool done = false;
+    const int staged = np * k;
+    if (staged <= (Gq - 1) * kCandCap) {
+      float* st = tk.cand;                                 // staging: np*k values
+      float* sb = tk.cand + (Gq - 1) * kCandCap;           // selection: 128 values
+      for (int x = lane; x < staged; x += 32) {
+        const int j = x / k, e = x - j * k;
+        st[x] = __ldcg(p.part_topk + ((piece_warp(j, Us, w0, T, W) + seg) * Gq + r) * k + e);
       }
-      // top-k of the union of the pieces' top-k lists, merged piece by piece
-      float v[4];
+      __syncwarp();
+      float th = -INFINITY;
+      for (int j = lane; j < np; j += 32) {
+        float mn = INFINITY;
+        for (int e = 0; e < k; ++e) mn = fminf(mn, st[j * k + e]);
+        th = fmaxf(th, mn);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) th = fmaxf(th, __shfl_xor_sync(0xFFFFFFFFu, th, o));
+      int count = 0;
+      for (int xb = 0; xb < staged; xb += 32) {
+        const int x = xb + lane;
+        const float val = x < staged ? st[x] : -INFINITY;
+        const bool keep = x < staged && val >= th && val > -INFINITY;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+        const int at = count + __popc(bal & ((1u << lane) - 1u));
+        if (keep && at < kCandCap) sb[at] = val;
+        count += __popc(bal);
+      }
+      __syncwarp();
+      if (count <= kCandCap) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = (lane * 4 + j < count) ? sb[lane * 4 + j] : -INFINITY;
+        bitonic128_desc(v);
+        done = true;
+      }
+      __syncwarp();
+    }
+    if (!done) {
+      // general path: fold the lists in, one piece at a time
 #pragma unroll
       for (int j = 0; j < 4; ++j) v[j] = -INFINITY;
-      for (int64_t w = w0; w <= w1; ++w) {
-        if (w * T / W == (w + 1) * T / W) continue;
-        const float* src = p.part_topk + ((w + seg) * Gq + r) * k;
+      for (int j = 0; j < np; ++j) {
+        const float* src = p.part_topk + ((piece_warp(j, Us, w0, T, W) + seg) * Gq + r) * k;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = lane * 4 + j;
-          if (e >= k) v[j] = (e < 2 * k) ? __ldcg(src + e - k) : -INFINITY;
+        for (int x = 0; x < 4; ++x) {
+          const int e = lane * 4 + x;
+          if (e >= k) v[x] = (e < 2 * k) ? __ldcg(src + e - k) : -INFINITY;
         }
         bitonic128_desc(v);
       }
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (lane * 4 + j < k) sum += exp2_approx(v[j] - M);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
-      if (lane == 0) p.mass[row] = sum * inv;
     }
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (lane * 4 + j < k) sum += exp2_approx(v[j] - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane == 0) p.mass[row] = sum * inv;
   }
 }
 
@@ -336,7 +418,7 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
   old = __shfl_sync(0xFFFFFFFFu, old, 0);
   if (old == npieces - 1) {
     __threadfence();
-    merge_segment<D>(p, i, h, w0, w1, T, W);
+    merge_segment<D>(p, i, h, Us, w0, (int)npieces, T, W, tk);
   }
 }
 
@@ -648,7 +730,7 @@ __device__ inline UnitMeta shfl_meta(const UnitMeta& m, int src) {
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, 3)
     decode_split_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

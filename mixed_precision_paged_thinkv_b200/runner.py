@@ -90,3 +90,67 @@ class WorkloadRun:
         if decode:
             return self.decode(step, topk)
         return None
+
+
+# --------------------------------------------------------------------------- #
+# decode steps: one token appended per sequence, evict to budget, decode
+# --------------------------------------------------------------------------- #
+class StepInputs:
+    """Everything one step consumes, as tensors on one device (or pinned host)."""
+
+    FIELDS = ("seqs", "pos", "tags", "k", "v", "budgets", "q")
+
+    def __init__(self, **t):
+        for f in self.FIELDS:
+            setattr(self, f, t[f])
+
+    def nbytes(self) -> int:
+        return sum(getattr(self, f).numel() * getattr(self, f).element_size() for f in self.FIELDS)
+
+    def to(self, device, pin: bool = False) -> "StepInputs":
+        out = {}
+        for f in self.FIELDS:
+            x = getattr(self, f).to(device)
+            out[f] = x.pin_memory() if pin else x
+        return StepInputs(**out)
+
+
+def make_steps(run: "WorkloadRun", nsteps: int, first_step: int = 0, device=None):
+    """Inputs of the next ``nsteps`` steps of ``run`` (does not advance it)."""
+    w = run.w
+    device = run.device if device is None else device
+    gen = run.generated.copy()
+    steps = []
+    for k in range(nsteps):
+        call = run.sched.one_token_call(gen)
+        kk, vv = W.call_kv(w, call, device=device)
+        gen = gen + 1
+        steps.append(StepInputs(
+            seqs=to_dev(call.seqs, torch.int32, device), pos=to_dev(call.pos, torch.int32, device),
+            tags=to_dev(call.tags, torch.uint8, device), k=kk, v=vv,
+            budgets=to_dev(run.sched.budgets(gen), torch.int32, device),
+            q=W.q_values(w, first_step + k, device=device)))
+    return steps
+
+
+def run_step(cache: ThinKVCache, inp: StepInputs, out: torch.Tensor, topk: Optional[int] = None,
+             mass: Optional[torch.Tensor] = None):
+    """One step on device-resident inputs: append, evict to budget, decode."""
+    cache.append(inp.seqs, inp.pos, inp.tags, inp.k, inp.v)
+    cache.evict(inp.seqs, inp.budgets)
+    return cache.decode(inp.seqs, inp.q, topk=topk, out=out, mass=mass)
+
+
+def run_step_from_host(cache: ThinKVCache, host: StepInputs, dev: StepInputs,
+                       out_dev: torch.Tensor, out_host: torch.Tensor, topk: Optional[int] = None,
+                       mass_dev: Optional[torch.Tensor] = None,
+                       mass_host: Optional[torch.Tensor] = None):
+    """One step whose inputs start in pinned host memory and whose outputs end
+    there: host->device copies, the three library calls, device->host copies,
+    all queued on the current stream."""
+    for f in StepInputs.FIELDS:
+        getattr(dev, f).copy_(getattr(host, f), non_blocking=True)
+    run_step(cache, dev, out_dev, topk=topk, mass=mass_dev)
+    out_host.copy_(out_dev, non_blocking=True)
+    if topk:
+        mass_host.copy_(mass_dev, non_blocking=True)

@@ -229,7 +229,7 @@ class Oracle:
             "fifo_head": self._arr("or_fifo_head", np.int32, (ns, 3)),
             "fifo_tail": self._arr("or_fifo_tail", np.int32, (ns, 3)),
             "live_count": self._arr("or_live_count", np.int32, (ns,)),
-            "live_list": self._arr("or_live_list", np.int32, (ns, nb)),
+            "live_list": self._arr("or_live_list", np.uint64, (ns, nb)),
             "live_index": self._arr("or_live_index", np.int32, (ns, nb)),
             "num_live": self._arr("or_num_live", np.int32, (ns,)),
             "page_bump": self._arr("or_page_bump", np.int32, (3,)),
@@ -247,3 +247,8 @@ def entry_class(e):
 
 def entry_mask(e):
     return ((np.asarray(e, dtype=np.uint64) >> np.uint64(48)) & np.uint64(0xFFFF)).astype(np.int64)
+
+
+def live_entry(x):
+    """Table entry index held in a live-list descriptor (page | class<<32 | entry<<40)."""
+    return (np.asarray(x, dtype=np.uint64) >> np.uint64(40)).astype(np.int64)

@@ -161,7 +161,7 @@ struct or_state {
   int32_t* fifo_head;
   int32_t* fifo_tail;
   int32_t* live_count;
-  int32_t* live_list;
+  uint64_t* live_list;
   int32_t* live_index;
   int32_t* num_live;
   int32_t page_bump[3];
@@ -170,6 +170,11 @@ struct or_state {
 #define ENTRY_PAGE(e) ((int32_t)((e) & 0xFFFFFFFFull))
 #define ENTRY_CLASS(e) ((int32_t)(((e) >> 32) & 0xFF))
 #define ENTRY_MASK(e) ((uint32_t)(((e) >> 48) & 0xFFFF))
+/* live-list descriptor of a table entry: page | class << 32 | entry << 40 */
+#define LIVE_ENTRY(x) ((int32_t)((x) >> 40))
+static uint64_t live_desc(int32_t page, int c, int32_t e) {
+  return (uint64_t)(uint32_t)page | ((uint64_t)c << 32) | ((uint64_t)e << 40);
+}
 
 static size_t code_elem_size(const or_layout* L, int c) { return L->bits[c] == 16 ? 2 : 1; }
 static size_t codes_per_page(const or_layout* L) {
@@ -218,7 +223,7 @@ or_state* or_create(const or_layout* L) {
   S->fifo_head = (int32_t*)calloc(ns * 3, sizeof(int32_t));
   S->fifo_tail = (int32_t*)calloc(ns * 3, sizeof(int32_t));
   S->live_count = (int32_t*)calloc(ns, sizeof(int32_t));
-  S->live_list = (int32_t*)calloc(ns * nb, sizeof(int32_t));
+  S->live_list = (uint64_t*)calloc(ns * nb, sizeof(uint64_t));
   S->live_index = (int32_t*)malloc(ns * nb * sizeof(int32_t));
   S->num_live = (int32_t*)calloc(ns, sizeof(int32_t));
   if (!S->table || !S->num_blocks || !S->free_slots || !S->free_top || !S->fifo ||
@@ -344,7 +349,7 @@ int or_append(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos,
     *ent |= (uint64_t)1 << (48 + slot);          /* eviction mask bit: live */
     if (before == 0) {                           /* the page became non-empty */
       int32_t at = S->num_live[s]++;
-      S->live_list[(size_t)s * L->max_blocks_per_seq + at] = e;
+      S->live_list[(size_t)s * L->max_blocks_per_seq + at] = live_desc(page, c, e);
       S->live_index[(size_t)s * L->max_blocks_per_seq + e] = at;
     }
     S->slot_pos[c][(size_t)page * OR_PAGE + slot] = pos[i];  /* start index */
@@ -396,12 +401,12 @@ int or_evict(or_state* S, int32_t n, const int32_t* seq, const int32_t* budget,
       uint64_t* ent = &table_row(S, s)[e];
       *ent &= ~((uint64_t)1 << (48 + slot));
       if (ENTRY_MASK(*ent) == 0) {               /* page emptied: swap-remove */
-        int32_t* list = S->live_list + (size_t)s * L->max_blocks_per_seq;
+        uint64_t* list = S->live_list + (size_t)s * L->max_blocks_per_seq;
         int32_t* index = S->live_index + (size_t)s * L->max_blocks_per_seq;
         int32_t at = index[e], last = --S->num_live[s];
-        int32_t moved = list[last];
+        uint64_t moved = list[last];
         list[at] = moved;
-        index[moved] = at;
+        index[LIVE_ENTRY(moved)] = at;
         index[e] = -1;
       }
       S->slot_pos[c][(size_t)ENTRY_PAGE(*ent) * OR_PAGE + slot] = -1;
@@ -538,7 +543,7 @@ const int32_t* or_fifo(const or_state* S) { return S->fifo; }
 const int32_t* or_fifo_head(const or_state* S) { return S->fifo_head; }
 const int32_t* or_fifo_tail(const or_state* S) { return S->fifo_tail; }
 const int32_t* or_live_count(const or_state* S) { return S->live_count; }
-const int32_t* or_live_list(const or_state* S) { return S->live_list; }
+const uint64_t* or_live_list(const or_state* S) { return S->live_list; }
 const int32_t* or_live_index(const or_state* S) { return S->live_index; }
 const int32_t* or_num_live(const or_state* S) { return S->num_live; }
 const int32_t* or_page_bump(const or_state* S) { return S->page_bump; }

@@ -77,7 +77,9 @@ void or_quantize_group(const uint16_t* x, int32_t G, int32_t bits,
  *   num_blocks, live_count, num_live : [max_seqs]     int32
  *   free_slots, fifo : [max_seqs][3][max_blocks*16]   int32 (entry*16+slot)
  *   free_top, fifo_head, fifo_tail : [max_seqs][3]    int32
- *   live_list, live_index : [max_seqs][max_blocks]    int32
+ *   live_list  : [max_seqs][max_blocks]               uint64 page|class<<32|entry<<40
+ *                of the entries with a non-zero mask (first num_live[s] valid)
+ *   live_index : [max_seqs][max_blocks]               int32 position in live_list or -1
  *   page_bump : [3]                                   int32
  */
 const void* or_codes(const or_state* S, int c);
@@ -91,7 +93,7 @@ const int32_t* or_fifo(const or_state* S);
 const int32_t* or_fifo_head(const or_state* S);
 const int32_t* or_fifo_tail(const or_state* S);
 const int32_t* or_live_count(const or_state* S);
-const int32_t* or_live_list(const or_state* S);
+const uint64_t* or_live_list(const or_state* S);
 const int32_t* or_live_index(const or_state* S);
 const int32_t* or_num_live(const or_state* S);
 const int32_t* or_page_bump(const or_state* S);

@@ -1,0 +1,67 @@
+"""Host-side logic of bench.py: clock parsing, aggregation over replicas, and
+the max/sum reduction over ranks (world size 2, gloo, CPU)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+CSV = """index, clocks.sm [MHz], clocks.max.sm [MHz], power.draw [W], clocks_event_reasons.active, clocks_event_reasons.hw_slowdown, clocks_event_reasons.hw_thermal_slowdown, clocks_event_reasons.sw_thermal_slowdown, clocks_event_reasons.sw_power_cap
+0, 1965 MHz, 1965 MHz, 400.1 W, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active
+0, 1950 MHz, 1965 MHz, 700.3 W, 0x0000000000000004, Not Active, Not Active, Not Active, Active
+0, 1900 MHz, 1965 MHz, 800.0 W, 0x0000000000000004, Not Active, Not Active, Not Active, Active
+1, 1000 MHz, 1965 MHz, 100.0 W, 0x0000000000000008, Active, Not Active, Not Active, Not Active
+"""
+
+
+def test_parse_clocks_selects_gpu_and_reasons():
+    c = bench.parse_clocks(CSV, index=0)
+    assert c["sm_mhz"] == 1950.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["samples"] == 3
+    c1 = bench.parse_clocks(CSV, index=1)
+    assert c1["reasons"] == ["hw_slowdown"]
+    assert bench.parse_clocks("")["sm_mhz"] is None
+
+
+def test_aggregate_is_total_tokens_over_slowest_rank():
+    v, worst = bench.aggregate([(160, 1.0), (160, 2.0)])
+    assert worst == 2.0 and v == 160.0
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE="2", LOCAL_RANK=str(rank), THINKV_BENCH_BACKEND="gloo")
+    world, r, _ = bench.dist_init()
+    secs = [1.5, 2.5][r]
+    toks = [16.0, 16.0][r]
+    m, n = bench.dist_max_sum(secs, toks, world, torch.device("cpu"))
+    bench.barrier(world)
+    q.put((r, m, n))
+    dist.destroy_process_group()
+
+
+def test_replicas_reduce_max_time_and_sum_tokens_over_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    for r, m, n in got:
+        assert m == 2.5 and n == 32.0

@@ -64,7 +64,13 @@ def test_scripted_history_worked_by_hand():
     assert _fifo(st, 0, 0) == e["fifo_seq0_R"]
     assert _fifo(st, 1, 2) == e["fifo_seq1_T"]
     assert _fifo(st, 1, 1) == e["fifo_seq1_E"]
-    assert [st["live_list"][s, :st["num_live"][s]].tolist() for s in range(2)] == e["live_list"]
+    assert [O.live_entry(st["live_list"][s, :st["num_live"][s]]).tolist() for s in range(2)] == e["live_list"]
+    # descriptors carry the page and class of their entry
+    for s in range(2):
+        for x in st["live_list"][s, :st["num_live"][s]]:
+            ent = st["table"][s, int(O.live_entry(x))]
+            assert int(O.entry_page(x)) == int(O.entry_page(ent))
+            assert int(O.entry_class(x)) == int(O.entry_class(ent))
     assert st["live_count"].tolist() == e["live_count"]
     assert st["slot_pos"][0][1].tolist() == e["slot_pos_R_page1"]
 
@@ -146,8 +152,11 @@ def _check_invariants(o, st, model, ns):
         assert live_pos == model.live[s]
         # live list = entries with a non-zero mask; live_index inverts it
         nl = st["num_live"][s]
-        lst = st["live_list"][s, :nl]
+        desc = st["live_list"][s, :nl]
+        lst = O.live_entry(desc)
         assert sorted(lst.tolist()) == [e for e in range(nb) if masks[e]]
+        assert np.array_equal(O.entry_page(desc), pages[lst])
+        assert np.array_equal(O.entry_class(desc), classes[lst])
         for i, e in enumerate(lst):
             assert st["live_index"][s, e] == i
         for e in range(nb):
