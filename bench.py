@@ -123,7 +123,8 @@ def algorithmic_decode_bytes(w, snap) -> int:
     pages = 0
     for s in range(w.batch):
         nl = int(snap["num_live"][s])
-        ents = snap["table"][s, snap["live_list"][s, :nl]]
+        desc = snap["live_list"][s, :nl]            # page | class << 32 | entry << 40
+        ents = snap["table"][s, (desc >> np.uint64(40)).astype(np.int64)]
         pages += nl
         for e in ents:
             live_by_class[int(entry_class(e))] += bin(int(entry_mask(e))).count("1")

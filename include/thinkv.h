@@ -68,7 +68,8 @@ enum { THINKV_R = 0, THINKV_E = 1, THINKV_T = 2 };
  *   h / (num_q_heads / num_kv_heads));
  *   head_dim in {64, 128}; group_size in {32, 64}, dividing head_dim;
  *   page_size == 16; bits[c] in {2, 4, 8, 16} for c = R, E, T;
- *   1 <= max_seqs <= 65536; 1 <= max_blocks_per_seq; pool_pages[c] >= 0. */
+ *   1 <= max_seqs <= 65536; 1 <= max_blocks_per_seq <= 2^21;
+ *   num_kv_heads <= 256; 0 <= pool_pages[c] < 2^27. */
 typedef struct {
   int32_t num_q_heads, num_kv_heads, head_dim, page_size, group_size;
   int32_t bits[3];
@@ -97,7 +98,8 @@ typedef struct {
  *                 fifo_head, fifo_tail int32 [max_seqs][3] monotone counters
  *                 (ring index = counter mod capacity).
  *   live_count    int32 [max_seqs]       live tokens per sequence
- *   live_list     int32 [max_seqs][max_blocks_per_seq]  table entries with a
+ *   live_list     uint64 [max_seqs][max_blocks_per_seq]  one descriptor
+ *                 page | class << 32 | entry << 40 per table entry with a
  *                 non-zero live_mask (first num_live[s] valid); an entry joins
  *                 at the end when it gains its first live token and leaves by
  *                 swap-with-last when it loses its last one.
@@ -110,7 +112,7 @@ typedef struct {
  * group_size, ng = d/G), byte offsets:
  *   [0, 2db)          K codes      [2db, 4db)  V codes
  *   [4db, 4db+64ng)   K params     [4db+64ng, 4db+128ng)  V params
- * params: [slot 16][group ng][scale, zero] fp16.
+ * params: [group ng][slot 16][scale, zero] fp16.
  * Codes of one block are "lane-major": 32 lanes x (d*b/16) bytes; lane
  * l = 4*gid + tid (gid 0..7, tid 0..3).  Within 32-bit words (or a 16-bit
  * piece) the codes of even channels sit in the low half and those of odd
@@ -144,7 +146,7 @@ typedef struct {
   int32_t* fifo_head;
   int32_t* fifo_tail;
   int32_t* live_count;
-  int32_t* live_list;
+  uint64_t* live_list;
   int32_t* live_index;
   int32_t* num_live;
   int32_t* page_bump;

@@ -253,7 +253,7 @@ class ThinKVCache:
             "fifo_head": self._host("fifo_head", np.int32, (ns, 3)),
             "fifo_tail": self._host("fifo_tail", np.int32, (ns, 3)),
             "live_count": self._host("live_count", np.int32, (ns,)),
-            "live_list": self._host("live_list", np.int32, (ns, nb)),
+            "live_list": self._host("live_list", np.uint64, (ns, nb)),
             "live_index": self._host("live_index", np.int32, (ns, nb)),
             "num_live": self._host("num_live", np.int32, (ns,)),
             "page_bump": self._host("page_bump", np.int32, (3,)),

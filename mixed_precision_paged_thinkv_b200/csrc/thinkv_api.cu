@@ -32,7 +32,8 @@ bool layout_ok(const thinkv_layout* L) {
     if (L->pool_pages[c] < 0 || L->pool_pages[c] >= (1 << 27)) return false;
   }
   if (L->max_seqs < 1 || L->max_seqs > 65536) return false;
-  if (L->max_blocks_per_seq < 1 || L->max_blocks_per_seq >= (1 << 26)) return false;
+  if (L->max_blocks_per_seq < 1 || L->max_blocks_per_seq > (1 << 21)) return false;
+  if (L->num_kv_heads > 256) return false;
   return true;
 }
 
@@ -124,7 +125,7 @@ size_t thinkv_buffer_bytes(const thinkv_layout* L, int32_t which) {
     case THINKV_BUF_FIFO_HEAD: return ns * 3 * 4;
     case THINKV_BUF_FIFO_TAIL: return ns * 3 * 4;
     case THINKV_BUF_LIVE_COUNT: return ns * 4;
-    case THINKV_BUF_LIVE_LIST: return ns * nb * 4;
+    case THINKV_BUF_LIVE_LIST: return ns * nb * 8;
     case THINKV_BUF_LIVE_INDEX: return ns * nb * 4;
     case THINKV_BUF_NUM_LIVE: return ns * 4;
     case THINKV_BUF_PAGE_BUMP: return 3 * 4;

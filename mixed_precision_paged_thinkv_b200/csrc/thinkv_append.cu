@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const RunInfo ri = ws.runs[r];
     const int s = ri.seq;
     uint64_t* table = C.block_table + (int64_t)s * nb_max;
-    int32_t* llist = C.live_list + (int64_t)s * nb_max;
+    uint64_t* llist = C.live_list + (int64_t)s * nb_max;
     int32_t* lidx = C.live_index + (int64_t)s * nb_max;
     int F[3], tail[3], rank[3] = {0, 0, 0}, last_entry[3] = {-1, -1, -1};
 #pragma unroll
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       const unsigned abal = __ballot_sync(0xFFFFFFFFu, adder);
       if (adder) {
         int at = nlive + __popc(abal & lanemask_lt());
-        llist[at] = entry;
+        llist[at] = make_live_desc(page, c, entry);
         lidx[entry] = at;
       }
       nlive += __popc(abal);
@@ -354,7 +354,7 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
     if ((lane % LPG) == 0) {
       uint16_t* prm = reinterpret_cast<uint16_t*>(blk + 4LL * D * b + (kv ? 64LL * NG : 0));
       uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
-      *reinterpret_cast<uint32_t*>(prm + (slot * NG + grp) * 2) = pair;
+      *reinterpret_cast<uint32_t*>(prm + (grp * 16 + slot) * 2) = pair;
     }
   }
   __syncwarp();

@@ -31,6 +31,11 @@ __host__ __device__ inline uint32_t entry_mask(uint64_t e) { return (uint32_t)(e
 __host__ __device__ inline uint64_t make_entry(uint32_t page, int cls, uint32_t mask) {
   return (uint64_t)page | ((uint64_t)cls << 32) | ((uint64_t)mask << 48);
 }
+// Live-list descriptor: page | class << 32 | table entry << 40.
+__host__ __device__ inline uint64_t make_live_desc(uint32_t page, int cls, int entry) {
+  return (uint64_t)page | ((uint64_t)cls << 32) | ((uint64_t)entry << 40);
+}
+__host__ __device__ inline int live_desc_entry(uint64_t x) { return (int)(x >> 40); }
 
 // ---------------------------------------------------------------------------
 // sticky status: the first error wins
@@ -135,6 +140,11 @@ template <int B>
 __device__ inline uint32_t unpack_pair(uint32_t w, int k) {
   constexpr uint32_t m = (1u << B) - 1u;
   return ((w >> (B * k)) & (m | (m << 16))) | 0x64006400u;
+}
+// 8-bit codes: one byte permute places bytes k and k+2 under the 0x64 exponent byte.
+template <>
+__device__ inline uint32_t unpack_pair<8>(uint32_t w, int k) {
+  return __byte_perm(w, 0x64646464u, k == 0 ? 0x4240u : 0x4341u);
 }
 
 // fp16 pair (1024 + 2^(b-1), same): subtracting it centres a code pair.

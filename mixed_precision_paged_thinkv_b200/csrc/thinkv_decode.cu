@@ -35,8 +35,12 @@ namespace {
 
 constexpr int kDecWarps = 4;
 constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecMinBlocks = 3;                       // CTAs per SM the kernel is built for
+constexpr int kDecRegs = 65536 / (kDecThreads * kDecMinBlocks) / 8 * 8;  // register cap (168)
 constexpr int kPbufStride = 12;                 // floats per row of the p transpose buffer
-constexpr int kPbufBytes = 16 * kPbufStride * 4;
+// per-warp scratch: the p transpose (16 x 12 floats) during pages, the
+// (m, l) table of a segment's pieces (32 x 8 float2 + 16 floats) in a merge
+constexpr int kPbufBytes = 2 * 32 * 8 * 4 + 16 * 4 + 64;
 constexpr int kSigmaInit = 1 << 20;
 constexpr int kCandCap = 128;                   // top-k candidate slots per head
 constexpr int kTopkHdrBytes = 64;               // per-head counts and thresholds
@@ -46,7 +50,7 @@ struct DecodeParams {
   int32_t phb[3];
   int32_t bits[3];
   const uint64_t* table;
-  const int32_t* live_list;
+  const uint64_t* live_list;
   const int32_t* num_live;
   int32_t max_blocks, max_seqs;
   int32_t Hkv, Hq, Gq;
@@ -146,79 +150,121 @@ __device__ inline int64_t piece_warp(int j, int64_t Us, int64_t w0, int64_t T, i
 }
 
 template <int D>
-__device__ void merge_segment(const DecodeParams& p, int i, int h, int64_t Us, int64_t w0,
-                              int np, int64_t T, int64_t W, const TopkCtx& tk) {
+__device__ void merge_segment(const DecodeParams& p, int i, int h, int64_t Us,
+                                           int64_t w0, int np, int64_t T, int64_t W,
+                                           const TopkCtx& tk, float* scratch) {
   const int lane = threadIdx.x & 31;
-  constexpr int PER = D / 32;
-  constexpr int BATCH = 8;
+  constexpr int QD = D / 4;                     // float4 quads per head row
+  constexpr int CH = 32;                        // pieces per chunk (scratch: 2 * CH * 8 floats)
   const int Gq = p.Gq;
   const int64_t seg = (int64_t)i * p.Hkv + h;
-  for (int r = 0; r < Gq; ++r) {
-    const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
-    // ---- running max and row sum: pieces across lanes ----
-    float mloc = -INFINITY;
-    for (int j = lane; j < np; j += 32)
-      mloc = fmaxf(mloc, __ldcg(&p.part_ml[((piece_warp(j, Us, w0, T, W) + seg) * Gq + r) * 2]));
+  const int npair = Gq * QD;
+  float2* ml = reinterpret_cast<float2*>(scratch);            // [CH][Gq] (m, l)
+  float* Mh = scratch + 2 * CH * 8;                           // [Gq] running max
+  float* Lh = Mh + 8;                                         // [Gq] row sums
+
+  // ---- pass 1: M per head over all pieces ----
+  if (lane < Gq) Mh[lane] = -INFINITY;
+  __syncwarp();
+  for (int jb = 0; jb < np; jb += CH) {
+    const int cnt = min(CH, np - jb);
+    for (int x = lane; x < cnt * Gq; x += 32) {
+      const int j = x / Gq, r = x - j * Gq;
+      const int64_t pc = (piece_warp(jb + j, Us, w0, T, W) + seg) * Gq + r;
+      ml[x] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + pc * 2));
+    }
+    __syncwarp();
+    if (lane < Gq) {
+      float mx = Mh[lane];
+      for (int j = 0; j < cnt; ++j) mx = fmaxf(mx, ml[j * Gq + lane].x);
+      Mh[lane] = mx;
+    }
+    __syncwarp();
+  }
+  // ---- pass 2: weights and row sums ----
+  if (lane < Gq) Lh[lane] = 0.f;
+  __syncwarp();
+  // (head, quad) pairs of this lane: lane + 32 x; done in groups of PG pairs,
+  // each over all pieces with BATCH pieces of independent loads in flight
+  constexpr int PG = 4, BATCH = 4;
+  const int npl = (npair + 31) / 32;
+  for (int x0 = 0; x0 < npl; x0 += PG) {
+    float4 acc[PG];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xFFFFFFFFu, mloc, o));
-    const float M = mloc;
-    float lloc = 0.f;
-    float acc[PER];
-#pragma unroll
-    for (int x = 0; x < PER; ++x) acc[x] = 0.f;
-    for (int jb = 0; jb < np; jb += 32) {
-      // this lane's piece of the chunk: weight f = 2^(m - M)
-      float f = 0.f;
-      if (jb + lane < np) {
-        const int64_t pc = (piece_warp(jb + lane, Us, w0, T, W) + seg) * Gq + r;
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + pc * 2));
-        f = exp2_approx(ml.x - M);
-        lloc = fmaf(ml.y, f, lloc);
+    for (int x = 0; x < PG; ++x) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int jb = 0; jb < np; jb += CH) {
+      const int cnt = min(CH, np - jb);
+      if (np > CH || x0 > 0) {  // (m, l) of this chunk (a single chunk is still in scratch)
+        for (int x = lane; x < cnt * Gq; x += 32) {
+          const int j = x / Gq, r = x - j * Gq;
+          const int64_t pc = (piece_warp(jb + j, Us, w0, T, W) + seg) * Gq + r;
+          ml[x] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + pc * 2));
+        }
+        __syncwarp();
       }
-      const int cnt = min(32, np - jb);
+      for (int x = lane; x < cnt * Gq; x += 32) ml[x].x = exp2_approx(ml[x].x - Mh[x % Gq]);
+      __syncwarp();
+      if (x0 == 0 && lane < Gq) {
+        float l = Lh[lane];
+        for (int j = 0; j < cnt; ++j) l = fmaf(ml[j * Gq + lane].y, ml[j * Gq + lane].x, l);
+        Lh[lane] = l;
+      }
       for (int jj = 0; jj < cnt; jj += BATCH) {
-        float vals[BATCH][PER];
+        float4 v[BATCH][PG];
 #pragma unroll
         for (int b = 0; b < BATCH; ++b) {
           if (jj + b < cnt) {
-            const int64_t pc = (piece_warp(jb + jj + b, Us, w0, T, W) + seg) * Gq + r;
-            const float* po = p.part_o + pc * D + lane * PER;
-            if constexpr (PER == 4) {
-              const float4 v = __ldcg(reinterpret_cast<const float4*>(po));
-              vals[b][0] = v.x; vals[b][1] = v.y; vals[b][2] = v.z; vals[b][3] = v.w;
-            } else {
-              const float2 v = __ldcg(reinterpret_cast<const float2*>(po));
-              vals[b][0] = v.x; vals[b][1] = v.y;
+            const int64_t base = (piece_warp(jb + jj + b, Us, w0, T, W) + seg) * Gq;
+#pragma unroll
+            for (int x = 0; x < PG; ++x) {
+              const int pr = lane + 32 * (x0 + x);
+              if (pr < npair) {
+                const int r = pr / QD, q = pr - r * QD;
+                v[b][x] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (base + r) * D) + q);
+              }
             }
           }
         }
 #pragma unroll
         for (int b = 0; b < BATCH; ++b) {
-          const float fb = __shfl_sync(0xFFFFFFFFu, f, (jj + b) & 31);
           if (jj + b < cnt) {
 #pragma unroll
-            for (int x = 0; x < PER; ++x) acc[x] = fmaf(vals[b][x], fb, acc[x]);
+            for (int x = 0; x < PG; ++x) {
+              const int pr = lane + 32 * (x0 + x);
+              if (pr < npair) {
+                const float fw = ml[(jj + b) * Gq + pr / QD].x;
+                acc[x].x = fmaf(v[b][x].x, fw, acc[x].x);
+                acc[x].y = fmaf(v[b][x].y, fw, acc[x].y);
+                acc[x].z = fmaf(v[b][x].z, fw, acc[x].z);
+                acc[x].w = fmaf(v[b][x].w, fw, acc[x].w);
+              }
+            }
           }
         }
       }
+      __syncwarp();
     }
+    // ---- fp16 output rows for this group of pairs ----
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lloc += __shfl_xor_sync(0xFFFFFFFFu, lloc, o);
-    const float inv = 1.f / lloc;
-    uint16_t* out = p.out + row * D + lane * PER;
-    if constexpr (PER == 4) {
-      const uint32_t a = (uint32_t)__half_as_ushort(__float2half_rn(acc[0] * inv)) |
-                         ((uint32_t)__half_as_ushort(__float2half_rn(acc[1] * inv)) << 16);
-      const uint32_t b = (uint32_t)__half_as_ushort(__float2half_rn(acc[2] * inv)) |
-                         ((uint32_t)__half_as_ushort(__float2half_rn(acc[3] * inv)) << 16);
-      *reinterpret_cast<uint2*>(out) = make_uint2(a, b);
-    } else {
-      *reinterpret_cast<uint32_t*>(out) =
-          (uint32_t)__half_as_ushort(__float2half_rn(acc[0] * inv)) |
-          ((uint32_t)__half_as_ushort(__float2half_rn(acc[1] * inv)) << 16);
+    for (int x = 0; x < PG; ++x) {
+      const int pr = lane + 32 * (x0 + x);
+      if (pr < npair) {
+        const int r = pr / QD, q = pr - r * QD;
+        const float inv = 1.f / Lh[r];
+        const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].x * inv)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].y * inv)) << 16);
+        const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].z * inv)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].w * inv)) << 16);
+        const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
+        reinterpret_cast<uint2*>(p.out + row * D)[q] = make_uint2(lo, hi);
+      }
     }
-
-    if (!p.mass) continue;
+  }
+  if (!p.mass) return;
+  for (int r = 0; r < Gq; ++r) {
+    const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
+    const float M = Mh[r];
+    const float inv = 1.f / Lh[r];
     const int k = p.topk;
     if (p.live_count[p.seq[i]] <= k) {
       if (lane == 0) p.mass[row] = 1.f;
@@ -313,8 +359,9 @@ struct SegState {
   float qsum[NG][2];                  // per-group sum of q for heads 2t, 2t+1
   float m[2], lp[2];                  // running max (log2 units), partial row sums
   float z[NG][2];                     // zero-term accumulators (heads 2t, 2t+1)
-  float acc[MT][4];                   // PV accumulators, units of 2^-sigma[group]
-  int sigma[NG];
+  float acc[MT][4];                   // PV accumulators, units of 2^-sigma
+  float accc[NG][2];                  // sum of W * (1024 + 2^(b-1)) per group (heads 2t, 2t+1)
+  int sigma;                          // W = p * s_V * 2^sigma is the fp16 PV operand
 };
 
 template <int D, int G>
@@ -343,8 +390,9 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i
     S.qsum[gr][0] = __shfl_sync(0xFFFFFFFFu, qs[gr], 8 * t);
     S.qsum[gr][1] = __shfl_sync(0xFFFFFFFFu, qs[gr], 8 * t + 4);
     S.z[gr][0] = S.z[gr][1] = 0.f;
-    S.sigma[gr] = kSigmaInit;
+    S.accc[gr][0] = S.accc[gr][1] = 0.f;
   }
+  S.sigma = kSigmaInit;               // the first page sets sigma
   S.m[0] = S.m[1] = -INFINITY;
   S.lp[0] = S.lp[1] = 0.f;
 #pragma unroll
@@ -361,7 +409,7 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i
 template <int D, int G>
 __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t piece,
                                const TopkCtx& tk, const int32_t* P, int i, int h, int64_t T,
-                               int64_t W) {
+                               int64_t W, float* scratch) {
   constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -386,14 +434,14 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
       }
     }
   }
+  const float inv = pow2i(-S.sigma);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int gr = (mt * 16) / G;
-    const float inv = pow2i(-S.sigma[gr]);
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       const int c = x & 1, ch = mt * 16 + g + 8 * (x >> 1), hd = 2 * t + c;
-      if (hd < Gq) po[hd * D + ch] = S.acc[mt][x] * inv + S.z[gr][c];
+      if (hd < Gq) po[hd * D + ch] = (S.acc[mt][x] - S.accc[gr][c]) * inv + S.z[gr][c];
     }
   }
   if (tk.topk > 0) {
@@ -418,11 +466,16 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
   old = __shfl_sync(0xFFFFFFFFu, old, 0);
   if (old == npieces - 1) {
     __threadfence();
-    merge_segment<D>(p, i, h, Us, w0, (int)npieces, T, W, tk);
+    merge_segment<D>(p, i, h, Us, w0, (int)npieces, T, W, tk, scratch);
   }
 }
 
 // One live page-head block (in shared memory) of a class with B-bit codes.
+//   QK: S^T[16 slots x 8 heads] = K(codes) x Q^T per group, with codes as
+//       fp16 (1024 + code); the 1024 offset folds into the group's zero term:
+//       q.k = s * sum q (1024 + c) + (z - 1024 s) * sum q.
+//   PV: O^T[16 channels x 8 heads] += V^T(codes - 2^(b-1)) x W per m-tile,
+//       W = p * s_V * 2^sigma rounded to fp16, plus sum p (z + 2^(b-1) s) in fp32.
 template <int D, int G, int B>
 __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
                                  float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
@@ -430,31 +483,33 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   constexpr int LANE_BYTES = D * B / 16;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const bool live0 = (mask >> g) & 1, live1 = (mask >> (g + 8)) & 1;
+  const uint32_t* kpar = reinterpret_cast<const uint32_t*>(blk + 4 * D * B);      // [NG][16]
+  const uint32_t* vpar = reinterpret_cast<const uint32_t*>(blk + 4 * D * B + 64 * NG);
 
-  // ---------------- logits: S^T = K(codes) x Q^T, per group ----------------
+  // ---------------- logits ----------------
   float lg[4] = {0.f, 0.f, 0.f, 0.f};
   {
     const uint8_t* kl = blk + lane * LANE_BYTES;
-    constexpr int PB = G * B / 32 > 0 ? G * B / 32 : 1;  // piece bytes
+    constexpr int PB = G * B / 32;                        // piece bytes (>= 2)
+    constexpr int NW = PB >= 4 ? PB / 4 : 1;              // words per piece
 #pragma unroll
     for (int gr = 0; gr < NG; ++gr) {
-      // the two pieces (rows gid and gid+8) of this group
-      uint32_t w[2][PB >= 4 ? PB / 4 : 1];
+      uint32_t w[2][NW];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const uint8_t* src = kl + (gr * 2 + r) * PB;
         if constexpr (PB == 2) {
-          uint32_t h16 = *reinterpret_cast<const uint16_t*>(src);
+          const uint32_t h16 = *reinterpret_cast<const uint16_t*>(src);
           w[r][0] = (h16 & 0xFFu) | ((h16 & 0xFF00u) << 8);  // bytes -> half-words
         } else if constexpr (PB == 4) {
           w[r][0] = *reinterpret_cast<const uint32_t*>(src);
         } else if constexpr (PB == 8) {
-          uint2 v = *reinterpret_cast<const uint2*>(src);
+          const uint2 v = *reinterpret_cast<const uint2*>(src);
           w[r][0] = v.x; w[r][1] = v.y;
         } else {
 #pragma unroll
           for (int x = 0; x < PB / 16; ++x) {
-            uint4 v = *reinterpret_cast<const uint4*>(src + 16 * x);
+            const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * x);
             w[r][4 * x] = v.x; w[r][4 * x + 1] = v.y; w[r][4 * x + 2] = v.z; w[r][4 * x + 3] = v.w;
           }
         }
@@ -465,17 +520,15 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
         uint32_t a[4];
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
-          const int u = 2 * s + hi;  // pair index inside the piece
+          const int u = 2 * s + hi;                          // pair index inside the piece
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            uint32_t reg;
             if constexpr (B == 16) {
-              reg = w[r][u];
+              a[hi * 2 + r] = w[r][u];
             } else {
               constexpr int PAIRS = (PB == 2 ? 4 : 16 / B);  // pairs per (spread) word
-              reg = hsub2_bits(unpack_pair<B>(w[r][u / PAIRS], u % PAIRS), centre_bits<B>());
+              a[hi * 2 + r] = unpack_pair<B>(w[r][u / PAIRS], u % PAIRS);
             }
-            a[hi * 2 + r] = reg;
           }
         }
         mma_16816(c, a, S.qf[gr][s][0], S.qf[gr][s][1]);
@@ -483,26 +536,21 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
       if constexpr (B == 16) {
         lg[0] += c[0]; lg[1] += c[1]; lg[2] += c[2]; lg[3] += c[3];
       } else {
-        const uint16_t* kp = reinterpret_cast<const uint16_t*>(blk + 4 * D * B);
-        const uint32_t p0 = *reinterpret_cast<const uint32_t*>(kp + (g * NG + gr) * 2);
-        const uint32_t p1 = *reinterpret_cast<const uint32_t*>(kp + ((g + 8) * NG + gr) * 2);
-        const float s0 = __half2float(__ushort_as_half(p0 & 0xFFFF));
-        const float z0 = __half2float(__ushort_as_half(p0 >> 16));
-        const float s1 = __half2float(__ushort_as_half(p1 & 0xFFFF));
-        const float z1 = __half2float(__ushort_as_half(p1 >> 16));
-        const float zc0 = fmaf((float)(1 << (B - 1)), s0, z0);
-        const float zc1 = fmaf((float)(1 << (B - 1)), s1, z1);
-        lg[0] += fmaf(s0, c[0], zc0 * S.qsum[gr][0]);
-        lg[1] += fmaf(s0, c[1], zc0 * S.qsum[gr][1]);
-        lg[2] += fmaf(s1, c[2], zc1 * S.qsum[gr][0]);
-        lg[3] += fmaf(s1, c[3], zc1 * S.qsum[gr][1]);
+        const uint32_t p0 = kpar[gr * 16 + g], p1 = kpar[gr * 16 + g + 8];
+        const float2 sz0 = __half22float2(*reinterpret_cast<const __half2*>(&p0));  // (s, z)
+        const float2 sz1 = __half22float2(*reinterpret_cast<const __half2*>(&p1));
+        const float zc0 = fmaf(-1024.f, sz0.x, sz0.y), zc1 = fmaf(-1024.f, sz1.x, sz1.y);
+        lg[0] = fmaf(sz0.x, c[0], fmaf(zc0, S.qsum[gr][0], lg[0]));
+        lg[1] = fmaf(sz0.x, c[1], fmaf(zc0, S.qsum[gr][1], lg[1]));
+        lg[2] = fmaf(sz1.x, c[2], fmaf(zc1, S.qsum[gr][0], lg[2]));
+        lg[3] = fmaf(sz1.x, c[3], fmaf(zc1, S.qsum[gr][1], lg[3]));
       }
     }
   }
-#pragma unroll
-  for (int x = 0; x < 4; ++x) lg[x] *= scale_log2;
-  if (!live0) lg[0] = lg[1] = -INFINITY;
-  if (!live1) lg[2] = lg[3] = -INFINITY;
+  lg[0] = live0 ? lg[0] * scale_log2 : -INFINITY;
+  lg[1] = live0 ? lg[1] * scale_log2 : -INFINITY;
+  lg[2] = live1 ? lg[2] * scale_log2 : -INFINITY;
+  lg[3] = live1 ? lg[3] * scale_log2 : -INFINITY;
 
   // ---------------- top-k candidates (logits above the head's threshold) ----------------
   if (tk.topk > 0) {
@@ -542,18 +590,14 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   S.lp[0] = fmaf(S.lp[0], a0, pr[0] + pr[2]);
   S.lp[1] = fmaf(S.lp[1], a1, pr[1] + pr[3]);
 
-  const uint16_t* vpar = reinterpret_cast<const uint16_t*>(blk + 4 * D * B + 64 * NG);
   if constexpr (B != 16) {
 #pragma unroll
     for (int gr = 0; gr < NG; ++gr) {
-      const uint32_t p0 = *reinterpret_cast<const uint32_t*>(vpar + (g * NG + gr) * 2);
-      const uint32_t p1 = *reinterpret_cast<const uint32_t*>(vpar + ((g + 8) * NG + gr) * 2);
-      float zv0 = fmaf((float)(1 << (B - 1)), __half2float(__ushort_as_half(p0 & 0xFFFF)),
-                       __half2float(__ushort_as_half(p0 >> 16)));
-      float zv1 = fmaf((float)(1 << (B - 1)), __half2float(__ushort_as_half(p1 & 0xFFFF)),
-                       __half2float(__ushort_as_half(p1 >> 16)));
-      zv0 = live0 ? zv0 : 0.f;
-      zv1 = live1 ? zv1 : 0.f;
+      const uint32_t p0 = vpar[gr * 16 + g], p1 = vpar[gr * 16 + g + 8];
+      const float2 sz0 = __half22float2(*reinterpret_cast<const __half2*>(&p0));
+      const float2 sz1 = __half22float2(*reinterpret_cast<const __half2*>(&p1));
+      const float zv0 = live0 ? fmaf((float)(1 << (B - 1)), sz0.x, sz0.y) : 0.f;
+      const float zv1 = live1 ? fmaf((float)(1 << (B - 1)), sz1.x, sz1.y) : 0.f;
       S.z[gr][0] = fmaf(S.z[gr][0], a0, fmaf(pr[0], zv0, pr[2] * zv1));
       S.z[gr][1] = fmaf(S.z[gr][1], a1, fmaf(pr[1], zv0, pr[3] * zv1));
     }
@@ -569,81 +613,99 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   pt[1] = pbuf[(2 * t + 1) * kPbufStride + g];
   pt[2] = pbuf[(2 * t + 8) * kPbufStride + g];
   pt[3] = pbuf[(2 * t + 9) * kPbufStride + g];
-  const int tok[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
-  bool tl[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) tl[j] = (mask >> tok[j]) & 1;
+  const uint32_t tmask = mask >> (2 * t);
+  const bool tl[4] = {(tmask & 1u) != 0, (tmask & 2u) != 0, (tmask & 0x100u) != 0,
+                      (tmask & 0x200u) != 0};
 
-  // ---------------- per-group B fragments W = p * s_V * 2^sigma ----------------
-  uint32_t wf[NG][2];
-  float fac[NG];
-  bool rescale = (a0 != 1.f) || (a1 != 1.f);
+  // ---------------- PV operands W = p * s_V * 2^sigma (one sigma per segment) ----------------
+  float sv[NG][4];
 #pragma unroll
   for (int gr = 0; gr < NG; ++gr) {
-    float sv[4];
-    int e5 = 0;
+    if constexpr (B == 16) {
+      sv[gr][0] = sv[gr][1] = sv[gr][2] = sv[gr][3] = 1.f;
+    } else {
+      const uint2 q0 = *reinterpret_cast<const uint2*>(vpar + gr * 16 + 2 * t);
+      const uint2 q1 = *reinterpret_cast<const uint2*>(vpar + gr * 16 + 2 * t + 8);
+      sv[gr][0] = __half2float(__ushort_as_half((uint16_t)(q0.x & 0xFFFFu)));
+      sv[gr][1] = __half2float(__ushort_as_half((uint16_t)(q0.y & 0xFFFFu)));
+      sv[gr][2] = __half2float(__ushort_as_half((uint16_t)(q1.x & 0xFFFFu)));
+      sv[gr][3] = __half2float(__ushort_as_half((uint16_t)(q1.y & 0xFFFFu)));
+    }
+  }
+  // dead slots: p is 0, their scale bytes are stale; zero the packed operand instead
+  const uint32_t dm0 = (tl[0] ? 0xFFFFu : 0u) | (tl[1] ? 0xFFFF0000u : 0u);
+  const uint32_t dm1 = (tl[2] ? 0xFFFFu : 0u) | (tl[3] ? 0xFFFF0000u : 0u);
+  float f = S.sigma == kSigmaInit ? 0.f : pow2i(S.sigma);
+  float wv[NG][4];
+  float wmax = 0.f;
+#pragma unroll
+  for (int gr = 0; gr < NG; ++gr)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      if constexpr (B == 16) {
-        sv[j] = 1.f;
-        e5 = 15;
-      } else {
-        const uint16_t sb = vpar[(tok[j] * NG + gr) * 2];
-        sv[j] = __half2float(__ushort_as_half(sb));
-        const int ef = max((int)((sb >> 10) & 31), 1);
+      wv[gr][j] = pt[j] * f * sv[gr][j];
+      wmax = tl[j] ? fmaxf(wmax, wv[gr][j]) : wmax;
+    }
+  float fac = 1.f;
+  // slow path: first page of the segment, or a scale large enough to overflow fp16
+  if (__any_sync(0xFFFFFFFFu, S.sigma == kSigmaInit || !(wmax < 32768.f))) {
+    int e5 = 1;
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int ef = (__float_as_int(sv[gr][j]) >> 23) - 112;  // fp16 exponent field
         e5 = tl[j] ? max(e5, ef) : e5;
       }
+    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 1));
+    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 2));
+    const int sp = 29 - e5;             // s * 2^sp < 2^15 for every live scale of the page
+    if (sp < S.sigma) {
+      if (S.sigma != kSigmaInit) fac = pow2i(sp - S.sigma);
+      S.sigma = sp;
     }
-    if constexpr (B != 16) {
-      e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 1));
-      e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 2));
-    }
-    const int sp = 29 - e5;  // s * 2^sp < 2^15, so p * s * 2^sigma fits in fp16
-    fac[gr] = 1.f;
-    if (sp < S.sigma[gr]) {
-      if (S.sigma[gr] != kSigmaInit) {
-        fac[gr] = pow2i(sp - S.sigma[gr]);
-        rescale = true;
-      }
-      S.sigma[gr] = sp;
-    }
-    const float f = pow2i(S.sigma[gr]);
-    float wv[4];
+    f = pow2i(S.sigma);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) wv[j] = tl[j] ? pt[j] * sv[j] * f : 0.f;
-    wf[gr][0] = pack_half2_rn(wv[0], wv[1]);
-    wf[gr][1] = pack_half2_rn(wv[2], wv[3]);
+    for (int gr = 0; gr < NG; ++gr)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wv[gr][j] = pt[j] * f * sv[gr][j];
   }
-  if (__any_sync(0xFFFFFFFFu, rescale)) {
+  uint32_t wf[NG][2];
+#pragma unroll
+  for (int gr = 0; gr < NG; ++gr) {
+    wf[gr][0] = pack_half2_rn(wv[gr][0], wv[gr][1]) & dm0;
+    wf[gr][1] = pack_half2_rn(wv[gr][2], wv[gr][3]) & dm1;
+  }
+  if (__any_sync(0xFFFFFFFFu, a0 != 1.f || a1 != 1.f || fac != 1.f)) {
+    const float r0 = a0 * fac, r1 = a1 * fac;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      const float f = fac[(mt * 16) / G];
-      S.acc[mt][0] *= a0 * f;
-      S.acc[mt][1] *= a1 * f;
-      S.acc[mt][2] *= a0 * f;
-      S.acc[mt][3] *= a1 * f;
+      S.acc[mt][0] *= r0;
+      S.acc[mt][1] *= r1;
+      S.acc[mt][2] *= r0;
+      S.acc[mt][3] *= r1;
+    }
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr) {
+      S.accc[gr][0] *= r0;
+      S.accc[gr][1] *= r1;
     }
   }
 
-  // ---------------- O^T += V^T(codes) x W ----------------
+  // ---------------- O^T += V^T(1024 + codes) x W ----------------
   {
-    constexpr int Q = D * B / 128 > 0 ? D * B / 128 : 1;  // words per token pair
-    constexpr int PER = 16 / B;                          // codes per half-word
-    const uint32_t* vw = reinterpret_cast<const uint32_t*>(blk + 2 * D * B + lane * LANE_BYTES);
+    constexpr int Q = (B == 16) ? D / 8 : D * B / 128;   // words per token pair
+    constexpr int PER = (B == 16) ? 1 : 16 / B;          // codes per half-word
+    const uint8_t* vl = blk + 2 * D * B + lane * LANE_BYTES;
     uint32_t vr[2 * Q];
+    if constexpr ((2 * Q) % 4 == 0) {
 #pragma unroll
-    for (int x = 0; x < (2 * Q) / 4; ++x) {
-      uint4 v = reinterpret_cast<const uint4*>(vw)[x];
-      vr[4 * x] = v.x; vr[4 * x + 1] = v.y; vr[4 * x + 2] = v.z; vr[4 * x + 3] = v.w;
-    }
-    if constexpr ((2 * Q) % 4 == 2) {
-      uint2 v = reinterpret_cast<const uint2*>(vw)[(2 * Q) / 2 - 1];
-      vr[2 * Q - 2] = v.x; vr[2 * Q - 1] = v.y;
-    }
-    uint32_t dead_mask[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
-    if constexpr (B == 16) {
-      dead_mask[0] = (tl[0] ? 0xFFFFu : 0u) | (tl[1] ? 0xFFFF0000u : 0u);
-      dead_mask[1] = (tl[2] ? 0xFFFFu : 0u) | (tl[3] ? 0xFFFF0000u : 0u);
+      for (int x = 0; x < (2 * Q) / 4; ++x) {
+        const uint4 v = reinterpret_cast<const uint4*>(vl)[x];
+        vr[4 * x] = v.x; vr[4 * x + 1] = v.y; vr[4 * x + 2] = v.z; vr[4 * x + 3] = v.w;
+      }
+    } else {
+      const uint2 v = *reinterpret_cast<const uint2*>(vl);
+      vr[0] = v.x; vr[1] = v.y;
     }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
@@ -654,16 +716,25 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int e = 2 * mt + r;
-          uint32_t reg;
           if constexpr (B == 16) {
-            reg = vr[P * Q + e] & dead_mask[P];
+            a[P * 2 + r] = vr[P * Q + e] & (P ? dm1 : dm0);  // raw values of dead slots: zero
           } else {
-            reg = hsub2_bits(unpack_pair<B>(vr[P * Q + e / PER], e % PER), centre_bits<B>());
+            a[P * 2 + r] = unpack_pair<B>(vr[P * Q + e / PER], e % PER);
           }
-          a[P * 2 + r] = reg;
         }
       }
       mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
+    }
+    if constexpr (B != 16) {
+      // the code offset 1024 + 2^(b-1): one constant-row product per group
+      const uint32_t ka[4] = {centre_bits<B>(), centre_bits<B>(), centre_bits<B>(), centre_bits<B>()};
+#pragma unroll
+      for (int gr = 0; gr < NG; ++gr) {
+        float cc[4] = {S.accc[gr][0], S.accc[gr][1], S.accc[gr][0], S.accc[gr][1]};
+        mma_16816(cc, ka, wf[gr][0], wf[gr][1]);
+        S.accc[gr][0] = cc[0];
+        S.accc[gr][1] = cc[1];
+      }
     }
   }
 }
@@ -679,23 +750,21 @@ __device__ inline void page_dispatch(SegState<D, G>& S, const uint8_t* blk, int 
   }
 }
 
-// Everything a lane needs to know about one unit (sequence, kv-head, live page).
+// What a lane knows about one unit (sequence, kv-head, live page): the page-head
+// block's address, its class and segment (seg = i * Hkv + h), and the page's
+// live mask.  The mask is loaded last and only needed once the page is computed.
 struct UnitMeta {
-  const uint8_t* src;
-  int32_t seg;       // i * Hkv + h
-  int32_t i;         // index into the call's sequences
-  int32_t h;
-  uint32_t cls_mask; // class << 16 | live mask
+  uint32_t src_lo, src_hi;
+  uint32_t cls_seg;   // class << 24 | segment
+  uint32_t mask;
 };
 
 __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P, int64_t u,
                                         int64_t U1) {
   UnitMeta m;
-  m.src = nullptr;
-  m.seg = -1;
-  m.i = 0;
-  m.h = 0;
-  m.cls_mask = 0;
+  m.src_lo = m.src_hi = 0;
+  m.cls_seg = 0;
+  m.mask = 0;
   if (u >= U1) return m;
   int lo = 0, hi = p.n;
   while (hi - lo > 1) {
@@ -704,33 +773,22 @@ __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P,
   }
   const int i = lo;
   const int nl = P[i + 1] - P[i];
-  const int64_t rel = u - (int64_t)P[i] * p.Hkv;
-  const int h = (int)(rel / nl), j = (int)(rel % nl);
-  const int s = p.seq[i];
-  const int e = p.live_list[(int64_t)s * p.max_blocks + j];
-  const uint64_t ent = p.table[(int64_t)s * p.max_blocks + e];
-  const int cls = entry_class(ent);
-  m.src = p.pool[cls] + ((int64_t)entry_page(ent) * p.Hkv + h) * p.phb[cls];
-  m.seg = i * p.Hkv + h;
-  m.i = i;
-  m.h = h;
-  m.cls_mask = ((uint32_t)cls << 16) | entry_mask(ent);
+  const int rel = (int)(u - (int64_t)P[i] * p.Hkv);   // < Hkv * max_blocks_per_seq < 2^31
+  const int h = rel / nl, j = rel - h * nl;
+  const int64_t row = (int64_t)p.seq[i] * p.max_blocks;
+  const uint64_t desc = p.live_list[row + j];       // page | class << 32 | entry << 40
+  const int cls = entry_class(desc);
+  const uint64_t src = reinterpret_cast<uint64_t>(p.pool[cls]) +
+                       ((uint64_t)entry_page(desc) * p.Hkv + h) * (uint64_t)p.phb[cls];
+  m.src_lo = (uint32_t)src;
+  m.src_hi = (uint32_t)(src >> 32);
+  m.cls_seg = ((uint32_t)cls << 24) | (uint32_t)(i * p.Hkv + h);
+  m.mask = entry_mask(p.table[row + live_desc_entry(desc)]);
   return m;
 }
 
-__device__ inline UnitMeta shfl_meta(const UnitMeta& m, int src) {
-  UnitMeta r;
-  r.src = reinterpret_cast<const uint8_t*>(
-      __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(m.src), src));
-  r.seg = __shfl_sync(0xFFFFFFFFu, m.seg, src);
-  r.i = __shfl_sync(0xFFFFFFFFu, m.i, src);
-  r.h = __shfl_sync(0xFFFFFFFFu, m.h, src);
-  r.cls_mask = __shfl_sync(0xFFFFFFFFu, m.cls_mask, src);
-  return r;
-}
-
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, 3)
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_split_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -798,57 +856,66 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   // prologue: fill the ring
   const int64_t nunits = U1 - U0;
   for (int s = 0; s < p.nstage && s < nunits; ++s) {
-    const UnitMeta m = shfl_meta(cur, s);  // nstage <= 8 < 32
+    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, cur.src_lo, s);
+    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, cur.src_hi, s);
+    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, s);
     if (lane == 0) {
-      const uint32_t bytes = (uint32_t)p.phb[m.cls_mask >> 16];
+      const uint32_t bytes = (uint32_t)p.phb[cs >> 24];
       mbar_arrive_expect_tx(&bars[s], bytes);
-      bulk_g2s(wsm + s * p.stage_bytes, m.src, bytes, &bars[s]);
+      bulk_g2s(wsm + s * p.stage_bytes,
+               reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[s]);
     }
   }
 
   SegState<D, G> S;
-  int seg = -1, cur_i = 0, cur_h = 0;
-  for (int64_t k = 0; k < nunits; ++k) {
-    const int kk = (int)(k & 31);
+  int seg = -1;
+  int stage = 0;
+  uint32_t parity = 0;
+  const int nu = (int)nunits;   // units of one warp: < 2^31
+  for (int k = 0; k < nu; ++k) {
+    const int kk = k & 31;
     if (kk == 0 && k > 0) {
       cur = nxt;
       nxt = resolve_unit(p, P, U0 + k + 32 + lane, U1);
     }
-    const UnitMeta m = shfl_meta(cur, kk);
-    if (m.seg != seg) {
-      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, cur_i, cur_h, T, W);
-      seg = m.seg;
-      cur_i = m.i;
-      cur_h = m.h;
-      seg_begin<D, G>(S, p, m.i, m.h, tk);
+    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, kk);
+    const int useg = (int)(cs & 0xFFFFFFu);
+    if (useg != seg) {
+      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, seg / p.Hkv, seg % p.Hkv, T, W, pbuf);
+      seg = useg;
+      seg_begin<D, G>(S, p, seg / p.Hkv, seg % p.Hkv, tk);
     }
-    const int stage = (int)(k % p.nstage);
-    const uint32_t parity = (uint32_t)((k / p.nstage) & 1);
     if (!mbar_wait_bounded(&bars[stage], parity)) {
       if (lane == 0) set_status(p.status, THINKV_ERR_TIMEOUT);
       // drain the copies still in flight (bounded), then leave
-      for (int64_t k2 = k + 1; k2 < nunits && k2 < k + p.nstage; ++k2)
+      for (int k2 = k + 1; k2 < nu && k2 < k + p.nstage; ++k2)
         mbar_wait_bounded(&bars[k2 % p.nstage], (uint32_t)((k2 / p.nstage) & 1));
       return;
     }
-    const int cls = (int)(m.cls_mask >> 16);
-    page_dispatch<D, G>(S, wsm + stage * p.stage_bytes, p.bits[cls], m.cls_mask & 0xFFFFu,
+    const uint32_t mask = __shfl_sync(0xFFFFFFFFu, cur.mask, kk);
+    page_dispatch<D, G>(S, wsm + stage * p.stage_bytes, p.bits[cs >> 24], mask & 0xFFFFu,
                         p.scale_log2, pbuf, tk, p.Gq);
     __syncwarp();
-    // refill this stage with unit k + nstage
-    const int64_t kn = k + p.nstage;
-    const int srcl = (int)(kn & 31);
-    const UnitMeta ma = shfl_meta(cur, srcl);
-    const UnitMeta mb = shfl_meta(nxt, srcl);
-    const UnitMeta& mn = ((kn >> 5) == (k >> 5)) ? ma : mb;
-    if (lane == 0 && kn < nunits) {
+    // refill this stage with unit k + nstage (from this batch of 32 or the next)
+    const int kn = k + p.nstage;
+    const bool same = (kn >> 5) == (k >> 5);
+    const int srcl = kn & 31;
+    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, same ? cur.src_lo : nxt.src_lo, srcl);
+    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, same ? cur.src_hi : nxt.src_hi, srcl);
+    const uint32_t ncs = __shfl_sync(0xFFFFFFFFu, same ? cur.cls_seg : nxt.cls_seg, srcl);
+    if (lane == 0 && kn < nu) {
       fence_proxy_async_smem();
-      const uint32_t bytes = (uint32_t)p.phb[mn.cls_mask >> 16];
+      const uint32_t bytes = (uint32_t)p.phb[ncs >> 24];
       mbar_arrive_expect_tx(&bars[stage], bytes);
-      bulk_g2s(wsm + stage * p.stage_bytes, mn.src, bytes, &bars[stage]);
+      bulk_g2s(wsm + stage * p.stage_bytes,
+               reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[stage]);
+    }
+    if (++stage == p.nstage) {
+      stage = 0;
+      parity ^= 1u;
     }
   }
-  if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, cur_i, cur_h, T, W);
+  if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, seg / p.Hkv, seg % p.Hkv, T, W, pbuf);
 }
 
 template <int D, int G>
@@ -882,7 +949,8 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
     if (b > maxphb) maxphb = b;
   }
   const int stage_bytes = (int)((maxphb + 127) / 128 * 128);
-  int nstage = (int)(18432 / stage_bytes);
+  // ~15 KB of page-head stages per warp keeps three 4-warp CTAs per SM
+  int nstage = (int)(15360 / stage_bytes);
   if (nstage < 2) nstage = 2;
   if (nstage > 8) nstage = 8;
   const int Gq = L.num_q_heads / L.num_kv_heads;
@@ -899,8 +967,14 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
   if (cudaDeviceGetAttribute(&smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
       cudaSuccess)
     return false;
-  // CTAs per SM limited by shared memory (1 KB reserved per CTA) and threads
+  // CTAs per SM: limited by shared memory (1 KB reserved per CTA) and by registers
   int per_sm = smem_per_sm / (int)(smem + 1024);
+  int regs_per_sm = 0;
+  if (cudaDeviceGetAttribute(&regs_per_sm, cudaDevAttrMaxRegistersPerMultiprocessor, device) !=
+      cudaSuccess)
+    return false;
+  const int by_regs = regs_per_sm / (kDecRegs * kDecThreads);
+  if (per_sm > by_regs) per_sm = by_regs;
   if (per_sm > 16) per_sm = 16;
   if (per_sm < 1) per_sm = 1;
   out->grid = sms * per_sm;

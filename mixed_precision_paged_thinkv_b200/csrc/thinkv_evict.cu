@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kEvictThreads, 1)
     int remaining = C.live_count[s] - budget[i];
     if (remaining <= 0) continue;
     uint64_t* table = C.block_table + (int64_t)s * nb_max;
-    int32_t* llist = C.live_list + (int64_t)s * nb_max;
+    uint64_t* llist = C.live_list + (int64_t)s * nb_max;
     int32_t* lidx = C.live_index + (int64_t)s * nb_max;
     int nlive = C.num_live[s];
     int evicted = 0;
@@ -107,9 +107,9 @@ __global__ void __launch_bounds__(kEvictThreads, 1)
           if (lane == 0) {
             const int at = lidx[ee];
             const int lastpos = --nlive;
-            const int moved = llist[lastpos];
+            const uint64_t moved = llist[lastpos];
             llist[at] = moved;
-            lidx[moved] = at;
+            lidx[live_desc_entry(moved)] = at;
             lidx[ee] = -1;
           }
           nlive = __shfl_sync(0xFFFFFFFFu, nlive, 0);

@@ -22,7 +22,7 @@ struct CacheView {
   int32_t* fifo_head;
   int32_t* fifo_tail;
   int32_t* live_count;
-  int32_t* live_list;
+  uint64_t* live_list;
   int32_t* live_index;
   int32_t* num_live;
   int32_t* page_bump;

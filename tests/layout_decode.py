@@ -9,8 +9,9 @@ the oracle's natural [slot][channel] codes:
   V codes: lane l owns words (P, q); word (P, q) has slot 2*tid + 8P in its low
     half and slot 2*tid + 8P + 1 in its high half, element k of each half being
     channel 16*(e//2) + gid + 8*(e%2), e = q*16/b + k;
+  params are [group][slot][scale, zero] fp16;
   inside a 32-bit word (or a 16-bit piece) even channels fill the low half and
-  odd channels the high half, little-endian; params [slot][group][scale, zero].
+  odd channels the high half, little-endian.
 """
 from functools import lru_cache
 
@@ -84,6 +85,7 @@ def decode_blocks(blocks: np.ndarray, d: int, G: int, b: int):
     vc = ((blocks[..., vb] >> vs) & mask).astype(np.uint8)
     ng = d // G
     po = 4 * d * b
-    kp = blocks[..., po:po + 64 * ng].copy().view(np.uint16).reshape(blocks.shape[:-1] + (PAGE, ng, 2))
-    vp = blocks[..., po + 64 * ng:po + 128 * ng].copy().view(np.uint16).reshape(blocks.shape[:-1] + (PAGE, ng, 2))
-    return kc, vc, kp, vp
+    # params are stored [group][slot][scale, zero]; returned as [slot][group][2]
+    kp = blocks[..., po:po + 64 * ng].copy().view(np.uint16).reshape(blocks.shape[:-1] + (ng, PAGE, 2))
+    vp = blocks[..., po + 64 * ng:po + 128 * ng].copy().view(np.uint16).reshape(blocks.shape[:-1] + (ng, PAGE, 2))
+    return kc, vc, np.swapaxes(kp, -3, -2), np.swapaxes(vp, -3, -2)
