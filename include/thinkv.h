@@ -20,7 +20,9 @@
  * Conventions for every entry point
  *   - All array arguments are DEVICE pointers owned by the caller, except the
  *     ones documented as host arrays.  The library allocates nothing and keeps
- *     no global state.  fp16 values travel as uint16_t bit patterns.
+ *     no global state, apart from the fixed scratch array of
+ *     thinkv_decode_attention_noalloc.  fp16 values travel as uint16_t bit
+ *     patterns.
  *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous
  *     on it.
  *   - Host-checkable errors (bad layout, null pointers, sizes) return a
@@ -243,6 +245,32 @@ THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs
                             const uint16_t* q, uint16_t* out, float* topk_mass,
                             int32_t topk, float softmax_scale,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Size of the library-owned scratch of thinkv_decode_attention_noalloc. */
+#define THINKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* Decode attention without a caller-provided workspace -- the same operation,
+ * arguments and results as thinkv_decode_attention, for callers that cannot
+ * allocate device memory at the point where they decode: code running inside
+ * a host framework that owns every device allocation and hands its plugins no
+ * allocator, or latency-critical paths where cudaMalloc's implicit device-wide
+ * synchronisation is not acceptable.  (The ThinKV pages have no counterpart;
+ * this is an interface convenience of this library.)
+ * The split-K scratch lives in one file-scope device array of
+ * THINKV_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
+ * until the process exits.  A call whose scratch need (what
+ * thinkv_decode_workspace_bytes reports for the same n_seqs and topk) exceeds
+ * that size returns THINKV_ERR_WORKSPACE before launching anything.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Each call clears the array's arrival counters on `stream`, and
+ * calls share the array: two calls that overlap on the GPU (different streams,
+ * or different host threads) race and must not be issued.  Nothing is
+ * allocated or freed. */
+THINKV_API int thinkv_decode_attention_noalloc(const thinkv_cache* cache, int32_t n_seqs,
+                                               const int32_t* seq, const uint16_t* q,
+                                               uint16_t* out, float* topk_mass, int32_t topk,
+                                               float softmax_scale, void* stream);
 
 /* Synchronises `stream`, then copies *status to *out (host). */
 THINKV_API int thinkv_get_status(const thinkv_cache* cache, void* stream, int32_t* out);

@@ -33,6 +33,7 @@ EXPORTED = [
     "thinkv_cache_reset", "thinkv_append_workspace_bytes", "thinkv_append_quantize",
     "thinkv_evict", "thinkv_decode_workspace_bytes", "thinkv_decode_attention",
     "thinkv_get_status", "thinkv_clear_status", "thinkv_status_string",
+    "thinkv_decode_attention_noalloc",
 ]
 
 

@@ -14,7 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libthinkv.so")
-SOURCES = ["thinkv_api.cu", "thinkv_append.cu", "thinkv_evict.cu", "thinkv_decode.cu"]
+SOURCES = ["thinkv_api.cu", "thinkv_append.cu", "thinkv_evict.cu", "thinkv_decode.cu",
+           "thinkv_noalloc.cu"]
 HEADERS = ["thinkv_common.cuh", "thinkv_internal.h"]
 
 NVCC_FLAGS = [

@@ -37,6 +37,10 @@ bool layout_ok(const thinkv_layout* L) {
   return true;
 }
 
+}  // namespace
+
+namespace thinkv {
+
 bool cache_ok(const thinkv_cache* C) {
   if (!C || !layout_ok(&C->L)) return false;
   for (int c = 0; c < 3; ++c)
@@ -68,6 +72,10 @@ CacheView view_of(const thinkv_cache* C) {
   v.status = C->status;
   return v;
 }
+
+}  // namespace thinkv
+
+namespace {
 
 int num_sms_current() {
   static int cached[64] = {0};

@@ -53,6 +53,10 @@ cudaError_t launch_append(const CacheView& C, int32_t n, const int32_t* seq, con
 cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
                          const uint8_t order[3], cudaStream_t stream);
 
+// host-side checks shared by the entry points
+bool cache_ok(const thinkv_cache* C);
+CacheView view_of(const thinkv_cache* C);
+
 // decode
 struct DecodeLaunch {
   int grid;            // CTAs of the split kernel
