@@ -37,7 +37,8 @@ if ROOT not in sys.path:
 METRIC = "decode-attention tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
 DEFAULT_WORKLOAD = "r1-llama-8b"
 FLUSH_BYTES = 512 << 20
-DECODE_SRC = os.path.join(ROOT, "mixed_precision_paged_thinkv_b200", "csrc", "thinkv_decode.cu")
+DECODE_SRC = [os.path.join(ROOT, "mixed_precision_paged_thinkv_b200", "csrc", f)
+              for f in ("thinkv_decode.cu", "thinkv_common.cuh", "thinkv_internal.h")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 
@@ -89,8 +90,12 @@ def peak_hbm_gbs():
 
 
 def decode_source_hash() -> str:
-    with open(DECODE_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the sources the decode kernel is compiled from."""
+    h = hashlib.sha256()
+    for p in DECODE_SRC:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_per_launch(workload: str):

@@ -85,9 +85,24 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of phase `parity`.
+__device__ inline bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` with an iteration bound; false if the bound ran out.
+// The non-blocking probe answers at once when the data has already landed.
 constexpr uint32_t kWaitLimit = 1u << 22;
 __device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_test_wait(bar, parity)) return true;
   for (uint32_t it = 0; it < kWaitLimit; ++it)
     if (mbar_try_wait(bar, parity)) return true;
   return false;

@@ -38,9 +38,14 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecMinBlocks = 3;                       // CTAs per SM the kernel is built for
 constexpr int kDecRegs = 65536 / (kDecThreads * kDecMinBlocks) / 8 * 8;  // register cap (168)
 constexpr int kPbufStride = 12;                 // floats per row of the p transpose buffer
-// per-warp scratch: the p transpose (16 x 12 floats) during pages, the
-// (m, l) table of a segment's pieces (32 x 8 float2 + 16 floats) in a merge
-constexpr int kPbufBytes = 2 * 32 * 8 * 4 + 16 * 4 + 64;
+// per-warp scratch: during pages, the p transpose (16 x 12 floats) and the
+// segment's Q fragments (lane-contiguous, up to 2 KB); during a merge, which
+// runs between two segments, the (m, l) table of the pieces (32 x 8 float2 +
+// 16 floats) overlays both
+constexpr int kPtBytes = 16 * kPbufStride * 4;          // 768
+constexpr int kQfragOff = kPtBytes;
+constexpr int kQfragBytes = 2048;                       // (D / 16) k-steps x 32 lanes x 8 B
+constexpr int kPbufBytes = kPtBytes + kQfragBytes;      // >= 2 * 32 * 8 * 4 + 16 * 4
 constexpr int kSigmaInit = 1 << 20;
 constexpr int kCandCap = 128;                   // top-k candidate slots per head
 constexpr int kTopkHdrBytes = 64;               // per-head counts and thresholds
@@ -68,6 +73,7 @@ struct DecodeParams {
   int32_t topk;
   int32_t* status;
   int32_t nstage, stage_bytes, warp_smem, plan_smem;
+  int32_t q_off, q_bytes;  // Q rows of a segment ride with its first page: stage + q_off
 };
 
 __device__ inline float pow2i(int e) { return __int_as_float((127 + e) << 23); }
@@ -355,22 +361,20 @@ struct SegState {
   static constexpr int NG = D / G;
   static constexpr int KS = G / 16;   // k-steps per group
   static constexpr int MT = D / 16;   // m-tiles (16 channels) of the PV product
-  uint32_t qf[NG][KS][2];             // Q^T B-fragments (head = gid)
   float qsum[NG][2];                  // per-group sum of q for heads 2t, 2t+1
   float m[2], lp[2];                  // running max (log2 units), partial row sums
   float z[NG][2];                     // zero-term accumulators (heads 2t, 2t+1)
-  float acc[MT][4];                   // PV accumulators, units of 2^-sigma
-  float accc[NG][2];                  // sum of W * (1024 + 2^(b-1)) per group (heads 2t, 2t+1)
+  float acc[MT][4];                   // PV accumulators (centred codes), units of 2^-sigma
   int sigma;                          // W = p * s_V * 2^sigma is the fp16 PV operand
 };
 
 template <int D, int G>
-__device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i, int h,
-                                 const TopkCtx& tk) {
+__device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, const uint16_t* qsm,
+                                 uint2* qfrag, const TopkCtx& tk) {
   constexpr int NG = SegState<D, G>::NG, KS = SegState<D, G>::KS, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const bool has = g < p.Gq;
-  const uint16_t* qrow = p.q + ((int64_t)i * p.Hq + h * p.Gq + (has ? g : 0)) * D;
+  const uint16_t* qrow = qsm + (has ? g : 0) * D;   // the segment's Gq query rows, in smem
   float qs[NG];
 #pragma unroll
   for (int gr = 0; gr < NG; ++gr) {
@@ -379,8 +383,7 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i
     for (int s = 0; s < KS; ++s) {
       const uint16_t* qp = qrow + gr * G + t * (G / 4) + 4 * s;
       uint2 v = has ? *reinterpret_cast<const uint2*>(qp) : make_uint2(0, 0);
-      S.qf[gr][s][0] = v.x;
-      S.qf[gr][s][1] = v.y;
+      qfrag[(gr * KS + s) * 32 + lane] = v;   // Q^T B-fragment of k-step (gr, s), head = gid
       __half2 a = *reinterpret_cast<__half2*>(&v.x), b = *reinterpret_cast<__half2*>(&v.y);
       float2 fa = __half22float2(a), fb = __half22float2(b);
       qs[gr] += (fa.x + fa.y) + (fb.x + fb.y);
@@ -390,7 +393,6 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, int i
     S.qsum[gr][0] = __shfl_sync(0xFFFFFFFFu, qs[gr], 8 * t);
     S.qsum[gr][1] = __shfl_sync(0xFFFFFFFFu, qs[gr], 8 * t + 4);
     S.z[gr][0] = S.z[gr][1] = 0.f;
-    S.accc[gr][0] = S.accc[gr][1] = 0.f;
   }
   S.sigma = kSigmaInit;               // the first page sets sigma
   S.m[0] = S.m[1] = -INFINITY;
@@ -441,7 +443,7 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       const int c = x & 1, ch = mt * 16 + g + 8 * (x >> 1), hd = 2 * t + c;
-      if (hd < Gq) po[hd * D + ch] = (S.acc[mt][x] - S.accc[gr][c]) * inv + S.z[gr][c];
+      if (hd < Gq) po[hd * D + ch] = fmaf(S.acc[mt][x], inv, S.z[gr][c]);
     }
   }
   if (tk.topk > 0) {
@@ -479,6 +481,7 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
 template <int D, int G, int B>
 __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
                                  float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
+  const uint2* qfrag = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(pbuf) + kQfragOff);
   constexpr int NG = D / G, KS = G / 16, MT = D / 16;
   constexpr int LANE_BYTES = D * B / 16;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -531,7 +534,8 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
             }
           }
         }
-        mma_16816(c, a, S.qf[gr][s][0], S.qf[gr][s][1]);
+        const uint2 qb = qfrag[(gr * KS + s) * 32 + lane];
+        mma_16816(c, a, qb.x, qb.y);
       }
       if constexpr (B == 16) {
         lg[0] += c[0]; lg[1] += c[1]; lg[2] += c[2]; lg[3] += c[3];
@@ -684,56 +688,60 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
       S.acc[mt][2] *= r0;
       S.acc[mt][3] *= r1;
     }
-#pragma unroll
-    for (int gr = 0; gr < NG; ++gr) {
-      S.accc[gr][0] *= r0;
-      S.accc[gr][1] *= r1;
-    }
   }
 
-  // ---------------- O^T += V^T(1024 + codes) x W ----------------
+  // ---------------- O^T += V^T(codes - 2^(b-1)) x W ----------------
   {
     constexpr int Q = (B == 16) ? D / 8 : D * B / 128;   // words per token pair
     constexpr int PER = (B == 16) ? 1 : 16 / B;          // codes per half-word
-    const uint8_t* vl = blk + 2 * D * B + lane * LANE_BYTES;
-    uint32_t vr[2 * Q];
-    if constexpr ((2 * Q) % 4 == 0) {
+    const uint32_t* vl = reinterpret_cast<const uint32_t*>(blk + 2 * D * B + lane * LANE_BYTES);
+    // m-tiles in two halves (words q of P = 0 and P = 1 for half of the chunk
+    // range); a single word per token pair (d = 64 at 2 bits) is one half
+    constexpr int NHF = Q >= 2 ? 2 : 1;                    // halves
+    constexpr int MH = MT / NHF;                           // m-tiles per half
+    constexpr int QH = Q / NHF;                            // words per token pair per half
 #pragma unroll
-      for (int x = 0; x < (2 * Q) / 4; ++x) {
-        const uint4 v = reinterpret_cast<const uint4*>(vl)[x];
-        vr[4 * x] = v.x; vr[4 * x + 1] = v.y; vr[4 * x + 2] = v.z; vr[4 * x + 3] = v.w;
-      }
-    } else {
-      const uint2 v = *reinterpret_cast<const uint2*>(vl);
-      vr[0] = v.x; vr[1] = v.y;
-    }
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int gr = (mt * 16) / G;
-      uint32_t a[4];
+    for (int hf = 0; hf < NHF; ++hf) {
+      uint32_t vr[2][QH];
 #pragma unroll
       for (int P = 0; P < 2; ++P) {
+        if constexpr (QH % 4 == 0) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int e = 2 * mt + r;
-          if constexpr (B == 16) {
-            a[P * 2 + r] = vr[P * Q + e] & (P ? dm1 : dm0);  // raw values of dead slots: zero
-          } else {
-            a[P * 2 + r] = unpack_pair<B>(vr[P * Q + e / PER], e % PER);
+          for (int x = 0; x < QH / 4; ++x) {
+            const uint4 v = reinterpret_cast<const uint4*>(vl + P * Q + hf * QH)[x];
+            vr[P][4 * x] = v.x; vr[P][4 * x + 1] = v.y; vr[P][4 * x + 2] = v.z; vr[P][4 * x + 3] = v.w;
           }
+        } else if constexpr (QH % 2 == 0) {
+#pragma unroll
+          for (int x = 0; x < QH / 2; ++x) {
+            const uint2 v = reinterpret_cast<const uint2*>(vl + P * Q + hf * QH)[x];
+            vr[P][2 * x] = v.x; vr[P][2 * x + 1] = v.y;
+          }
+        } else {
+          vr[P][0] = vl[P * Q + hf * QH];
         }
       }
-      mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
-    }
-    if constexpr (B != 16) {
-      // the code offset 1024 + 2^(b-1): one constant-row product per group
-      const uint32_t ka[4] = {centre_bits<B>(), centre_bits<B>(), centre_bits<B>(), centre_bits<B>()};
 #pragma unroll
-      for (int gr = 0; gr < NG; ++gr) {
-        float cc[4] = {S.accc[gr][0], S.accc[gr][1], S.accc[gr][0], S.accc[gr][1]};
-        mma_16816(cc, ka, wf[gr][0], wf[gr][1]);
-        S.accc[gr][0] = cc[0];
-        S.accc[gr][1] = cc[1];
+      for (int mh = 0; mh < MH; ++mh) {
+        const int mt = hf * MH + mh;
+        const int gr = (mt * 16) / G;
+        uint32_t a[4];
+#pragma unroll
+        for (int P = 0; P < 2; ++P) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int e = 2 * mt + r;                       // element of L_g
+            const int wq = e / PER - hf * QH;               // word within this half
+            if constexpr (B == 16) {
+              a[P * 2 + r] = vr[P][wq] & (P ? dm1 : dm0);   // raw values of dead slots: zero
+            } else {
+              // centred code pair c - 2^(b-1), exact in fp16: the sum over a
+              // whole segment then carries no large offset to cancel
+              a[P * 2 + r] = hsub2_bits(unpack_pair<B>(vr[P][wq], e % PER), centre_bits<B>());
+            }
+          }
+        }
+        mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
       }
     }
   }
@@ -852,64 +860,72 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 
   UnitMeta cur = resolve_unit(p, P, U0 + lane, U1);
   UnitMeta nxt = resolve_unit(p, P, U0 + 32 + lane, U1);
+  const int nu = (int)(U1 - U0);   // units of one warp: < 2^31
 
-  // prologue: fill the ring
-  const int64_t nunits = U1 - U0;
-  for (int s = 0; s < p.nstage && s < nunits; ++s) {
-    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, cur.src_lo, s);
-    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, cur.src_hi, s);
-    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, s);
+  // Issues unit ku (its lane in `m`) into stage st: the page-head block, plus
+  // the segment's Q rows when ku is the first unit of a segment in this warp.
+  int last_issued_seg = -1;
+  auto issue = [&](const UnitMeta& m, int ku, int st) {
+    const int srcl = ku & 31;
+    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, m.src_lo, srcl);
+    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, m.src_hi, srcl);
+    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, m.cls_seg, srcl);
+    const int useg = (int)(cs & 0xFFFFFFu);
+    const bool needq = useg != last_issued_seg;
+    last_issued_seg = useg;
     if (lane == 0) {
+      uint8_t* dst = wsm + st * p.stage_bytes;
       const uint32_t bytes = (uint32_t)p.phb[cs >> 24];
-      mbar_arrive_expect_tx(&bars[s], bytes);
-      bulk_g2s(wsm + s * p.stage_bytes,
-               reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[s]);
+      mbar_arrive_expect_tx(&bars[st], bytes + (needq ? (uint32_t)p.q_bytes : 0u));
+      bulk_g2s(dst, reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[st]);
+      if (needq) {
+        const int i = useg / p.Hkv, h = useg - (useg / p.Hkv) * p.Hkv;
+        bulk_g2s(dst + p.q_off, p.q + ((int64_t)i * p.Hq + (int64_t)h * p.Gq) * D,
+                 (uint32_t)p.q_bytes, &bars[st]);
+      }
     }
-  }
+  };
+
+  // only the first page goes out before the loop: copies issued together all
+  // land together, so the rest of the ring is filled once the first has landed
+  issue(cur, 0, 0);
 
   SegState<D, G> S;
   int seg = -1;
   int stage = 0;
   uint32_t parity = 0;
-  const int nu = (int)nunits;   // units of one warp: < 2^31
   for (int k = 0; k < nu; ++k) {
     const int kk = k & 31;
     if (kk == 0 && k > 0) {
       cur = nxt;
       nxt = resolve_unit(p, P, U0 + k + 32 + lane, U1);
     }
-    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, kk);
-    const int useg = (int)(cs & 0xFFFFFFu);
-    if (useg != seg) {
-      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, seg / p.Hkv, seg % p.Hkv, T, W, pbuf);
-      seg = useg;
-      seg_begin<D, G>(S, p, seg / p.Hkv, seg % p.Hkv, tk);
-    }
     if (!mbar_wait_bounded(&bars[stage], parity)) {
       if (lane == 0) set_status(p.status, THINKV_ERR_TIMEOUT);
       // drain the copies still in flight (bounded), then leave
-      for (int k2 = k + 1; k2 < nu && k2 < k + p.nstage; ++k2)
+      const int issued = k == 0 ? 1 : min(nu, k + p.nstage);
+      for (int k2 = k + 1; k2 < issued; ++k2)
         mbar_wait_bounded(&bars[k2 % p.nstage], (uint32_t)((k2 / p.nstage) & 1));
       return;
     }
+    if (k == 0)
+      for (int s2 = 1; s2 < p.nstage && s2 < nu; ++s2) issue(cur, s2, s2);
+    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, kk);
+    const int useg = (int)(cs & 0xFFFFFFu);
+    uint8_t* blk = wsm + stage * p.stage_bytes;
+    if (useg != seg) {
+      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, seg / p.Hkv, seg % p.Hkv, T, W, pbuf);
+      seg = useg;
+      seg_begin<D, G>(S, p, reinterpret_cast<const uint16_t*>(blk + p.q_off),
+                      reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(pbuf) + kQfragOff), tk);
+      __syncwarp();
+    }
     const uint32_t mask = __shfl_sync(0xFFFFFFFFu, cur.mask, kk);
-    page_dispatch<D, G>(S, wsm + stage * p.stage_bytes, p.bits[cs >> 24], mask & 0xFFFFu,
-                        p.scale_log2, pbuf, tk, p.Gq);
+    page_dispatch<D, G>(S, blk, p.bits[cs >> 24], mask & 0xFFFFu, p.scale_log2, pbuf, tk, p.Gq);
     __syncwarp();
     // refill this stage with unit k + nstage (from this batch of 32 or the next)
     const int kn = k + p.nstage;
-    const bool same = (kn >> 5) == (k >> 5);
-    const int srcl = kn & 31;
-    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, same ? cur.src_lo : nxt.src_lo, srcl);
-    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, same ? cur.src_hi : nxt.src_hi, srcl);
-    const uint32_t ncs = __shfl_sync(0xFFFFFFFFu, same ? cur.cls_seg : nxt.cls_seg, srcl);
-    if (lane == 0 && kn < nu) {
-      fence_proxy_async_smem();
-      const uint32_t bytes = (uint32_t)p.phb[ncs >> 24];
-      mbar_arrive_expect_tx(&bars[stage], bytes);
-      bulk_g2s(wsm + stage * p.stage_bytes,
-               reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[stage]);
-    }
+    if (kn < nu) issue(((kn >> 5) == (k >> 5)) ? cur : nxt, kn, stage);
     if (++stage == p.nstage) {
       stage = 0;
       parity ^= 1u;
@@ -948,7 +964,9 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
     int64_t b = page_head_bytes(D, G, L.bits[c]);
     if (b > maxphb) maxphb = b;
   }
-  const int stage_bytes = (int)((maxphb + 127) / 128 * 128);
+  const int Gq0 = L.num_q_heads / L.num_kv_heads;
+  const int q_bytes = Gq0 * D * 2;
+  const int stage_bytes = (int)((maxphb + 127) / 128 * 128) + (q_bytes + 127) / 128 * 128;
   // ~15 KB of page-head stages per warp keeps three 4-warp CTAs per SM
   int nstage = (int)(15360 / stage_bytes);
   if (nstage < 2) nstage = 2;
@@ -1037,6 +1055,12 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   p.nstage = dl.nstage;
   p.stage_bytes = dl.stage_bytes;
   p.warp_smem = dl.warp_smem;
+  {
+    int64_t maxphb = 0;
+    for (int c = 0; c < 3; ++c) maxphb = maxphb > p.phb[c] ? maxphb : p.phb[c];
+    p.q_off = (int32_t)((maxphb + 127) / 128 * 128);
+    p.q_bytes = p.Gq * D * 2;
+  }
   p.plan_smem = plan_smem_bytes(n);
   cudaError_t e;
   if (D == 128 && G == 64) e = launch_split<128, 64>(p, dl, stream);

@@ -212,28 +212,38 @@ def _normal_fp16_from_ids(ids: torch.Tensor, seed: int, stream: int) -> torch.Te
     return (centred * (1.0 / 65536.0)).to(torch.float16)
 
 
-def kv_values(w: Workload, seq: int, pos0: int, n: int,
-              device="cpu", chunk_elems: int = 1 << 25) -> Tuple[torch.Tensor, torch.Tensor]:
-    """K and V (fp16, shape [n, Hkv, d]) of positions pos0..pos0+n-1 of ``seq``."""
+def kv_for_tokens(w: Workload, seqs, pos, device="cpu",
+                  chunk_tokens: int = 1 << 14) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K and V (fp16, shape [n, Hkv, d]) of the tokens (seqs[i], pos[i]).
+
+    Every value is a function of (seed, sequence, position, head, channel, K|V)
+    only, so any subset of tokens can be regenerated on any device."""
     H, d = w.num_kv_heads, w.head_dim
     per_tok = H * d * 2
-    out = torch.empty(n * per_tok, dtype=torch.float16, device=device)
-    base_id = ((seq << 26) + pos0) * per_tok
-    total = n * per_tok
-    for s in range(0, total, chunk_elems):
-        e = min(total, s + chunk_elems)
-        ids = torch.arange(base_id + s, base_id + e, dtype=torch.int64, device=device)
-        out[s:e] = _normal_fp16_from_ids(ids, w.seed, _STREAM_KV)
+    seqs_t = torch.as_tensor(np.asarray(seqs, dtype=np.int64), device=device)
+    pos_t = torch.as_tensor(np.asarray(pos, dtype=np.int64), device=device)
+    n = int(seqs_t.numel())
+    out = torch.empty(n, per_tok, dtype=torch.float16, device=device)
+    lane = torch.arange(per_tok, dtype=torch.int64, device=device)
+    for a in range(0, n, chunk_tokens):
+        b = min(n, a + chunk_tokens)
+        base = ((seqs_t[a:b] << 26) + pos_t[a:b]) * per_tok
+        ids = base[:, None] + lane[None, :]
+        out[a:b] = _normal_fp16_from_ids(ids, w.seed, _STREAM_KV)
     kv = out.view(n, H, d, 2)
     pairs = outlier_pairs(w)
-    if len(pairs):
+    if len(pairs) and n:
         hh = torch.as_tensor(pairs[:, 0], device=device)
         cc = torch.as_tensor(pairs[:, 1], device=device)
         kv32 = kv[:, hh, cc, :].to(torch.float32) * 8.0
         kv[:, hh, cc, :] = kv32.to(torch.float16)
-    k = kv[..., 0].contiguous()
-    v = kv[..., 1].contiguous()
-    return k, v
+    return kv[..., 0].contiguous(), kv[..., 1].contiguous()
+
+
+def kv_values(w: Workload, seq: int, pos0: int, n: int,
+              device="cpu") -> Tuple[torch.Tensor, torch.Tensor]:
+    """K and V (fp16, shape [n, Hkv, d]) of positions pos0..pos0+n-1 of ``seq``."""
+    return kv_for_tokens(w, np.full(n, seq, dtype=np.int64), np.arange(pos0, pos0 + n), device)
 
 
 def q_values(w: Workload, step: int, device="cpu") -> torch.Tensor:
@@ -277,15 +287,7 @@ def make_append_call(runs: Sequence[Tuple[int, int, int]], tags_of) -> AppendCal
 
 def call_kv(w: Workload, call: AppendCall, device="cpu") -> Tuple[torch.Tensor, torch.Tensor]:
     """K and V ([n, Hkv, d] fp16) of every token of ``call``, in call order."""
-    ks, vs = [], []
-    for (s, p0, c) in call.runs:
-        k, v = kv_values(w, s, p0, c, device=device)
-        ks.append(k)
-        vs.append(v)
-    if not ks:
-        e = torch.zeros(0, w.num_kv_heads, w.head_dim, dtype=torch.float16, device=device)
-        return e, e.clone()
-    return torch.cat(ks), torch.cat(vs)
+    return kv_for_tokens(w, call.seqs, call.pos, device=device)
 
 
 class Schedule:

@@ -144,3 +144,160 @@ def attn_error(gpu_out: np.ndarray, ref: np.ndarray) -> float:
     den = np.abs(r).max(axis=1)
     err = np.where(den > 0, num / np.where(den > 0, den, 1), num)
     return float(err.max()) if err.size else 0.0
+
+
+# --------------------------------------------------------------------------- #
+# full-size checks on sampled sequences
+# --------------------------------------------------------------------------- #
+class OracleSubset:
+    """The oracle replaying only some sequences of a workload.
+
+    Sequences never interact except through the numbering of pages, so each
+    sampled sequence's live set, codes and attention output equal those of a
+    run over the whole batch.  Oracle sequence j stands for workload sequence
+    seqs[j]; inputs come from the shared generator keyed by the original id."""
+
+    def __init__(self, w: W.Workload, seqs, extra: int = 0, gen_device: str = "cuda"):
+        import math
+        self.w = w
+        self.seqs = [int(s) for s in seqs]
+        self.sched = W.Schedule(w, extra)
+        self.gen_device = gen_device
+        pool, mb = [0, 0, 0], 1
+        for s in self.seqs:
+            cnt = np.bincount(self.sched.tags(s), minlength=3)
+            pages = [int(math.ceil(int(cnt[c]) / 16)) for c in range(3)]
+            for c in range(3):
+                pool[c] += pages[c]
+            mb = max(mb, sum(pages))
+        self.o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
+                          len(self.seqs), mb, [max(1, p) for p in pool])
+        self.generated = self.sched.lengths[self.seqs].astype(np.int64).copy()
+
+    def _append(self, runs):
+        """runs: [(j, pos0, count)] in call order (j = oracle sequence index)."""
+        if not runs:
+            return
+        S, P, T, orig = [], [], [], []
+        for (j, p0, c) in runs:
+            s = self.seqs[j]
+            S.append(np.full(c, j, dtype=np.int32))
+            P.append(np.arange(p0, p0 + c, dtype=np.int32))
+            T.append(self.sched.tags(s)[p0:p0 + c])
+            orig.append(np.full(c, s, dtype=np.int64))
+        S, P, T, orig = map(np.concatenate, (S, P, T, orig))
+        k, v = W.kv_for_tokens(self.w, orig, P.astype(np.int64), device=self.gen_device)
+        assert self.o.append(S, P, T.astype(np.uint8), k.cpu(), v.cpu()) == O.OK
+
+    def _evict(self):
+        b = self.sched.budgets(self.generated)
+        assert self.o.evict(np.arange(len(self.seqs), dtype=np.int32), b) == O.OK
+
+    def setup(self, churn: bool = True):
+        where = {s: j for j, s in enumerate(self.seqs)}
+        for call in self.sched.prefill_calls():
+            self._append([(where[s], p0, c) for (s, p0, c) in call.runs if s in where])
+        self._evict()
+        if self.w.post_evict_append:
+            n = self.w.post_evict_append
+            self._append([(j, int(self.generated[j]), n) for j in range(len(self.seqs))])
+            self.generated += n
+        if churn:
+            for _ in range(self.w.churn_steps):
+                self.churn_step()
+
+    def churn_step(self):
+        self._append([(j, int(self.generated[j]), 1) for j in range(len(self.seqs))])
+        self.generated += 1
+        self._evict()
+
+    def decode(self, step, topk=None):
+        q = W.q_values(self.w, step, device="cpu")[self.seqs]
+        return self.o.decode(np.arange(len(self.seqs), dtype=np.int32), q, topk=topk, threads=8)
+
+    def live_by_pos(self, j):
+        st = self.o.state()
+        out = {}
+        nb = int(st["num_blocks"][j])
+        for e in st["table"][j, :nb]:
+            page, cls, mask = int(O.entry_page(e)), int(O.entry_class(e)), int(O.entry_mask(e))
+            for sl in range(PAGE):
+                if (mask >> sl) & 1:
+                    out[int(st["slot_pos"][cls][page, sl])] = (cls, page, sl)
+        return out
+
+
+def gpu_live_by_pos(snap, s):
+    """pos -> (class, page, slot) of every live token of GPU sequence s."""
+    out = {}
+    nb = int(snap["num_blocks"][s])
+    for e in snap["table"][s, :nb]:
+        page, cls, mask = int(O.entry_page(e)), int(O.entry_class(e)), int(O.entry_mask(e))
+        for sl in range(PAGE):
+            if (mask >> sl) & 1:
+                out[int(snap["slot_pos"][cls][page, sl])] = (cls, page, sl)
+    return out
+
+
+def _gpu_blocks(cache, c, pages):
+    """Page-head blocks [len(pages), Hkv, phb] of class c, copied from the GPU."""
+    import torch
+    phb = cache.page_head_bytes(c)
+    pool = cache.buf["pool_" + "RET"[c]].view(cache.pool_pages[c], cache.H, phb)
+    idx = torch.as_tensor(np.asarray(pages, dtype=np.int64), device=pool.device)
+    return pool[idx].cpu().numpy()
+
+
+def compare_codes_by_pos(cache, gl: dict, oracle: O.Oracle, ol: dict):
+    """Codes and params of every live token, matched by position, bit for bit."""
+    d, G = cache.d, cache.G
+    for c in range(3):
+        poss = [p for p in gl if gl[p][0] == c]
+        if not poss:
+            continue
+        b = cache.bits[c]
+        gpages = [gl[p][1] for p in poss]
+        gslots = np.array([gl[p][2] for p in poss])
+        kc, vc, kp, vp = decode_blocks(_gpu_blocks(cache, c, gpages), d, G, b)
+        n = np.arange(len(poss))
+        opages = np.array([ol[p][1] for p in poss])
+        oslots = np.array([ol[p][2] for p in poss])
+        ocodes = oracle.codes(c)
+        assert np.array_equal(kc[n, :, gslots], ocodes[opages, :, 0, oslots]), f"K codes class {c}"
+        assert np.array_equal(vc[n, :, gslots], ocodes[opages, :, 1, oslots]), f"V codes class {c}"
+        if b < 16:
+            op = oracle.params(c)
+            assert np.array_equal(kp[n, :, gslots], op[opages, :, 0, oslots]), f"K params class {c}"
+            assert np.array_equal(vp[n, :, gslots], op[opages, :, 1, oslots]), f"V params class {c}"
+
+
+def check_slot_invariants(snap, ns):
+    """Free-slot invariants of every sequence (no oracle needed): per (sequence,
+    class) the allocated slots are exactly the live ones plus the free-stack
+    ones, each once; live_count and num_live agree with the masks; the live
+    list and its index invert each other; the FIFO window holds the live slots."""
+    cap = snap["fifo"].shape[2]
+    for s in range(ns):
+        nb = int(snap["num_blocks"][s])
+        ents = snap["table"][s, :nb]
+        cls = O.entry_class(ents)
+        masks = O.entry_mask(ents)
+        bits = ((masks[:, None] >> np.arange(PAGE)[None, :]) & 1).astype(bool)
+        assert int(bits.sum()) == int(snap["live_count"][s])
+        nl = int(snap["num_live"][s])
+        assert nl == int((masks != 0).sum())
+        lst = O.live_entry(snap["live_list"][s, :nl])
+        assert np.array_equal(snap["live_index"][s, lst], np.arange(nl))
+        for c in range(3):
+            mark = np.zeros(nb * PAGE, dtype=np.int32)
+            own = np.repeat(cls == c, PAGE)
+            live_ids = np.flatnonzero(bits.reshape(-1) & own)
+            mark[live_ids] += 1
+            top = int(snap["free_top"][s, c])
+            free = snap["free_slots"][s, c, :top]
+            assert free.size == 0 or (free.min() >= 0 and free.max() < nb * PAGE)
+            np.add.at(mark, free, 1)
+            assert np.array_equal(mark, own.astype(np.int32)), f"free/live slots, seq {s} class {c}"
+            h, t = int(snap["fifo_head"][s, c]), int(snap["fifo_tail"][s, c])
+            win = snap["fifo"][s, c, np.arange(h, t) % cap]
+            assert np.array_equal(np.sort(win), live_ids)

@@ -34,9 +34,11 @@ def _check_all(g, o, step=0, topk=None, codes=True, max_pages=None):
     out, mass = g.decode(step, topk=topk)
     ref, rmass = o.decode(step, topk=topk)
     err = Hn.attn_error(out.cpu().numpy(), ref)
+    print(f"{g.w.name} step {step}: attention error {err:.3e}")
     assert err <= Hn.TOL, err
     if topk:
         merr = float(np.abs(mass.cpu().numpy().astype(np.float64) - rmass).max())
+        print(f"{g.w.name} step {step}: top-k mass error {merr:.3e}")
         assert merr <= Hn.MASS_TOL, merr
     return err
 
