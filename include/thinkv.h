@@ -202,7 +202,12 @@ THINKV_API size_t thinkv_append_workspace_bytes(const thinkv_layout* L, int32_t 
  * INVALID; pool exhausted -> OUT_OF_PAGES; table full -> OUT_OF_BLOCKS,
  * checked in that order) set *status and change nothing.
  * workspace: device, >= thinkv_append_workspace_bytes(L, n_tokens) bytes,
- * caller-owned scratch; contents need not be initialised. */
+ * caller-owned scratch.  Its first 4 bytes are an arrival counter of the
+ * one-launch path taken by calls of up to 512 tokens: zero-fill the workspace
+ * once before its first use; every call leaves the counter zero (a call that
+ * stops on a device-detected error stops before anything arrives).  The
+ * rest needs no initialisation.  Calls that share a workspace must not
+ * overlap on the GPU. */
 THINKV_API int thinkv_append_quantize(const thinkv_cache* cache, int32_t n_tokens,
                            const int32_t* seq, const int32_t* pos, const uint8_t* tag,
                            const uint16_t* k, const uint16_t* v,
@@ -235,11 +240,10 @@ THINKV_API size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t 
  * probability held by the topk (1..64) most probable live tokens (1 when the
  * sequence has <= topk live tokens, 0 when it has none).
  * workspace: device, >= thinkv_decode_workspace_bytes(L, n_seqs, topk) bytes,
- * caller-owned scratch.  Its first n_seqs*num_kv_heads 32-bit words are the
- * per-(sequence, kv-head) arrival counters of the split-K merge: zero-fill the
- * workspace once before its first use; every call that completes leaves them
- * zero again (after a call that stopped on a device error, zero them again).
- * Calls that share a workspace must not overlap on the GPU.
+ * caller-owned scratch for the split-K partial results; its contents need no
+ * initialisation.  Calls that share a workspace must not overlap on the GPU.
+ * Two kernels run per call: the split kernel over the live page-heads and the
+ * combine of the segments it left in several pieces.
  * 1 <= n_seqs <= 16384. */
 THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs, const int32_t* seq,
                             const uint16_t* q, uint16_t* out, float* topk_mass,
@@ -263,10 +267,9 @@ THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs
  * that size returns THINKV_ERR_WORKSPACE before launching anything.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  Each call clears the array's arrival counters on `stream`, and
- * calls share the array: two calls that overlap on the GPU (different streams,
- * or different host threads) race and must not be issued.  Nothing is
- * allocated or freed. */
+ * capture.  Calls share the array: two calls that overlap on the GPU
+ * (different streams, or different host threads) race and must not be
+ * issued.  Nothing is allocated or freed. */
 THINKV_API int thinkv_decode_attention_noalloc(const thinkv_cache* cache, int32_t n_seqs,
                                                const int32_t* seq, const uint16_t* q,
                                                uint16_t* out, float* topk_mass, int32_t topk,

@@ -168,8 +168,8 @@ class ThinKVCache:
         return int(lib().thinkv_page_head_bytes(C.byref(self.layout), c))
 
     def _workspace(self, key: str, nbytes: int) -> torch.Tensor:
-        # zero-filled once: the decode workspace starts with arrival counters
-        # that every completed call leaves at zero
+        # zero-filled once: the append and decode workspaces start with arrival
+        # counters that every completed call leaves at zero
         t = self._ws.get(key)
         if t is None or t.numel() < nbytes:
             t = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "thinkv.h"
 
 namespace thinkv {
@@ -45,6 +47,39 @@ __device__ inline void set_status(int32_t* status, int32_t code) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start while the previous kernel of the
+// stream still runs, once every CTA of that kernel has called
+// pdl_launch_dependents() (or exited).  Before pdl_wait() returns -- when the
+// previous kernel has completed and its writes are visible -- it may only
+// read its own inputs, never cache state.  Without the attribute both are
+// no-ops.
+// ---------------------------------------------------------------------------
+__device__ inline void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ inline void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+#ifdef __CUDACC__
+// Launches kernel k with the programmatic stream-serialisation attribute.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*k)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+#endif
+
+// ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
 __device__ inline uint32_t smem_u32(const void* p) {
@@ -62,6 +97,12 @@ __device__ inline void fence_mbar_init() {
 
 __device__ inline void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Orders this thread's view of global memory (generic proxy) before its
+// later bulk copies (async proxy) that read it.
+__device__ inline void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {

@@ -13,16 +13,19 @@
 //   matter how lengths and budgets vary.  Per warp, lane 0 streams page-head
 //   blocks (K codes, V codes, params: one contiguous block per page and head)
 //   into a shared-memory ring with cp.async.bulk (TMA) + mbarriers; the warp
-//   unpacks codes straight into mma.sync m16n8k16 operands (fp16 magic-number
-//   conversion, codes centred by 2^(b-1) so products stay exact), computes
-//   q.k for the whole GQA group at once (tokens x heads), applies the per-group
-//   scale/zero in fp32, runs the online softmax, transposes p through a small
-//   shared buffer and accumulates p*scale (fp16, exponent-shifted) times the V
-//   codes on the tensor cores, with the zero terms summed in fp32.  Each warp
-//   writes one partial (m, l, o, top-k logits) per (sequence, kv-head) segment
-//   it touched and counts itself in on the segment's arrival counter; the
-//   last warp to arrive merges the segment's partials with the log-sum-exp
-//   rule and writes fp16 O and the top-k mass -- one launch per decode.
+//   unpacks codes straight into mma.sync m16n8k16 operands (byte-permute
+//   conversion to fp16 1024 + code), computes q.k for the whole GQA group at
+//   once (tokens x heads), applies the per-group scale/zero in fp32, runs the
+//   online softmax, transposes p through a small shared buffer and accumulates
+//   p*scale (fp16, exponent-shifted) times the centred V codes on the tensor
+//   cores, with the zero terms summed in fp32.  A segment (sequence, kv-head)
+//   that lies wholly in one warp is written out at once; otherwise each warp
+//   writes one piece record (m, l, o, top-k logits) per segment it touched.
+//
+//   combine kernel (launched right behind, programmatic dependent launch): one
+//   CTA per segment left in several pieces merges the records with the
+//   log-sum-exp rule -- a thread per quad of each head's output row, a warp per
+//   head for the top-k lists -- and writes fp16 O and the top-k mass.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -47,6 +50,7 @@ constexpr int kQfragOff = kPtBytes;
 constexpr int kQfragBytes = 2048;                       // (D / 16) k-steps x 32 lanes x 8 B
 constexpr int kPbufBytes = kPtBytes + kQfragBytes;      // >= 2 * 32 * 8 * 4 + 16 * 4
 constexpr int kSigmaInit = 1 << 20;
+constexpr int kMaxStages = 8;                   // page ring stages (one mbarrier each)
 constexpr int kCandCap = 128;                   // top-k candidate slots per head
 constexpr int kTopkHdrBytes = 64;               // per-head counts and thresholds
 
@@ -63,10 +67,9 @@ struct DecodeParams {
   int32_t n;
   const uint16_t* q;
   float scale_log2;
-  float* part_o;   // [pieces][Gq][D]
-  float* part_ml;  // [pieces][Gq][2]   (m in log2 units, l)
-  float* part_topk;  // [pieces][Gq][topk] largest logits (log2 units), -inf padded
-  uint32_t* ctr;     // [n * Hkv] arrival counters of the segments (zero between calls)
+  void* rec;         // piece records of split segments (index warp + segment)
+  int32_t* pref;      // [n + 1] prefix of live pages over the call's sequences
+  int64_t split_warps;  // warps of the split kernel's grid
   const int32_t* live_count;
   uint16_t* out;     // [n][Hq][D]
   float* mass;       // [n][Hq] or null
@@ -112,6 +115,31 @@ __device__ inline void bitonic128_desc(float (&v)[4]) {
   }
 }
 
+// Sorts 64 values held 2 per lane (element lane*2 + j) into descending order.
+__device__ inline void bitonic64_desc(float (&v)[2]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 2) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int i = lane * 2 + j;
+          const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], stride >> 1);
+          const bool desc = (i & size) == 0, lower = (i & stride) == 0;
+          v[j] = (lower == desc) ? fmaxf(v[j], o) : fminf(v[j], o);
+        }
+      } else {
+        const bool desc = ((lane * 2) & size) == 0;
+        const float a = v[0], b = v[1];
+        v[0] = desc ? fmaxf(a, b) : fminf(a, b);
+        v[1] = desc ? fminf(a, b) : fmaxf(a, b);
+      }
+    }
+  }
+}
+
 struct TopkCtx {
   float* cand;    // [Gq][kCandCap]
   int* cnt;       // [Gq]
@@ -124,6 +152,27 @@ __device__ inline void cand_compact(const TopkCtx& tk, int h) {
   const int lane = threadIdx.x & 31;
   float* c = tk.cand + h * kCandCap;
   const int n = tk.cnt[h];
+  if (n <= 64) {
+    // the smaller network suffices
+    float u[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) u[j] = (lane * 2 + j < n) ? c[lane * 2 + j] : -INFINITY;
+    bitonic64_desc(u);
+    __syncwarp();
+    const int keep = min(n, tk.topk);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (lane * 2 + j < keep) c[lane * 2 + j] = u[j];
+    const int kl = tk.topk - 1;
+    const float kth = __shfl_sync(0xFFFFFFFFu, (kl & 1) ? u[1] : u[0], (kl >> 1) & 31);
+    __syncwarp();
+    if (lane == 0) {
+      tk.cnt[h] = keep;
+      if (n >= tk.topk) tk.theta[h] = kth;
+    }
+    __syncwarp();
+    return;
+  }
   float v[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) v[j] = (lane * 4 + j < n) ? c[lane * 4 + j] : -INFINITY;
@@ -144,201 +193,43 @@ __device__ inline void cand_compact(const TopkCtx& tk, int h) {
   __syncwarp();
 }
 
-// Merges the partials (m, l, o, top-k logits) of segment (i, h) into fp16 O
-// and the top-k mass of its Gq query heads.  Run by the last warp to finish a
-// piece of the segment.  Pieces are the non-empty warps from w0 on: with
-// T <= W every unit has its own warp, otherwise all of w0..w1 hold units.
-// Loads are issued lane-parallel or in independent batches (a loop of
-// dependent loads would put one L2 round trip per piece on the kernel tail);
-// partials are read through L2 (ld.global.cg).
-__device__ inline int64_t piece_warp(int j, int64_t Us, int64_t w0, int64_t T, int64_t W) {
-  return T <= W ? ((Us + j + 1) * W - 1) / T : w0 + j;
+// ---------------------------------------------------------------------------
+// partial results of split segments
+// ---------------------------------------------------------------------------
+// A piece of a (sequence, kv-head) segment is one contiguous record, so that a
+// merge can fetch it with a single bulk copy:
+//   [0, 64)                 (m, l) of query heads 0..7 (m in log2 units, l the
+//                           row sum relative to m)
+//   [64, 64 + 4*Gq*D)       the unnormalised output rows o[Gq][D]
+//   then 4*Gq*kpad bytes    per head, the top-k largest logits, descending,
+//                           -inf padded (kpad = topk rounded up to 4)
+__host__ __device__ inline int64_t record_bytes(int Gq, int D, int topk) {
+  const int kpad = (topk + 3) / 4 * 4;
+  return 64 + 4LL * Gq * D + 4LL * Gq * kpad;
 }
 
-template <int D>
-__device__ void merge_segment(const DecodeParams& p, int i, int h, int64_t Us,
-                                           int64_t w0, int np, int64_t T, int64_t W,
-                                           const TopkCtx& tk, float* scratch) {
+// Merges a bitonic sequence of 128 values held 4 per lane (element lane*4+j)
+// into descending order.
+__device__ inline void bitonic128_merge_desc(float (&v)[4]) {
   const int lane = threadIdx.x & 31;
-  constexpr int QD = D / 4;                     // float4 quads per head row
-  constexpr int CH = 32;                        // pieces per chunk (scratch: 2 * CH * 8 floats)
-  const int Gq = p.Gq;
-  const int64_t seg = (int64_t)i * p.Hkv + h;
-  const int npair = Gq * QD;
-  float2* ml = reinterpret_cast<float2*>(scratch);            // [CH][Gq] (m, l)
-  float* Mh = scratch + 2 * CH * 8;                           // [Gq] running max
-  float* Lh = Mh + 8;                                         // [Gq] row sums
-
-  // ---- pass 1: M per head over all pieces ----
-  if (lane < Gq) Mh[lane] = -INFINITY;
-  __syncwarp();
-  for (int jb = 0; jb < np; jb += CH) {
-    const int cnt = min(CH, np - jb);
-    for (int x = lane; x < cnt * Gq; x += 32) {
-      const int j = x / Gq, r = x - j * Gq;
-      const int64_t pc = (piece_warp(jb + j, Us, w0, T, W) + seg) * Gq + r;
-      ml[x] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + pc * 2));
-    }
-    __syncwarp();
-    if (lane < Gq) {
-      float mx = Mh[lane];
-      for (int j = 0; j < cnt; ++j) mx = fmaxf(mx, ml[j * Gq + lane].x);
-      Mh[lane] = mx;
-    }
-    __syncwarp();
-  }
-  // ---- pass 2: weights and row sums ----
-  if (lane < Gq) Lh[lane] = 0.f;
-  __syncwarp();
-  // (head, quad) pairs of this lane: lane + 32 x; done in groups of PG pairs,
-  // each over all pieces with BATCH pieces of independent loads in flight
-  constexpr int PG = 4, BATCH = 4;
-  const int npl = (npair + 31) / 32;
-  for (int x0 = 0; x0 < npl; x0 += PG) {
-    float4 acc[PG];
 #pragma unroll
-    for (int x = 0; x < PG; ++x) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int jb = 0; jb < np; jb += CH) {
-      const int cnt = min(CH, np - jb);
-      if (np > CH || x0 > 0) {  // (m, l) of this chunk (a single chunk is still in scratch)
-        for (int x = lane; x < cnt * Gq; x += 32) {
-          const int j = x / Gq, r = x - j * Gq;
-          const int64_t pc = (piece_warp(jb + j, Us, w0, T, W) + seg) * Gq + r;
-          ml[x] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + pc * 2));
-        }
-        __syncwarp();
+  for (int stride = 64; stride > 0; stride >>= 1) {
+    if (stride >= 4) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], stride >> 2);
+        const bool lower = ((lane * 4 + j) & stride) == 0;
+        v[j] = lower ? fmaxf(v[j], o) : fminf(v[j], o);
       }
-      for (int x = lane; x < cnt * Gq; x += 32) ml[x].x = exp2_approx(ml[x].x - Mh[x % Gq]);
-      __syncwarp();
-      if (x0 == 0 && lane < Gq) {
-        float l = Lh[lane];
-        for (int j = 0; j < cnt; ++j) l = fmaf(ml[j * Gq + lane].y, ml[j * Gq + lane].x, l);
-        Lh[lane] = l;
-      }
-      for (int jj = 0; jj < cnt; jj += BATCH) {
-        float4 v[BATCH][PG];
+    } else {
 #pragma unroll
-        for (int b = 0; b < BATCH; ++b) {
-          if (jj + b < cnt) {
-            const int64_t base = (piece_warp(jb + jj + b, Us, w0, T, W) + seg) * Gq;
-#pragma unroll
-            for (int x = 0; x < PG; ++x) {
-              const int pr = lane + 32 * (x0 + x);
-              if (pr < npair) {
-                const int r = pr / QD, q = pr - r * QD;
-                v[b][x] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (base + r) * D) + q);
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < BATCH; ++b) {
-          if (jj + b < cnt) {
-#pragma unroll
-            for (int x = 0; x < PG; ++x) {
-              const int pr = lane + 32 * (x0 + x);
-              if (pr < npair) {
-                const float fw = ml[(jj + b) * Gq + pr / QD].x;
-                acc[x].x = fmaf(v[b][x].x, fw, acc[x].x);
-                acc[x].y = fmaf(v[b][x].y, fw, acc[x].y);
-                acc[x].z = fmaf(v[b][x].z, fw, acc[x].z);
-                acc[x].w = fmaf(v[b][x].w, fw, acc[x].w);
-              }
-            }
-          }
-        }
-      }
-      __syncwarp();
-    }
-    // ---- fp16 output rows for this group of pairs ----
-#pragma unroll
-    for (int x = 0; x < PG; ++x) {
-      const int pr = lane + 32 * (x0 + x);
-      if (pr < npair) {
-        const int r = pr / QD, q = pr - r * QD;
-        const float inv = 1.f / Lh[r];
-        const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].x * inv)) |
-                            ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].y * inv)) << 16);
-        const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].z * inv)) |
-                            ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].w * inv)) << 16);
-        const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
-        reinterpret_cast<uint2*>(p.out + row * D)[q] = make_uint2(lo, hi);
+      for (int j = 0; j < 4; ++j) {
+        if (j & stride) continue;
+        const float x = v[j], y = v[j | stride];
+        v[j] = fmaxf(x, y);
+        v[j | stride] = fminf(x, y);
       }
     }
-  }
-  if (!p.mass) return;
-  for (int r = 0; r < Gq; ++r) {
-    const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
-    const float M = Mh[r];
-    const float inv = 1.f / Lh[r];
-    const int k = p.topk;
-    if (p.live_count[p.seq[i]] <= k) {
-      if (lane == 0) p.mass[row] = 1.f;
-      continue;
-    }
-    // ---- top-k of the union of the pieces' top-k lists ----
-    // Each list holds its piece's k largest logits (-inf padded), so the
-    // union's k-th largest is >= theta = max over pieces of min(list): only
-    // values >= theta can be in the top-k, and at least k of them exist.
-    float v[4];
-    bool done = false;
-    const int staged = np * k;
-    if (staged <= (Gq - 1) * kCandCap) {
-      float* st = tk.cand;                                 // staging: np*k values
-      float* sb = tk.cand + (Gq - 1) * kCandCap;           // selection: 128 values
-      for (int x = lane; x < staged; x += 32) {
-        const int j = x / k, e = x - j * k;
-        st[x] = __ldcg(p.part_topk + ((piece_warp(j, Us, w0, T, W) + seg) * Gq + r) * k + e);
-      }
-      __syncwarp();
-      float th = -INFINITY;
-      for (int j = lane; j < np; j += 32) {
-        float mn = INFINITY;
-        for (int e = 0; e < k; ++e) mn = fminf(mn, st[j * k + e]);
-        th = fmaxf(th, mn);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) th = fmaxf(th, __shfl_xor_sync(0xFFFFFFFFu, th, o));
-      int count = 0;
-      for (int xb = 0; xb < staged; xb += 32) {
-        const int x = xb + lane;
-        const float val = x < staged ? st[x] : -INFINITY;
-        const bool keep = x < staged && val >= th && val > -INFINITY;
-        const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
-        const int at = count + __popc(bal & ((1u << lane) - 1u));
-        if (keep && at < kCandCap) sb[at] = val;
-        count += __popc(bal);
-      }
-      __syncwarp();
-      if (count <= kCandCap) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = (lane * 4 + j < count) ? sb[lane * 4 + j] : -INFINITY;
-        bitonic128_desc(v);
-        done = true;
-      }
-      __syncwarp();
-    }
-    if (!done) {
-      // general path: fold the lists in, one piece at a time
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = -INFINITY;
-      for (int j = 0; j < np; ++j) {
-        const float* src = p.part_topk + ((piece_warp(j, Us, w0, T, W) + seg) * Gq + r) * k;
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int e = lane * 4 + x;
-          if (e >= k) v[x] = (e < 2 * k) ? __ldcg(src + e - k) : -INFINITY;
-        }
-        bitonic128_desc(v);
-      }
-    }
-    float sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (lane * 4 + j < k) sum += exp2_approx(v[j] - M);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    if (lane == 0) p.mass[row] = sum * inv;
   }
 }
 
@@ -408,12 +299,30 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, const
   }
 }
 
+// Unit range [Us, Ue) of segment (i, h) in the call's list of live page-heads.
+__device__ inline void seg_range(const DecodeParams& p, const int32_t* P, int i, int h,
+                                 int64_t* Us, int64_t* Ue) {
+  const int nl = P[i + 1] - P[i];
+  *Us = (int64_t)P[i] * p.Hkv + (int64_t)h * nl;
+  *Ue = *Us + nl;
+}
+
+// The warp of the stream-K split (warp w holds units [w*T/W, (w+1)*T/W))
+// that holds unit u.
+__device__ inline int64_t warp_of_unit(int64_t u, int64_t T, int64_t W) {
+  return ((u + 1) * W - 1) / T;
+}
+
+// Ends the warp's work on segment seg = i * Hkv + h.  If the whole segment
+// was in this warp (Us >= U0 and Ue <= U1) its O rows and top-k mass are
+// written at once; otherwise the warp's piece record goes to rec[w + seg]
+// for the merge.
 template <int D, int G>
-__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t piece,
-                               const TopkCtx& tk, const int32_t* P, int i, int h, int64_t T,
-                               int64_t W, float* scratch) {
+__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t w, int seg,
+                               const TopkCtx& tk, bool whole) {
   constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int i = seg / p.Hkv, h = seg - (seg / p.Hkv) * p.Hkv;
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     S.lp[0] += __shfl_xor_sync(0xFFFFFFFFu, S.lp[0], o);
@@ -425,51 +334,60 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
     }
   }
   const int Gq = p.Gq;
-  float* po = p.part_o + piece * Gq * D;
-  if (g == 0) {
+  const float sinv = pow2i(-S.sigma);
+  const int64_t rb = record_bytes(Gq, D, tk.topk);
+  uint8_t* rec = reinterpret_cast<uint8_t*>(p.rec) + (w + seg) * rb;
+  float* po = reinterpret_cast<float*>(rec + 64);
+  const float li0 = whole ? 1.f / S.lp[0] : 1.f, li1 = whole ? 1.f / S.lp[1] : 1.f;
+  if (!whole && g == 0) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int hd = 2 * t + c;
-      if (hd < Gq) {
-        p.part_ml[(piece * Gq + hd) * 2 + 0] = S.m[c];
-        p.part_ml[(piece * Gq + hd) * 2 + 1] = S.lp[c];
-      }
+      if (hd < Gq) reinterpret_cast<float2*>(rec)[hd] = make_float2(S.m[c], S.lp[c]);
     }
   }
-  const float inv = pow2i(-S.sigma);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int gr = (mt * 16) / G;
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       const int c = x & 1, ch = mt * 16 + g + 8 * (x >> 1), hd = 2 * t + c;
-      if (hd < Gq) po[hd * D + ch] = fmaf(S.acc[mt][x], inv, S.z[gr][c]);
+      if (hd < Gq) {
+        const float o = fmaf(S.acc[mt][x], sinv, S.z[gr][c]);
+        if (whole)
+          p.out[((int64_t)i * p.Hq + h * Gq + hd) * D + ch] =
+              __half_as_ushort(__float2half_rn(o * (c ? li1 : li0)));
+        else
+          po[hd * D + ch] = o;
+      }
     }
   }
   if (tk.topk > 0) {
+    const int kpad = (tk.topk + 3) / 4 * 4;
+    const bool all = whole && p.live_count[p.seq[i]] <= tk.topk;
+    float* tl = reinterpret_cast<float*>(rec + 64 + 4 * Gq * D);
     for (int hd = 0; hd < Gq; ++hd) {
-      if (tk.cnt[hd] > tk.topk) cand_compact(tk, hd);
-      const int n = tk.cnt[hd];
-      float* dst = p.part_topk + (piece * Gq + hd) * tk.topk;
-      for (int j = lane; j < tk.topk; j += 32) dst[j] = j < n ? tk.cand[hd * kCandCap + j] : -INFINITY;
+      float sum = 0.f;
+      if (!all) {
+        if (tk.cnt[hd] > 0) cand_compact(tk, hd);      // sorted, the k largest kept
+        const int n = tk.cnt[hd];
+        if (whole) {
+          const float m = __shfl_sync(0xFFFFFFFFu, (hd & 1) ? S.m[1] : S.m[0], hd >> 1);
+          for (int j = lane; j < n; j += 32) sum += exp2_approx(tk.cand[hd * kCandCap + j] - m);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        } else {
+          for (int j = lane; j < kpad; j += 32)
+            tl[hd * kpad + j] = j < n ? tk.cand[hd * kCandCap + j] : -INFINITY;
+        }
+      }
+      if (whole) {
+        const float l = __shfl_sync(0xFFFFFFFFu, (hd & 1) ? S.lp[1] : S.lp[0], hd >> 1);
+        if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + hd] = all ? 1.f : sum / l;
+      }
     }
-    __syncwarp();
   }
-  // arrival: the last warp to finish a piece of this segment merges all pieces
-  const int nl = P[i + 1] - P[i];
-  const int64_t Us = (int64_t)P[i] * p.Hkv + (int64_t)h * nl, Ue = Us + nl;
-  const int64_t w0 = ((Us + 1) * W - 1) / T, w1 = (Ue * W - 1) / T;
-  // with T <= W every non-empty warp holds exactly one unit; otherwise none is empty
-  const uint32_t npieces = (uint32_t)(T <= W ? (int64_t)nl : w1 - w0 + 1);
-  __threadfence();
   __syncwarp();
-  uint32_t old = 0;
-  if (lane == 0) old = atomicInc(&p.ctr[(int64_t)i * p.Hkv + h], npieces - 1);
-  old = __shfl_sync(0xFFFFFFFFu, old, 0);
-  if (old == npieces - 1) {
-    __threadfence();
-    merge_segment<D>(p, i, h, Us, w0, (int)npieces, T, W, tk, scratch);
-  }
 }
 
 // One live page-head block (in shared memory) of a class with B-bit codes.
@@ -783,7 +701,7 @@ __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P,
   const int nl = P[i + 1] - P[i];
   const int rel = (int)(u - (int64_t)P[i] * p.Hkv);   // < Hkv * max_blocks_per_seq < 2^31
   const int h = rel / nl, j = rel - h * nl;
-  const int64_t row = (int64_t)p.seq[i] * p.max_blocks;
+  const int64_t row = (int64_t)P[p.n + 1 + i] * p.max_blocks;   // the sequence id, cached
   const uint64_t desc = p.live_list[row + j];       // page | class << 32 | entry << 40
   const int cls = entry_class(desc);
   const uint64_t src = reinterpret_cast<uint64_t>(p.pool[cls]) +
@@ -800,7 +718,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_split_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int32_t* P = reinterpret_cast<int32_t*>(smem);
+  int32_t* P = reinterpret_cast<int32_t*>(smem);      // [n + 1] prefix of live pages
+  int32_t* Sq = P + (p.n + 1);                         // [n] the call's sequence ids
+  pdl_launch_dependents();
+  // the call's own inputs may be read before the previous kernel has finished
+  for (int i = tid; i < p.n; i += kDecThreads) Sq[i] = p.seq[i];
+  // everything below reads cache state: wait for the previous kernel
+  pdl_wait();
+  __syncthreads();
 
   // ---- prefix of live pages over the call's sequences (per CTA) ----
   {
@@ -810,7 +735,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       const int i = base + tid;
       int v = 0;
       if (i < p.n) {
-        const int s = p.seq[i];
+        const int s = Sq[i];
         if (s >= 0 && s < p.max_seqs) v = p.num_live[s];
         else if (blockIdx.x == 0) set_status(p.status, THINKV_ERR_INVALID);  // decoded as empty
       }
@@ -833,6 +758,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     if (tid == 0) P[p.n] = carry;
     __syncthreads();
   }
+  if (blockIdx.x == 0)
+    for (int x = tid; x <= p.n; x += kDecThreads) p.pref[x] = P[x];   // for the combine
   write_empty_outputs(p, P, D);
 
   const int64_t T = (int64_t)P[p.n] * p.Hkv;
@@ -894,6 +821,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   int seg = -1;
   int stage = 0;
   uint32_t parity = 0;
+  bool failed = false;
   for (int k = 0; k < nu; ++k) {
     const int kk = k & 31;
     if (kk == 0 && k > 0) {
@@ -902,11 +830,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     }
     if (!mbar_wait_bounded(&bars[stage], parity)) {
       if (lane == 0) set_status(p.status, THINKV_ERR_TIMEOUT);
-      // drain the copies still in flight (bounded), then leave
+      // drain the copies still in flight (bounded), then stop
       const int issued = k == 0 ? 1 : min(nu, k + p.nstage);
       for (int k2 = k + 1; k2 < issued; ++k2)
         mbar_wait_bounded(&bars[k2 % p.nstage], (uint32_t)((k2 / p.nstage) & 1));
-      return;
+      failed = true;
+      break;
     }
     if (k == 0)
       for (int s2 = 1; s2 < p.nstage && s2 < nu; ++s2) issue(cur, s2, s2);
@@ -914,7 +843,11 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     const int useg = (int)(cs & 0xFFFFFFu);
     uint8_t* blk = wsm + stage * p.stage_bytes;
     if (useg != seg) {
-      if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, seg / p.Hkv, seg % p.Hkv, T, W, pbuf);
+      if (seg >= 0) {
+        int64_t Us, Ue;
+        seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
+        seg_end<D, G>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
+      }
       seg = useg;
       seg_begin<D, G>(S, p, reinterpret_cast<const uint16_t*>(blk + p.q_off),
                       reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(pbuf) + kQfragOff), tk);
@@ -931,7 +864,120 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       parity ^= 1u;
     }
   }
-  if (seg >= 0) seg_end<D, G>(S, p, w + seg, tk, P, seg / p.Hkv, seg % p.Hkv, T, W, pbuf);
+  if (failed || seg < 0) return;
+  {
+    int64_t Us, Ue;
+    seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
+    seg_end<D, G>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// split combine: one CTA per (sequence, kv-head) segment that the split
+// kernel left in more than one piece
+// ---------------------------------------------------------------------------
+constexpr int kCombineThreads = 256;
+
+// Merges the segment's piece records with the log-sum-exp rule: thread t <
+// Gq * D/4 owns one quad of one head's output row; warp r < Gq then merges
+// head r's top-k lists (bitonic merges, the next piece's list loaded while the
+// current one merges) for the top-k mass.
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(DecodeParams p) {
+  constexpr int QD = D / 4;
+  __shared__ float sM[8], sL[8];
+  pdl_launch_dependents();
+  pdl_wait();                                   // records and prefix come from the split kernel
+  const int seg = blockIdx.x;
+  const int i = seg / p.Hkv, h = seg - (seg / p.Hkv) * p.Hkv;
+  const int nl = p.pref[i + 1] - p.pref[i];
+  if (nl == 0) return;                          // written by the split kernel
+  const int64_t T = (int64_t)p.pref[p.n] * p.Hkv, W = p.split_warps;
+  const int64_t Us = (int64_t)p.pref[i] * p.Hkv + (int64_t)h * nl, Ue = Us + nl;
+  const int64_t w0 = warp_of_unit(Us, T, W), w1 = warp_of_unit(Ue - 1, T, W);
+  const bool by_unit = T <= W;                  // one unit per warp
+  const int np = (int)(by_unit ? nl : w1 - w0 + 1);
+  if (np <= 1) return;                          // finished inside one split warp
+  const int Gq = p.Gq, k = p.topk, kpad = (k + 3) / 4 * 4;
+  const int64_t rb = record_bytes(Gq, D, k);
+  const uint8_t* recs = reinterpret_cast<const uint8_t*>(p.rec);
+  auto rec = [&](int j) -> const uint8_t* {
+    const int64_t pc = (by_unit ? warp_of_unit(Us + j, T, W) : w0 + j) + seg;
+    return recs + pc * rb;
+  };
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- output rows ----
+  if (tid < Gq * QD) {
+    const int r = tid / QD, q = tid - r * QD;
+    float M = -INFINITY;
+#pragma unroll 4
+    for (int j = 0; j < np; ++j)
+      M = fmaxf(M, __ldcg(reinterpret_cast<const float*>(rec(j)) + 2 * r));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int j = 0; j < np; ++j) {
+      const uint8_t* rj = rec(j);
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(rj) + r);
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(rj + 64) + r * QD + q);
+      const float wgt = exp2_approx(ml.x - M);
+      L = fmaf(wgt, ml.y, L);
+      acc.x = fmaf(wgt, v.x, acc.x);
+      acc.y = fmaf(wgt, v.y, acc.y);
+      acc.z = fmaf(wgt, v.z, acc.z);
+      acc.w = fmaf(wgt, v.w, acc.w);
+    }
+    const float inv = 1.f / L;
+    const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc.x * inv)) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(acc.y * inv)) << 16);
+    const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc.z * inv)) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(acc.w * inv)) << 16);
+    const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
+    reinterpret_cast<uint2*>(p.out + row * D)[q] = make_uint2(lo, hi);
+    if (q == 0) { sM[r] = M; sL[r] = L; }
+  }
+  if (!p.mass) return;
+  __syncthreads();
+  if (warp >= Gq) return;
+  const int r = warp;
+  const int64_t mrow = (int64_t)i * p.Hq + h * Gq + r;
+  if (p.live_count[p.seq[i]] <= k) {
+    if (lane == 0) p.mass[mrow] = 1.f;
+    return;
+  }
+  // running list (descending) in elements 0..63, the next piece's list
+  // reversed in 64..127: a bitonic sequence
+  float tv[4], nx[4];
+  auto load_list = [&](int j, float (&x)[4]) {
+    const float* tl = reinterpret_cast<const float*>(rec(j) + 64 + 4 * Gq * D) + r * kpad;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int el = lane * 4 + e, m = 127 - el;
+      x[e] = (el >= 64 && m < k) ? __ldcg(tl + m) : -INFINITY;
+    }
+  };
+#pragma unroll
+  for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
+  load_list(0, nx);
+  for (int j = 0; j < np; ++j) {
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = (lane * 4 + e < 64) ? tv[e] : nx[e];
+    if (j + 1 < np) load_list(j + 1, nx);
+    bitonic128_merge_desc(v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tv[e] = v[e];
+  }
+  const float M = sM[r];
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (lane * 4 + e < k) sum += exp2_approx(tv[e] - M);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  if (lane == 0) p.mass[mrow] = sum / sL[r];
 }
 
 template <int D, int G>
@@ -948,11 +994,15 @@ cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStre
     if (e != cudaSuccess) return e;
     configured[dev] = dl.smem_bytes;
   }
-  decode_split_kernel<D, G><<<dl.grid, kDecThreads, dl.smem_bytes, stream>>>(p);
-  return cudaGetLastError();
+  e = launch_pdl(decode_split_kernel<D, G>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
+                 stream, p);
+  if (e != cudaSuccess) return e;
+  // the combine: one CTA per segment (most return at once)
+  return launch_pdl(decode_combine_kernel<D>, dim3((unsigned)(p.n * p.Hkv)),
+                    dim3(kCombineThreads), 0, stream, p);
 }
 
-int plan_smem_bytes(int32_t n) { return ((n + 1) * 4 + 127) / 128 * 128; }
+int plan_smem_bytes(int32_t n) { return ((2 * n + 1) * 4 + 127) / 128 * 128; }
 
 }  // namespace
 
@@ -970,7 +1020,7 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
   // ~15 KB of page-head stages per warp keeps three 4-warp CTAs per SM
   int nstage = (int)(15360 / stage_bytes);
   if (nstage < 2) nstage = 2;
-  if (nstage > 8) nstage = 8;
+  if (nstage > kMaxStages) nstage = kMaxStages;
   const int Gq = L.num_q_heads / L.num_kv_heads;
   const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes +
                         (topk > 0 ? kTopkHdrBytes + Gq * kCandCap * 4 : 0);
@@ -1002,16 +1052,18 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
   out->smem_bytes = smem;
   out->warp_smem = warp_smem;
   out->pieces = (int64_t)out->grid * kDecWarps + (int64_t)n_seqs * L.num_kv_heads;
+
   return true;
 }
 
 size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
                               const DecodeLaunch& dl) {
   const int Gq = L.num_q_heads / L.num_kv_heads;
-  size_t b = ((size_t)n_seqs * L.num_kv_heads * 4 + 255) / 256 * 256;  // arrival counters
-  b += ((size_t)dl.pieces * Gq * 2 * 4 + 255) / 256 * 256;
-  b += ((size_t)dl.pieces * Gq * L.head_dim * 4 + 255) / 256 * 256;
-  b += ((size_t)dl.pieces * Gq * (topk > 0 ? topk : 0) * 4 + 255) / 256 * 256;
+  // the prefix of live pages, then one record per (split warp, segment)
+  const size_t head = (size_t)(n_seqs + 1 > n_seqs * L.num_kv_heads ? n_seqs + 1
+                                                                     : n_seqs * L.num_kv_heads);
+  size_t b = (head * 4 + 255) / 256 * 256;
+  b += (size_t)dl.pieces * (size_t)record_bytes(Gq, L.head_dim, topk > 0 ? topk : 0);
   return b;
 }
 
@@ -1040,14 +1092,14 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
   uint8_t* w = static_cast<uint8_t*>(ws);
-  p.ctr = reinterpret_cast<uint32_t*>(w);
-  w += ((size_t)n * L.num_kv_heads * 4 + 255) / 256 * 256;
-  p.part_ml = reinterpret_cast<float*>(w);
-  w += ((size_t)dl.pieces * p.Gq * 2 * 4 + 255) / 256 * 256;
-  p.part_o = reinterpret_cast<float*>(w);
-  w += ((size_t)dl.pieces * p.Gq * D * 4 + 255) / 256 * 256;
-  p.part_topk = reinterpret_cast<float*>(w);
+  p.pref = reinterpret_cast<int32_t*>(w);
+  {
+    const size_t head = (size_t)(n + 1 > n * L.num_kv_heads ? n + 1 : n * L.num_kv_heads);
+    w += (head * 4 + 255) / 256 * 256;
+  }
   p.topk = mass ? topk : 0;
+  p.rec = w;
+  p.split_warps = (int64_t)dl.grid * kDecWarps;
   p.live_count = C.live_count;
   p.out = out;
   p.mass = p.topk > 0 ? mass : nullptr;

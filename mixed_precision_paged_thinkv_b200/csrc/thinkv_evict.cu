@@ -132,6 +132,154 @@ __global__ void __launch_bounds__(kEvictThreads, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// small calls (n <= kSmallEvict sequences, e.g. a decode step): one warp per
+// sequence over many CTAs.  Every CTA validates the whole call itself (the
+// same verdict everywhere, so the call stays all-or-nothing without a
+// grid-wide barrier); sequences share no state, so the warps are independent.
+// ---------------------------------------------------------------------------
+constexpr int kSmallEvict = 512;
+constexpr int kSmallEvictThreads = 256;
+constexpr int kSmallEvictWarps = kSmallEvictThreads / 32;
+
+// Evicts sequence s down to `bud` live tokens (one warp).  The class order is
+// packed one class per byte.  All of s's counters are loaded at once (with
+// the sticky status when check_status: a set status makes this a no-op); the
+// victims of all classes are then taken 32 at a time in victim order.
+__device__ void evict_seq(const CacheView& C, int s, int bud, uint32_t order,
+                          bool check_status = false) {
+  const int lane = threadIdx.x & 31;
+  const int nb_max = C.L.max_blocks_per_seq;
+  const int64_t cap = (int64_t)nb_max * kPage;
+  // lanes 0-2: FIFO heads, 3-5: FIFO tails, 6-8: stack tops (classes in
+  // order), 9: live_count, 10: num_live
+  int val = 0;
+  {
+    const int o = lane % 3, c = (int)((order >> (8 * o)) & 0xFFu);
+    if (lane < 3) val = C.fifo_head[s * 3 + c];
+    else if (lane < 6) val = C.fifo_tail[s * 3 + c];
+    else if (lane < 9) val = C.free_top[s * 3 + c];
+    else if (lane == 9) val = C.live_count[s];
+    else if (lane == 10) val = C.num_live[s];
+    else if (lane == 11 && check_status) val = *C.status;
+  }
+  if (check_status && __shfl_sync(0xFFFFFFFFu, val, 11) != 0) return;
+  const int live = __shfl_sync(0xFFFFFFFFu, val, 9);
+  int nlive = __shfl_sync(0xFFFFFFFFu, val, 10);
+  int remaining = live - bud;
+  if (remaining <= 0) return;
+  int head[3], take[3], top[3], cum[3];
+  int total = 0;
+#pragma unroll
+  for (int o = 0; o < 3; ++o) {
+    head[o] = __shfl_sync(0xFFFFFFFFu, val, o);
+    const int tail = __shfl_sync(0xFFFFFFFFu, val, 3 + o);
+    top[o] = __shfl_sync(0xFFFFFFFFu, val, 6 + o);
+    take[o] = min(max(tail - head[o], 0), remaining);
+    remaining -= take[o];
+    total += take[o];
+    cum[o] = total;                                  // victims of classes 0..o
+  }
+  uint64_t* table = C.block_table + (int64_t)s * nb_max;
+  uint64_t* llist = C.live_list + (int64_t)s * nb_max;
+  int32_t* lidx = C.live_index + (int64_t)s * nb_max;
+  for (int v0 = 0; v0 < total; v0 += 32) {
+    const int vv = v0 + lane;
+    const bool valid = vv < total;
+    const int o = vv < cum[0] ? 0 : (vv < cum[1] ? 1 : 2);
+    const int c = (int)((order >> (8 * o)) & 0xFFu);
+    const int r = vv - (o == 0 ? 0 : (o == 1 ? cum[0] : cum[1]));   // rank inside the class
+    const int hd = o == 0 ? head[0] : (o == 1 ? head[1] : head[2]);
+    const int tp = o == 0 ? top[0] : (o == 1 ? top[1] : top[2]);
+    int32_t ts = 0;
+    if (valid) ts = C.fifo[((int64_t)s * 3 + c) * cap + ((int64_t)hd + r) % cap];
+    const int e = ts >> 4, slot = ts & 15;
+    // merge the bits of victims that share an entry (entries are class-pure);
+    // the highest such lane writes the entry
+    const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? e : -1 - lane);
+    const uint32_t bits = __reduce_or_sync(grp, valid ? (1u << slot) : 0u);
+    const bool last = valid && (31 - __clz(grp)) == lane;
+    bool emptied = false;
+    if (valid) {
+      // through L2: an earlier batch may have rewritten this entry
+      const uint64_t ent = __ldcg(&table[e]);
+      const uint32_t page = entry_page(ent);
+      if (last) {
+        const uint32_t mask = entry_mask(ent) & ~bits;
+        table[e] = (ent & 0x0000FFFFFFFFFFFFull) | ((uint64_t)mask << 48);
+        emptied = (mask == 0);
+      }
+      C.slot_pos[c][(int64_t)page * kPage + slot] = -1;
+      C.free_slots[((int64_t)s * 3 + c) * cap + tp + r] = ts;
+    }
+    // entries emptied in this batch leave the live list in victim order
+    unsigned ev = __ballot_sync(0xFFFFFFFFu, emptied);
+    __syncwarp();
+    while (ev) {
+      const int src = __ffs(ev) - 1;
+      const int ee = __shfl_sync(0xFFFFFFFFu, e, src);
+      if (lane == 0) {
+        const int lastpos = nlive - 1;
+        const int at = __ldcg(&lidx[ee]);
+        const uint64_t moved = __ldcg(&llist[lastpos]);
+        llist[at] = moved;
+        lidx[live_desc_entry(moved)] = at;
+        lidx[ee] = -1;
+      }
+      --nlive;
+      __syncwarp();
+      ev &= ev - 1;
+    }
+  }
+  if (lane < 3) {
+    const int c = (int)((order >> (8 * lane)) & 0xFFu);
+    C.fifo_head[s * 3 + c] = head[lane == 0 ? 0 : (lane == 1 ? 1 : 2)] + take[lane == 0 ? 0 : (lane == 1 ? 1 : 2)];
+    C.free_top[s * 3 + c] = top[lane == 0 ? 0 : (lane == 1 ? 1 : 2)] + take[lane == 0 ? 0 : (lane == 1 ? 1 : 2)];
+  }
+  if (lane == 0) {
+    C.live_count[s] = live - total;
+    C.num_live[s] = nlive;
+  }
+}
+
+__global__ void __launch_bounds__(kSmallEvictThreads)
+    evict_small_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
+                       const int32_t* __restrict__ budget, uint32_t order) {
+  extern __shared__ uint32_t seen[];  // max_seqs bits
+  __shared__ int s_err;
+  __shared__ int my_seq[kSmallEvictWarps], my_bud[kSmallEvictWarps];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int max_seqs = C.L.max_seqs;
+  const int first = blockIdx.x * kSmallEvictWarps;
+  pdl_launch_dependents();
+  // ---- the call's own inputs (before the previous kernel has finished) ----
+  for (int i = tid; i < (max_seqs + 31) / 32; i += kSmallEvictThreads) seen[i] = 0;
+  if (tid == 0) s_err = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kSmallEvictThreads) {
+    const int s = seq[i], b = budget[i];
+    bool bad = s < 0 || s >= max_seqs || b < 0;
+    if (!bad) {
+      const uint32_t old = atomicOr(&seen[s >> 5], 1u << (s & 31));
+      if (old & (1u << (s & 31))) bad = true;
+    }
+    if (bad) s_err = THINKV_ERR_INVALID;
+    if (i >= first && i < first + kSmallEvictWarps) {
+      my_seq[i - first] = s;
+      my_bud[i - first] = b;
+    }
+  }
+  __syncthreads();
+  // ---- cache state: only once the previous kernel is done ----
+  pdl_wait();
+  if (s_err != 0) {
+    if (blockIdx.x == 0 && tid == 0) set_status(C.status, s_err);
+    return;
+  }
+  const int i = first + warp;
+  if (i < n) evict_seq(C, my_seq[warp], my_bud[warp], order, true);
+}
 }  // namespace
 
 cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
@@ -142,6 +290,12 @@ cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, cons
   o.c[2] = order[2];
   o.c[3] = 0;
   const size_t seen_bytes = (size_t)((C.L.max_seqs + 31) / 32) * 4;
+  if (n <= kSmallEvict) {
+    const uint32_t packed = (uint32_t)order[0] | ((uint32_t)order[1] << 8) | ((uint32_t)order[2] << 16);
+    const int grid = (n + kSmallEvictWarps - 1) / kSmallEvictWarps;
+    return launch_pdl(evict_small_kernel, dim3(grid), dim3(kSmallEvictThreads), seen_bytes, stream,
+                      C, n, seq, budget, packed);
+  }
   evict_kernel<<<1, kEvictThreads, seen_bytes, stream>>>(C, n, seq, budget, o);
   return cudaGetLastError();
 }

@@ -39,6 +39,7 @@ struct RunInfo {
 };
 
 struct AppendWorkspace {
+  uint32_t* arrive;   // arrival counter of the one-launch path (zero between calls)
   int32_t* ok;        // 1 once the slot assignment succeeded
   int32_t* tok_slot;  // [n] pool slot id (page*16 + slot) of every token
   RunInfo* runs;      // [n] sequence runs
@@ -65,7 +66,7 @@ struct DecodeLaunch {
   int stage_bytes;     // bytes per stage
   size_t smem_bytes;   // dynamic shared memory of the split kernel
   int warp_smem;       // bytes of shared memory per warp
-  int64_t pieces;      // partial slots
+  int64_t pieces;      // piece records (warps + segments)
 };
 bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, int device,
                         DecodeLaunch* out);

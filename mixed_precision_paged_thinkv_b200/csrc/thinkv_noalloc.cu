@@ -3,9 +3,10 @@
 // For callers that cannot allocate device memory where they decode (a host
 // framework that owns all device memory and gives its plugins no allocator;
 // paths that cannot afford cudaMalloc's device-wide synchronisation).  The
-// split-K scratch of the decode kernel -- arrival counters, per-piece
-// partial outputs and top-k lists -- is one file-scope device array of fixed
-// size instead of a caller workspace.  The ThinKV pages have no counterpart.
+// split-K scratch of the decode kernels -- the live-page prefix and the
+// per-piece partial outputs and top-k lists -- is one file-scope device array
+// of fixed size instead of a caller workspace.  The ThinKV pages have no
+// counterpart.
 #include <cuda_runtime.h>
 #include <mutex>
 #include <stdint.h>
@@ -61,9 +62,6 @@ extern "C" int thinkv_decode_attention_noalloc(const thinkv_cache* C, int32_t n,
   void* ws = nullptr;
   if (scratch_address(&ws) != cudaSuccess) return THINKV_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the arrival counters (first n * Hkv words) must start at zero
-  if (cudaMemsetAsync(ws, 0, (size_t)n * C->L.num_kv_heads * sizeof(uint32_t), s) != cudaSuccess)
-    return THINKV_ERR_CUDA;
   return launch_decode(view_of(C), n, seq, q, out, topk_mass, k, softmax_scale, ws, dl, s) ==
                  cudaSuccess
              ? THINKV_OK

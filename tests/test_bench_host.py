@@ -65,3 +65,10 @@ def test_replicas_reduce_max_time_and_sum_tokens_over_two_ranks():
     got = sorted(q.get(timeout=10) for _ in range(2))
     for r, m, n in got:
         assert m == 2.5 and n == 32.0
+
+
+def test_launches_per_step_counts_the_one_launch_append_path():
+    import bench
+    assert bench.launches_per_step(16) == 4
+    assert bench.launches_per_step(512) == 4
+    assert bench.launches_per_step(513) == 5
