@@ -27,6 +27,7 @@
 //   log-sum-exp rule -- a thread per quad of each head's output row, a warp per
 //   head for the top-k lists -- and writes fp16 O and the top-k mass.
 #include <cuda_fp16.h>
+#include <limits.h>
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
@@ -494,16 +495,24 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   }
 
   // ---------------- online softmax (heads 2t, 2t+1) ----------------
-  float pm0 = fmaxf(lg[0], lg[2]), pm1 = fmaxf(lg[1], lg[3]);
+  // Most pages raise no head's running max: the max over the page's tokens is
+  // only formed (and the rescale factors with it) when some logit exceeds it.
+  float a0 = 1.f, a1 = 1.f;
+  float mn0 = S.m[0], mn1 = S.m[1];
+  if (__any_sync(0xFFFFFFFFu, fmaxf(lg[0], lg[2]) > mn0 || fmaxf(lg[1], lg[3]) > mn1)) {
+    float pm0 = fmaxf(lg[0], lg[2]), pm1 = fmaxf(lg[1], lg[3]);
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    pm0 = fmaxf(pm0, __shfl_xor_sync(0xFFFFFFFFu, pm0, o));
-    pm1 = fmaxf(pm1, __shfl_xor_sync(0xFFFFFFFFu, pm1, o));
+    for (int o = 4; o < 32; o <<= 1) {
+      pm0 = fmaxf(pm0, __shfl_xor_sync(0xFFFFFFFFu, pm0, o));
+      pm1 = fmaxf(pm1, __shfl_xor_sync(0xFFFFFFFFu, pm1, o));
+    }
+    mn0 = fmaxf(S.m[0], pm0);
+    mn1 = fmaxf(S.m[1], pm1);
+    a0 = exp2_approx(S.m[0] - mn0);
+    a1 = exp2_approx(S.m[1] - mn1);
+    S.m[0] = mn0;
+    S.m[1] = mn1;
   }
-  const float mn0 = fmaxf(S.m[0], pm0), mn1 = fmaxf(S.m[1], pm1);
-  const float a0 = exp2_approx(S.m[0] - mn0), a1 = exp2_approx(S.m[1] - mn1);
-  S.m[0] = mn0;
-  S.m[1] = mn1;
   float pr[4];
   pr[0] = exp2_approx(lg[0] - mn0);
   pr[1] = exp2_approx(lg[1] - mn1);
@@ -608,7 +617,8 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
     }
   }
 
-  // ---------------- O^T += V^T(codes - 2^(b-1)) x W ----------------
+  // ---------------- O^T += V^T(codes - 2^(b-1)) x W, per m-tile: V^T(1024 + codes) x W
+  //                  plus one constant-row product that removes 1024 + 2^(b-1) ----------------
   {
     constexpr int Q = (B == 16) ? D / 8 : D * B / 128;   // words per token pair
     constexpr int PER = (B == 16) ? 1 : 16 / B;          // codes per half-word
@@ -653,13 +663,18 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
             if constexpr (B == 16) {
               a[P * 2 + r] = vr[P][wq] & (P ? dm1 : dm0);   // raw values of dead slots: zero
             } else {
-              // centred code pair c - 2^(b-1), exact in fp16: the sum over a
-              // whole segment then carries no large offset to cancel
-              a[P * 2 + r] = hsub2_bits(unpack_pair<B>(vr[P][wq], e % PER), centre_bits<B>());
+              a[P * 2 + r] = unpack_pair<B>(vr[P][wq], e % PER);   // 1024 + code
             }
           }
         }
         mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
+        if constexpr (B != 16) {
+          // centre at once: + (-(1024 + 2^(b-1))) * sum of W over the page's
+          // tokens, so the segment's accumulators never carry the offset
+          const uint32_t kc = neg_centre_bits<B>();
+          const uint32_t ka[4] = {kc, kc, kc, kc};
+          mma_16816(S.acc[mt], ka, wf[gr][0], wf[gr][1]);
+        }
       }
     }
   }
@@ -878,6 +893,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // kernel left in more than one piece
 // ---------------------------------------------------------------------------
 constexpr int kCombineThreads = 256;
+constexpr int kCombinePieces = 128;             // pieces per round of the weight table
+constexpr int kCombinePre = 16;                 // pieces whose quads are requested up front
 
 // Merges the segment's piece records with the log-sum-exp rule: thread t <
 // Gq * D/4 owns one quad of one head's output row; warp r < Gq then merges
@@ -887,6 +904,8 @@ template <int D>
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(DecodeParams p) {
   constexpr int QD = D / 4;
   __shared__ float sM[8], sL[8];
+  __shared__ int sMk[8];
+  __shared__ float cwt[kCombinePieces * 8], lt[kCombinePieces * 8];
   pdl_launch_dependents();
   pdl_wait();                                   // records and prefix come from the split kernel
   const int seg = blockIdx.x;
@@ -908,38 +927,92 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(DecodeP
   };
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // ---- output rows ----
-  if (tid < Gq * QD) {
-    const int r = tid / QD, q = tid - r * QD;
-    float M = -INFINITY;
-#pragma unroll 4
-    for (int j = 0; j < np; ++j)
-      M = fmaxf(M, __ldcg(reinterpret_cast<const float*>(rec(j)) + 2 * r));
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int j = 0; j < np; ++j) {
-      const uint8_t* rj = rec(j);
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(rj) + r);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(rj + 64) + r * QD + q);
-      const float wgt = exp2_approx(ml.x - M);
-      L = fmaf(wgt, ml.y, L);
-      acc.x = fmaf(wgt, v.x, acc.x);
-      acc.y = fmaf(wgt, v.y, acc.y);
-      acc.z = fmaf(wgt, v.z, acc.z);
-      acc.w = fmaf(wgt, v.w, acc.w);
+  // ---- per piece and head: the weight 2^(m - M) (M the head's max), and L ----
+  // (m, l) pairs are read once, lane-parallel; a table of weights in shared
+  // memory then lets every output thread stream its quads with many loads in
+  // flight.  Segments with more pieces than the table holds go in rounds.
+  float* wt = cwt;                                // [kCombinePieces][8]
+  // a float's order-preserving int key (negative floats: magnitude bits
+  // flipped); the map is its own inverse
+  auto okey = [](int b) { return b >= 0 ? b : b ^ 0x7FFFFFFF; };
+  const int r_o = tid / QD, q_o = tid - (tid / QD) * QD;
+  const bool out_thread = tid < Gq * QD;
+  auto quad = [&](int j) {
+    return __ldcg(reinterpret_cast<const float4*>(rec(j) + 64) + r_o * QD + q_o);
+  };
+  auto pair_ml = [&](int x) {
+    const int j = x / Gq, r = x - j * Gq;
+    return __ldcg(reinterpret_cast<const float2*>(rec(j)) + r);
+  };
+  // the first pieces' quads and (m, l) pairs do not depend on the weights:
+  // all of them are requested at once
+  float4 ov[kCombinePre];
+#pragma unroll
+  for (int j = 0; j < kCombinePre; ++j)
+    ov[j] = (out_thread && j < np) ? quad(j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float2 ml0 = tid < np * Gq ? pair_ml(tid) : make_float2(-INFINITY, 0.f);
+  if (tid < 8) { sMk[tid] = INT_MIN; sL[tid] = 0.f; }
+  __syncthreads();
+  for (int x = tid; x < np * Gq; x += kCombineThreads) {
+    const float m = x == tid ? ml0.x : pair_ml(x).x;
+    atomicMax(&sMk[x - (x / Gq) * Gq], okey(__float_as_int(m)));
+  }
+  __syncthreads();
+  if (tid < 8) sM[tid] = __int_as_float(okey(sMk[tid]));
+  __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < np; j0 += kCombinePieces) {
+    const int cnt = min(kCombinePieces, np - j0);
+    for (int x = tid; x < cnt * Gq; x += kCombineThreads) {
+      const int j = x / Gq, r = x - j * Gq;
+      const float2 ml = (j0 == 0 && x == tid) ? ml0 : pair_ml(j0 * Gq + x);
+      const float wgt = exp2_approx(ml.x - sM[r]);
+      wt[j * 8 + r] = wgt;
+      lt[j * 8 + r] = wgt * ml.y;
     }
-    const float inv = 1.f / L;
+    __syncthreads();
+    if (warp < Gq) {                              // L, summed in a fixed order
+      float l = 0.f;
+      for (int j = lane; j < cnt; j += 32) l += lt[j * 8 + warp];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+      if (lane == 0) sL[warp] += l;
+    }
+    if (out_thread) {
+      int jstart = 0;
+      if (j0 == 0) {
+#pragma unroll
+        for (int j = 0; j < kCombinePre; ++j) {
+          const float wgt = j < cnt ? wt[j * 8 + r_o] : 0.f;
+          acc.x = fmaf(wgt, ov[j].x, acc.x);
+          acc.y = fmaf(wgt, ov[j].y, acc.y);
+          acc.z = fmaf(wgt, ov[j].z, acc.z);
+          acc.w = fmaf(wgt, ov[j].w, acc.w);
+        }
+        jstart = kCombinePre;
+      }
+#pragma unroll 8
+      for (int j = jstart; j < cnt; ++j) {
+        const float4 v = quad(j0 + j);
+        const float wgt = wt[j * 8 + r_o];
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
+      }
+    }
+    __syncthreads();                              // the table is refilled by the next round
+  }
+  if (tid < Gq * QD) {
+    const float inv = 1.f / sL[r_o];
     const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc.x * inv)) |
                         ((uint32_t)__half_as_ushort(__float2half_rn(acc.y * inv)) << 16);
     const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc.z * inv)) |
                         ((uint32_t)__half_as_ushort(__float2half_rn(acc.w * inv)) << 16);
-    const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
-    reinterpret_cast<uint2*>(p.out + row * D)[q] = make_uint2(lo, hi);
-    if (q == 0) { sM[r] = M; sL[r] = L; }
+    const int64_t row = (int64_t)i * p.Hq + h * Gq + r_o;
+    reinterpret_cast<uint2*>(p.out + row * D)[q_o] = make_uint2(lo, hi);
   }
   if (!p.mass) return;
-  __syncthreads();
   if (warp >= Gq) return;
   const int r = warp;
   const int64_t mrow = (int64_t)i * p.Hq + h * Gq + r;
