@@ -115,8 +115,10 @@ typedef struct {
  *   [0, 2db)          K codes      [2db, 4db)  V codes
  *   [4db, 4db+64ng)   K params     [4db+64ng, 4db+128ng)  V params
  * params: [group ng][slot 16][scale, zero] fp16.
- * Codes of one block are "lane-major": 32 lanes x (d*b/16) bytes; lane
- * l = 4*gid + tid (gid 0..7, tid 0..3).  Within 32-bit words (or a 16-bit
+ * Each code region (K, V) holds a portion of d*b/16 bytes for each of 32
+ * lanes, l = 4*gid + tid (gid 0..7, tid 0..3).  The portions are interleaved
+ * in chunks of u = min(16, d*b/16) bytes: byte o of lane l's portion is at
+ * (o / u)*32*u + l*u + o % u of the region.  Within 32-bit words (or a 16-bit
  * piece) the codes of even channels sit in the low half and those of odd
  * channels in the high half, each half little-endian.
  *   K: lane l holds, for group gr = 0..ng-1 and r = 0..1, the codes of slot
@@ -127,7 +129,7 @@ typedef struct {
  *      high 16 bits; each half holds 16/b codes, element k of chunk q being
  *      channel 16*(e/2) + gid + 8*(e%2) with e = q*16/b + k.
  * For b == 16 the block is K raw fp16 [2db) then V raw fp16 [2db), in the same
- * lane-major orders, with no params.
+ * lane orders and chunk interleave, with no params.
  *
  * Quantiser (reading of TBQ's group quantisation): per token, per kv-head,
  * per K|V, per group of G consecutive channels: zero = min rounded toward

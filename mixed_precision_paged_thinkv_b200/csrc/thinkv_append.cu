@@ -15,7 +15,8 @@
 //      workspace, and a go/no-go flag (the call is all-or-nothing).
 //   2. append_scatter_kernel (grid): one warp per (token, kv-head, K|V):
 //      group min/max by warp shuffles, directed-rounded fp16 zero/scale,
-//      round-half-even codes, then scatter into the lane-major page-head block.
+//      round-half-even codes, then scatter into the page-head block (lane
+//      portions interleaved in 16-byte chunks).
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -398,7 +399,7 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
   }
   __syncwarp();
 
-  const int64_t lane_bytes = (int64_t)D * b / 16;
+  const int lane_bytes = D * b / 16;
   uint8_t* region = blk + (kv ? 2LL * D * b : 0);
   if (kv == 0) {
     // K: pieces (layout lane 4*(slot%8)+t, group gr, r = slot/8) of G/4 channels
@@ -408,10 +409,11 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
       // raw fp16: the piece is G/4 channels in natural order
       const int t = lane & 3, gr = lane >> 2;
       const int l = 4 * (slot & 7) + t, r = slot >> 3;
-      uint8_t* dst = region + l * lane_bytes + (int64_t)(gr * 2 + r) * pb;
+      const int o = (gr * 2 + r) * pb;
       const uint16_t* src = code_sm + gr * G + t * (G / 4);
       for (int e = 0; e < G / 4; e += 2)
-        *reinterpret_cast<uint32_t*>(dst + 2 * e) = (uint32_t)src[e] | ((uint32_t)src[e + 1] << 16);
+        *reinterpret_cast<uint32_t*>(region + lane_off(l, o + 2 * e, lane_bytes)) =
+            (uint32_t)src[e] | ((uint32_t)src[e + 1] << 16);
     } else if (lane < 4 * NG) {
       const int t = lane & 3, gr = lane >> 2;
       const int l = 4 * (slot & 7) + t, r = slot >> 3;
@@ -422,7 +424,7 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
         const int p = (el & 1) ? (m / 2 + el / 2) : (el / 2);
         words[wi] |= v << (p * b);
       }
-      uint8_t* dst = region + l * lane_bytes + (int64_t)(gr * 2 + r) * pb;
+      uint8_t* dst = region + lane_off(l, (gr * 2 + r) * pb, lane_bytes);   // pb <= chunk
       if (pb == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)words[0];
       else if (pb == 4) *reinterpret_cast<uint32_t*>(dst) = words[0];
       else if (pb == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
@@ -442,7 +444,7 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
         hw |= (uint32_t)code_sm[ch] << (b * k);
       }
       const int l = 4 * g + t;
-      uint8_t* dst = region + l * lane_bytes + (int64_t)(P * Q + q) * 4 + 2 * half;
+      uint8_t* dst = region + lane_off(l, (P * Q + q) * 4 + 2 * half, lane_bytes);
       *reinterpret_cast<uint16_t*>(dst) = (uint16_t)hw;
     }
   }

@@ -26,6 +26,16 @@ __host__ __device__ inline int64_t page_head_bytes(int d, int G, int b) {
   return 4LL * d * b + 128LL * (d / G);
 }
 
+// Code regions of a page-head block hold 32 lanes x lane_bytes bytes; the
+// lanes' portions are interleaved in chunks of min(16, lane_bytes) bytes, so
+// that 32 lanes reading the same chunk read one contiguous span of shared
+// memory (no bank conflicts).  Offset of byte o of lane l's portion:
+__host__ __device__ inline int chunk_bytes(int lane_bytes) { return lane_bytes < 16 ? lane_bytes : 16; }
+__host__ __device__ inline int lane_off(int lane, int o, int lane_bytes) {
+  const int u = chunk_bytes(lane_bytes);
+  return (o / u) * 32 * u + lane * u + (o % u);
+}
+
 // Table entry fields.
 __host__ __device__ inline uint32_t entry_page(uint64_t e) { return (uint32_t)(e & 0xFFFFFFFFull); }
 __host__ __device__ inline int entry_class(uint64_t e) { return (int)((e >> 32) & 0xFF); }

@@ -391,6 +391,26 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
   __syncwarp();
 }
 
+// Words [w0, w0 + NW) of this lane's portion of a code region laid out in
+// chunks of U = min(16, LB) bytes interleaved over the 32 lanes (see
+// lane_off); `base` is the region + lane * U.  w0 and NW are multiples of U/4,
+// so every load is one whole chunk: 32 lanes read one contiguous span.
+template <int LB, int NW>
+__device__ __forceinline__ void lane_words(const uint8_t* base, int w0, uint32_t (&dst)[NW]) {
+  constexpr int U = LB < 16 ? LB : 16;
+#pragma unroll
+  for (int x = 0; x < NW; x += U / 4) {
+    const uint8_t* ptr = base + ((w0 + x) * 4 / U) * 32 * U;
+    if constexpr (U == 16) {
+      const uint4 v = *reinterpret_cast<const uint4*>(ptr);
+      dst[x] = v.x; dst[x + 1] = v.y; dst[x + 2] = v.z; dst[x + 3] = v.w;
+    } else {
+      const uint2 v = *reinterpret_cast<const uint2*>(ptr);
+      dst[x] = v.x; dst[x + 1] = v.y;
+    }
+  }
+}
+
 // One live page-head block (in shared memory) of a class with B-bit codes.
 //   QK: S^T[16 slots x 8 heads] = K(codes) x Q^T per group, with codes as
 //       fp16 (1024 + code); the 1024 offset folds into the group's zero term:
@@ -411,29 +431,27 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   // ---------------- logits ----------------
   float lg[4] = {0.f, 0.f, 0.f, 0.f};
   {
-    const uint8_t* kl = blk + lane * LANE_BYTES;
+    constexpr int U = LANE_BYTES < 16 ? LANE_BYTES : 16;
+    const uint8_t* kbase = blk + lane * U;
     constexpr int PB = G * B / 32;                        // piece bytes (>= 2)
     constexpr int NW = PB >= 4 ? PB / 4 : 1;              // words per piece
+    // a lane portion of up to 32 bytes is loaded whole, a larger one per group
+    constexpr bool KALL = LANE_BYTES <= 32;
+    constexpr int KW = KALL ? LANE_BYTES / 4 : 2 * PB / 4;
+    uint32_t kw[KW];
+    if constexpr (KALL) lane_words<LANE_BYTES, KW>(kbase, 0, kw);
 #pragma unroll
     for (int gr = 0; gr < NG; ++gr) {
+      if constexpr (!KALL) lane_words<LANE_BYTES, KW>(kbase, gr * 2 * PB / 4, kw);
       uint32_t w[2][NW];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const uint8_t* src = kl + (gr * 2 + r) * PB;
         if constexpr (PB == 2) {
-          const uint32_t h16 = *reinterpret_cast<const uint16_t*>(src);
+          const uint32_t h16 = (kw[gr] >> (16 * r)) & 0xFFFFu;   // piece 2 gr + r
           w[r][0] = (h16 & 0xFFu) | ((h16 & 0xFF00u) << 8);  // bytes -> half-words
-        } else if constexpr (PB == 4) {
-          w[r][0] = *reinterpret_cast<const uint32_t*>(src);
-        } else if constexpr (PB == 8) {
-          const uint2 v = *reinterpret_cast<const uint2*>(src);
-          w[r][0] = v.x; w[r][1] = v.y;
         } else {
 #pragma unroll
-          for (int x = 0; x < PB / 16; ++x) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * x);
-            w[r][4 * x] = v.x; w[r][4 * x + 1] = v.y; w[r][4 * x + 2] = v.z; w[r][4 * x + 3] = v.w;
-          }
+          for (int x = 0; x < NW; ++x) w[r][x] = kw[(KALL ? gr * 2 * NW : 0) + r * NW + x];
         }
       }
       float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -622,7 +640,12 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   {
     constexpr int Q = (B == 16) ? D / 8 : D * B / 128;   // words per token pair
     constexpr int PER = (B == 16) ? 1 : 16 / B;          // codes per half-word
-    const uint32_t* vl = reinterpret_cast<const uint32_t*>(blk + 2 * D * B + lane * LANE_BYTES);
+    constexpr int U = LANE_BYTES < 16 ? LANE_BYTES : 16;
+    const uint8_t* vbase = blk + 2 * D * B + lane * U;
+    // a lane portion of up to 32 bytes is loaded whole, a larger one per half
+    constexpr bool VALL = LANE_BYTES <= 32;
+    uint32_t vall[VALL ? LANE_BYTES / 4 : 1];
+    if constexpr (VALL) lane_words<LANE_BYTES, (VALL ? LANE_BYTES / 4 : 1)>(vbase, 0, vall);
     // m-tiles in two halves (words q of P = 0 and P = 1 for half of the chunk
     // range); a single word per token pair (d = 64 at 2 bits) is one half
     constexpr int NHF = Q >= 2 ? 2 : 1;                    // halves
@@ -633,20 +656,11 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
       uint32_t vr[2][QH];
 #pragma unroll
       for (int P = 0; P < 2; ++P) {
-        if constexpr (QH % 4 == 0) {
+        if constexpr (VALL) {
 #pragma unroll
-          for (int x = 0; x < QH / 4; ++x) {
-            const uint4 v = reinterpret_cast<const uint4*>(vl + P * Q + hf * QH)[x];
-            vr[P][4 * x] = v.x; vr[P][4 * x + 1] = v.y; vr[P][4 * x + 2] = v.z; vr[P][4 * x + 3] = v.w;
-          }
-        } else if constexpr (QH % 2 == 0) {
-#pragma unroll
-          for (int x = 0; x < QH / 2; ++x) {
-            const uint2 v = reinterpret_cast<const uint2*>(vl + P * Q + hf * QH)[x];
-            vr[P][2 * x] = v.x; vr[P][2 * x + 1] = v.y;
-          }
+          for (int x = 0; x < QH; ++x) vr[P][x] = vall[P * Q + hf * QH + x];
         } else {
-          vr[P][0] = vl[P * Q + hf * QH];
+          lane_words<LANE_BYTES, QH>(vbase, P * Q + hf * QH, vr[P]);
         }
       }
 #pragma unroll

@@ -11,7 +11,10 @@ the oracle's natural [slot][channel] codes:
     channel 16*(e//2) + gid + 8*(e%2), e = q*16/b + k;
   params are [group][slot][scale, zero] fp16;
   inside a 32-bit word (or a 16-bit piece) even channels fill the low half and
-  odd channels the high half, little-endian.
+  odd channels the high half, little-endian;
+  the lanes' portions (d*b/16 bytes each) are interleaved in chunks of
+  u = min(16, d*b/16) bytes: byte o of lane l sits at (o // u)*32*u + l*u + o % u
+  of the K (or V) code region.
 """
 from functools import lru_cache
 
@@ -24,6 +27,11 @@ PAGE = 16
 def _maps(d: int, G: int, b: int):
     """(byte offset, bit shift) of every (slot, channel) code, for K and for V."""
     lane_bytes = d * b // 16
+    u = min(16, lane_bytes)
+
+    def lpos(lane, o):                      # byte o of the lane's portion
+        return (o // u) * 32 * u + lane * u + o % u
+
     kb = np.zeros((PAGE, d), dtype=np.int64)
     ks = np.zeros((PAGE, d), dtype=np.int64)
     vb = np.zeros((PAGE, d), dtype=np.int64)
@@ -32,16 +40,15 @@ def _maps(d: int, G: int, b: int):
     pb = G * b // 32                      # piece bytes
     for lane in range(32):
         gid, tid = lane // 4, lane % 4
-        base = lane * lane_bytes
         # K pieces
         for gr in range(ng):
             for r in range(2):
                 slot = gid + 8 * r
-                off = base + (gr * 2 + r) * pb
+                off = (gr * 2 + r) * pb
                 for e in range(G // 4):
                     ch = gr * G + tid * (G // 4) + e
                     if b == 16:
-                        kb[slot, ch] = off + 2 * e
+                        kb[slot, ch] = lpos(lane, off + 2 * e)
                         ks[slot, ch] = 0
                         continue
                     piece_bits = pb * 8
@@ -50,21 +57,21 @@ def _maps(d: int, G: int, b: int):
                     wi, el = divmod(e, m)
                     p = el // 2 if el % 2 == 0 else m // 2 + el // 2
                     bit = wi * word_bits + p * b
-                    kb[slot, ch] = off + bit // 8
+                    kb[slot, ch] = lpos(lane, off + bit // 8)
                     ks[slot, ch] = bit % 8
         # V words
         Q = d * b // 128 if b < 16 else d // 8
         per = 16 // b if b < 16 else 1
         for P in range(2):
             for q in range(Q):
-                woff = base + (P * Q + q) * 4
+                woff = (P * Q + q) * 4
                 for half in range(2):
                     slot = 2 * tid + 8 * P + half
                     for k in range(per):
                         e = q * per + k
                         ch = 16 * (e // 2) + gid + 8 * (e % 2)
                         bit = half * 16 + k * (b if b < 16 else 16)
-                        vb[slot, ch] = 2 * d * b + woff + bit // 8 if b < 16 else 32 * d + woff + bit // 8
+                        vb[slot, ch] = (2 * d * b if b < 16 else 32 * d) + lpos(lane, woff + bit // 8)
                         vs[slot, ch] = bit % 8
     return kb, ks, vb, vs
 
