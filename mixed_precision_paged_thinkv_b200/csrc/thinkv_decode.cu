@@ -141,12 +141,75 @@ __device__ inline void bitonic64_desc(float (&v)[2]) {
   }
 }
 
+// Sorts one value per lane into descending order across the warp.
+__device__ inline float bitonic32_desc(float v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const float o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+      const bool desc = (lane & size) == 0, lower = (lane & stride) == 0;
+      v = (lower == desc) ? fmaxf(v, o) : fminf(v, o);
+    }
+  }
+  return v;
+}
+
 struct TopkCtx {
   float* cand;    // [Gq][kCandCap]
   int* cnt;       // [Gq]
   float* theta;   // [Gq]  values <= theta cannot enter the top-k any more
   int topk;
 };
+
+// Cuts head h's candidates back to a few more than topk, without sorting
+// them.  Needs topk <= 32 and at least 32 candidates, so that every lane holds
+// one (candidate e sits at lane e % 32).  The lane maxima are sorted; the
+// threshold is the largest of them with at least topk candidates at or above
+// it (the topk-th largest lane maximum always qualifies).  Candidates below it
+// are dropped: at least topk larger ones remain, so none of them can be among
+// the topk largest.
+__device__ inline void cand_prune(const TopkCtx& tk, int h) {
+  const int lane = threadIdx.x & 31;
+  float* c = tk.cand + h * kCandCap;
+  const int n = tk.cnt[h];
+  float v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = (j * 32 + lane < n) ? c[j * 32 + lane] : -INFINITY;
+  const float s = bitonic32_desc(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+  int lo = 0, hi = tk.topk - 1;                    // the answer lies in [lo, hi]
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const float t = __shfl_sync(0xFFFFFFFFu, s, mid);
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) cnt += __popc(__ballot_sync(0xFFFFFFFFu, v[j] >= t));
+    if (cnt >= tk.topk) hi = mid; else lo = mid + 1;
+  }
+  const float theta = __shfl_sync(0xFFFFFFFFu, s, lo);
+  int kc = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) kc += v[j] >= theta;
+  int incl = kc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int kept = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  int at = incl - kc;
+  __syncwarp();                                    // every read of c is done
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (v[j] >= theta) c[at++] = v[j];
+  __syncwarp();
+  if (lane == 0) {
+    tk.cnt[h] = kept;
+    tk.theta[h] = theta;
+  }
+  __syncwarp();
+}
 
 // Keeps the topk largest candidates of head h and raises its threshold.
 __device__ inline void cand_compact(const TopkCtx& tk, int h) {
@@ -370,6 +433,7 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
     for (int hd = 0; hd < Gq; ++hd) {
       float sum = 0.f;
       if (!all) {
+        if (tk.topk <= 32 && tk.cnt[hd] > 64) cand_prune(tk, hd);   // then the 64-wide sort
         if (tk.cnt[hd] > 0) cand_compact(tk, hd);      // sorted, the k largest kept
         const int n = tk.cnt[hd];
         if (whole) {
@@ -504,10 +568,13 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
       }
     }
     __syncwarp();
-    // a head whose buffer could overflow on the next page is cut back to its top-k
+    // a head whose buffer could overflow on the next page is cut back
     unsigned full = __ballot_sync(0xFFFFFFFFu, lane < Gq && tk.cnt[lane] > kCandCap - 16);
     while (full) {
-      cand_compact(tk, __ffs(full) - 1);
+      const int hf = __ffs(full) - 1;
+      if (tk.topk <= 32) cand_prune(tk, hf);
+      // ties can keep too many: then the exact cut, which keeps topk
+      if (tk.cnt[hf] > kCandCap - 16) cand_compact(tk, hf);
       full &= full - 1;
     }
   }
@@ -908,14 +975,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kCombineThreads = 256;
 constexpr int kCombinePieces = 128;             // pieces per round of the weight table
-constexpr int kCombinePre = 16;                 // pieces whose quads are requested up front
+constexpr int kCombinePre = 8;                  // pieces whose quads are requested up front
 
 // Merges the segment's piece records with the log-sum-exp rule: thread t <
 // Gq * D/4 owns one quad of one head's output row; warp r < Gq then merges
 // head r's top-k lists (bitonic merges, the next piece's list loaded while the
 // current one merges) for the top-k mass.
 template <int D>
-__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(DecodeParams p) {
   constexpr int QD = D / 4;
   __shared__ float sM[8], sL[8];
   __shared__ int sMk[8];

@@ -143,3 +143,46 @@ def test_topk_mass_values_of_k(k):
     g.setup()
     o.setup()
     _check_all(g, o, topk=k, codes=False)
+
+
+@pytest.mark.parametrize("k", [8, 32, 40])
+def test_topk_mass_long_pieces_and_tied_logits(k):
+    """Enough live pages that every split warp handles about 20 pages of one
+    (sequence, kv-head), so its candidate lists fill and are cut back several
+    times.  Sequences 0-3 have one key for all tokens: every logit of a head
+    ties, no candidate can be dropped by a threshold, and the exact cut must
+    keep k of them (mass k / live tokens).  Sequences 4-7 have random keys."""
+    from oracle import oracle as O
+    from mixed_precision_paged_thinkv_b200.binding import ThinKVCache
+    Hq, Hkv, d, G, ns, L = 64, 8, 64, 32, 8, 6144
+    g = ThinKVCache(Hq, Hkv, d, G, (8, 4, 2), ns, 512, (ns * L // 16, 16, 16))
+    o = O.Oracle(Hq, Hkv, d, G, (8, 4, 2), ns, 512, (ns * L // 16, 16, 16))
+    dev = torch.device("cuda")
+    gen = torch.Generator().manual_seed(11)
+    key = torch.randn(Hkv, d, generator=gen)
+    chunk = 512
+    for c0 in range(0, L, chunk):
+        seq = np.repeat(np.arange(ns), chunk).astype(np.int32)
+        pos = np.tile(np.arange(c0, c0 + chunk), ns).astype(np.int32)
+        tag = np.zeros(seq.size, np.uint8)
+        kk = torch.randn(seq.size, Hkv, d, generator=gen)
+        kk[: 4 * chunk] = key                       # sequences 0-3: one key
+        kk = kk.half()
+        vv = torch.randn(seq.size, Hkv, d, generator=gen).half()
+        g.append(torch.as_tensor(seq, device=dev), torch.as_tensor(pos, device=dev),
+                 torch.as_tensor(tag, device=dev), kk.to(dev), vv.to(dev))
+        assert o.append(seq, pos, tag, kk, vv) == O.OK
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    q = torch.randn(ns, Hq, d, generator=gen).half()
+    out, mass = g.decode(torch.arange(ns, dtype=torch.int32, device=dev), q.to(dev), topk=k)
+    ref, rmass = o.decode(np.arange(ns, dtype=np.int32), q, topk=k, threads=8)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    err = Hn.attn_error(out.cpu().numpy(), ref)
+    m = mass.cpu().numpy().astype(np.float64)
+    merr = float(np.abs(m - rmass).max())
+    print(f"long pieces k={k}: attention error {err:.3e}, top-k mass error {merr:.3e}")
+    assert err <= Hn.TOL, err
+    assert merr <= Hn.MASS_TOL, merr
+    assert np.allclose(m[:4], k / L, rtol=1e-3, atol=0), m[:4].min()
