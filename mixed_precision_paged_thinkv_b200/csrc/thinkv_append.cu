@@ -343,21 +343,20 @@ __device__ inline RowVals<D> load_row(const uint16_t* __restrict__ x) {
 }
 
 // Quantises one K or V row of one kv-head (values held by the warp, D/32
-// channels per lane) at the bit width of class c and writes its codes and
-// params into slot pool_slot & 15 of page pool_slot >> 4's page-head block.
-template <int D, int G>
-__device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int h, int kv,
-                             const RowVals<D>& vals, uint16_t* code_sm) {
+// channels per lane) at bit width B (class c) and writes its codes and params
+// into slot pool_slot & 15 of page pool_slot >> 4's page-head block.
+template <int D, int G, int B>
+__device__ void scatter_unit_b(const CacheView& C, int c, uint32_t pool_slot, int h, int kv,
+                               const RowVals<D>& vals, uint16_t* code_sm) {
   constexpr int PER = D / 32;          // channels per lane
   constexpr int LPG = G / PER;         // lanes per group
   constexpr int NG = D / G;
   const int lane = threadIdx.x & 31;
-  const int b = C.L.bits[c];
   const uint32_t page = pool_slot >> 4, slot = pool_slot & 15;
-  const int64_t phb = page_head_bytes(D, G, b);
+  const int64_t phb = page_head_bytes(D, G, B);
   uint8_t* blk = C.pool[c] + ((int64_t)page * C.L.num_kv_heads + h) * phb;
   const uint16_t* raw = vals.raw;
-  if (b == 16) {
+  if constexpr (B == 16) {
 #pragma unroll
     for (int e = 0; e < PER; ++e) code_sm[lane * PER + e] = raw[e];
   } else {
@@ -375,7 +374,7 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
     }
     const __half zh = __float2half_rd(mn);
     const float zf = __half2float(zh);
-    const float levels = (float)((1 << b) - 1);
+    constexpr float levels = (float)((1 << B) - 1);
     const float s32 = __fdiv_rn(__fsub_rn(mx, zf), levels);
     const __half sh = __float2half_ru(s32);
     const float sf = __half2float(sh);
@@ -392,63 +391,81 @@ __device__ void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int 
     }
     const int grp = (lane * PER) / G;
     if ((lane % LPG) == 0) {
-      uint16_t* prm = reinterpret_cast<uint16_t*>(blk + 4LL * D * b + (kv ? 64LL * NG : 0));
+      uint16_t* prm = reinterpret_cast<uint16_t*>(blk + 4LL * D * B + (kv ? 64LL * NG : 0));
       uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
       *reinterpret_cast<uint32_t*>(prm + (grp * 16 + slot) * 2) = pair;
     }
   }
   __syncwarp();
 
-  const int lane_bytes = D * b / 16;
-  uint8_t* region = blk + (kv ? 2LL * D * b : 0);
+  constexpr int lane_bytes = D * B / 16;
+  uint8_t* region = blk + (kv ? 2LL * D * B : 0);
   if (kv == 0) {
     // K: pieces (layout lane 4*(slot%8)+t, group gr, r = slot/8) of G/4 channels
-    const int pb = G * b / 32;                 // piece bytes (>= 2)
-    const int m = min(32 / b, G / 4);          // channels per word (or per 16-bit piece)
-    if (b == 16 && lane < 4 * NG) {
-      // raw fp16: the piece is G/4 channels in natural order
+    constexpr int pb = G * B / 32;                 // piece bytes (>= 2)
+    if (lane < 4 * NG) {
       const int t = lane & 3, gr = lane >> 2;
       const int l = 4 * (slot & 7) + t, r = slot >> 3;
-      const int o = (gr * 2 + r) * pb;
       const uint16_t* src = code_sm + gr * G + t * (G / 4);
-      for (int e = 0; e < G / 4; e += 2)
-        *reinterpret_cast<uint32_t*>(region + lane_off(l, o + 2 * e, lane_bytes)) =
-            (uint32_t)src[e] | ((uint32_t)src[e + 1] << 16);
-    } else if (lane < 4 * NG) {
-      const int t = lane & 3, gr = lane >> 2;
-      const int l = 4 * (slot & 7) + t, r = slot >> 3;
-      uint32_t words[4] = {0, 0, 0, 0};
-      for (int e = 0; e < G / 4; ++e) {
-        const uint32_t v = code_sm[gr * G + t * (G / 4) + e];
-        const int wi = e / m, el = e % m;
-        const int p = (el & 1) ? (m / 2 + el / 2) : (el / 2);
-        words[wi] |= v << (p * b);
+      if constexpr (B == 16) {
+        // raw fp16: the piece is G/4 channels in natural order
+        const int o = (gr * 2 + r) * pb;
+#pragma unroll
+        for (int e = 0; e < G / 4; e += 2)
+          *reinterpret_cast<uint32_t*>(region + lane_off(l, o + 2 * e, lane_bytes)) =
+              (uint32_t)src[e] | ((uint32_t)src[e + 1] << 16);
+      } else {
+        constexpr int m = (32 / B) < (G / 4) ? (32 / B) : (G / 4);   // channels per word
+        uint32_t words[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int e = 0; e < G / 4; ++e) {
+          const uint32_t v = src[e];
+          const int wi = e / m, el = e % m;
+          const int p = (el & 1) ? (m / 2 + el / 2) : (el / 2);
+          words[wi] |= v << (p * B);
+        }
+        uint8_t* dst = region + lane_off(l, (gr * 2 + r) * pb, lane_bytes);   // pb <= chunk
+        if constexpr (pb == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)words[0];
+        else if constexpr (pb == 4) *reinterpret_cast<uint32_t*>(dst) = words[0];
+        else if constexpr (pb == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
       }
-      uint8_t* dst = region + lane_off(l, (gr * 2 + r) * pb, lane_bytes);   // pb <= chunk
-      if (pb == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)words[0];
-      else if (pb == 4) *reinterpret_cast<uint32_t*>(dst) = words[0];
-      else if (pb == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
     }
   } else {
-    // V: half-words (lane 4*g + t, P, q, half) holding 16/b codes each
+    // V: half-words (lane 4*g + t, P, q, half) holding 16/B codes each
     const int t = (slot & 7) >> 1, P = slot >> 3, half = slot & 1;
-    const int Q = D * b / 128;                 // chunks per P
-    const int per = 16 / b;                    // codes per half-word
-    for (int u = lane; u < 8 * Q; u += 32) {
-      const int g = u / Q, q = u % Q;
-      uint32_t hw = 0;
-      for (int k = 0; k < per; ++k) {
-        const int e = q * per + k;
-        const int ch = 16 * (e >> 1) + g + 8 * (e & 1);
-        hw |= (uint32_t)code_sm[ch] << (b * k);
+    constexpr int Q = D * B / 128;                 // chunks per P
+    constexpr int per = 16 / B;                    // codes per half-word
+#pragma unroll
+    for (int u0 = 0; u0 < 8 * Q; u0 += 32) {
+      const int u = u0 + lane;
+      if (u < 8 * Q) {
+        const int g = u / Q, q = u % Q;
+        uint32_t hw = 0;
+#pragma unroll
+        for (int k = 0; k < per; ++k) {
+          const int e = q * per + k;
+          const int ch = 16 * (e >> 1) + g + 8 * (e & 1);
+          hw |= (uint32_t)code_sm[ch] << (B * k);
+        }
+        const int l = 4 * g + t;
+        uint8_t* dst = region + lane_off(l, (P * Q + q) * 4 + 2 * half, lane_bytes);
+        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)hw;
       }
-      const int l = 4 * g + t;
-      uint8_t* dst = region + lane_off(l, (P * Q + q) * 4 + 2 * half, lane_bytes);
-      *reinterpret_cast<uint16_t*>(dst) = (uint16_t)hw;
     }
   }
   __syncwarp();
+}
+
+template <int D, int G>
+__device__ inline void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int h, int kv,
+                                    const RowVals<D>& vals, uint16_t* code_sm) {
+  switch (C.L.bits[c]) {
+    case 8: scatter_unit_b<D, G, 8>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 4: scatter_unit_b<D, G, 4>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 2: scatter_unit_b<D, G, 2>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    default: scatter_unit_b<D, G, 16>(C, c, pool_slot, h, kv, vals, code_sm); break;
+  }
 }
 
 template <int D, int G>
@@ -554,12 +571,18 @@ __global__ void __launch_bounds__(kSmallThreads)
   // ---- the call's own inputs (before the previous kernel has finished) ----
   // speculative prefetch: with one token per run (a decode step), run b is
   // token b; its first K/V rows are loaded while the call is validated
-  RowVals<D> pre;
+  RowVals<D> pre, pre2;
   const bool pre_ok = b < n && warp < 2 * H;
+  const bool pre2_ok = b < n && warp + kSmallWarps < 2 * H;
   if (pre_ok) {
     const int h = warp >> 1, kv = warp & 1;
     pre = load_row<D>((kv ? v : k) + ((int64_t)b * H + h) * D);
   }
+  if (pre2_ok) {                                  // the warp's second unit of token b
+    const int u2 = warp + kSmallWarps, h = u2 >> 1, kv = u2 & 1;
+    pre2 = load_row<D>((kv ? v : k) + ((int64_t)b * H + h) * D);
+  }
+  const int pre_tag = b < n ? tag[b] : 0;
   const int x0 = tid * kSmallPer;
   int s_[kSmallPer], c_[kSmallPer], p_[kSmallPer], sp_[kSmallPer], pp_[kSmallPer];
 #pragma unroll
@@ -703,10 +726,12 @@ __global__ void __launch_bounds__(kSmallThreads)
       const int64_t th = u >> 1;
       const int h = (int)(th % H);
       const int i = start + (int)(th / H);
-      const RowVals<D> vals = (u == warp && pre_ok && start == b)
-                                  ? pre
-                                  : load_row<D>((kv ? v : k) + ((int64_t)i * H + h) * D);
-      scatter_unit<D, G>(C, tag[i], (uint32_t)tok_slot[i - start], h, kv, vals, sm[warp].code);
+      const bool own = start == b;                  // token b opens run b: prefetched
+      const RowVals<D> vals = (u == warp && pre_ok && own)                 ? pre
+                              : (u == warp + kSmallWarps && pre2_ok && own) ? pre2
+                              : load_row<D>((kv ? v : k) + ((int64_t)i * H + h) * D);
+      scatter_unit<D, G>(C, (own && i == b) ? pre_tag : tag[i], (uint32_t)tok_slot[i - start], h,
+                         kv, vals, sm[warp].code);
     }
   }
 
