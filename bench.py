@@ -312,6 +312,8 @@ def workload_config(w, live):
            "parallelism": "replicas"}
     if live is not None:
         cfg["live_tokens_by_class"] = live
+    if w.budget == ("frac", 1.0):
+        cfg["state"] = "supplementary: before eviction (whole history live, mixed R/E/T)"
     return cfg
 
 
@@ -427,6 +429,7 @@ def thinkv_arm(args, w, world, rank, local):
             "config": workload_config(w, live),
             "decode_ms": sum(dec_ms) / len(dec_ms),
             "decode_hbm_gbs": achieved,
+            "decode_kv_tokens_per_s": float(sum(live)) / dec_avg_s,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
@@ -452,7 +455,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     from mixed_precision_paged_thinkv_b200 import workloads as W
-    w = W.WORKLOADS[args.workload]
+    w = W.get(args.workload)
     world, rank, local = dist_init()
     try:
         if args.impl == "reference":

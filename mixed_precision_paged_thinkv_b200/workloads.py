@@ -109,6 +109,29 @@ WORKLOADS = {
 WORKLOAD_ORDER = ["tiny", "r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b", "churn"]
 
 
+def before_eviction(w: Workload) -> Workload:
+    """The same layer shape and history, timed before any eviction: every
+    generated token stays live, with the segment tag mix (R/E/T about
+    0.3/0.5/0.2), so the 4-bit and 2-bit pages are read at full scale.  The
+    retained state of the budgeted workloads is almost all R (8-bit)."""
+    return dataclasses.replace(w, name=w.name + "-mixed", budget=("frac", 1.0), churn_steps=0,
+                               check_every=0)
+
+
+# Supplementary measurements (not the headline configurations).
+SUPPLEMENTARY = {n + "-mixed": before_eviction(WORKLOADS[n])
+                 for n in ("r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b", "churn")}
+
+
+def get(name: str) -> Workload:
+    """A workload by name: the five configurations, or a supplementary one."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    if name in SUPPLEMENTARY:
+        return SUPPLEMENTARY[name]
+    raise KeyError(f"unknown workload {name!r}")
+
+
 def scaled(w: Workload, **kw) -> Workload:
     """A copy of ``w`` with some fields replaced (used for reduced test cases)."""
     return dataclasses.replace(w, **kw)

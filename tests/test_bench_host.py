@@ -72,3 +72,27 @@ def test_launches_per_step_counts_the_one_launch_append_path():
     assert bench.launches_per_step(16) == 4
     assert bench.launches_per_step(512) == 4
     assert bench.launches_per_step(513) == 5
+
+
+def test_before_eviction_workloads_keep_the_shape_and_history():
+    """The supplementary '-mixed' workloads are the same layer and history with
+    nothing evicted: same lengths and tags, budget = every generated token."""
+    import numpy as np
+    from mixed_precision_paged_thinkv_b200 import workloads as W
+    for name, base in W.WORKLOADS.items():
+        if name == "tiny":
+            continue
+        m = W.get(name + "-mixed")
+        assert m.budget == ("frac", 1.0) and m.churn_steps == 0
+        for f in ("batch", "num_q_heads", "num_kv_heads", "head_dim", "group_size", "bits",
+                  "lengths", "segments", "tag_probs", "topk", "seed"):
+            assert getattr(m, f) == getattr(base, f), (name, f)
+        sb, sm = W.Schedule(base, 0), W.Schedule(m, 0)
+        assert np.array_equal(sb.lengths, sm.lengths)
+        n = int(sb.lengths[0])                      # the history (churn steps extend the base)
+        assert np.array_equal(sb.tags(0)[:n], sm.tags(0)[:n])
+        cfg = bench.workload_config(m, None)
+        assert "before eviction" in cfg["state"]
+        assert "state" not in bench.workload_config(base, None)
+    with pytest.raises(KeyError):
+        W.get("no-such-workload")

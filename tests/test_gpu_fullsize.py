@@ -48,10 +48,13 @@ def _check(g, osub, step, topk):
         assert merr <= Hn.MASS_TOL, merr
 
 
-@pytest.mark.parametrize("name", ["r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b"])
+# the '-mixed' cases keep the whole history live (R/E/T mix, 4- and 2-bit
+# pages at full scale); the budgeted ones retain almost only R tokens
+@pytest.mark.parametrize("name", ["r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b",
+                                  "r1-llama-8b-mixed", "gpt-oss-20b-mixed"])
 def test_full_size_workloads(name):
     from mixed_precision_paged_thinkv_b200.runner import WorkloadRun
-    w = W.WORKLOADS[name]
+    w = W.get(name)
     g = WorkloadRun(w, extra=2)
     g.setup()
     osub = Hn.OracleSubset(w, _sample(w, g.sched.lengths), extra=2)
