@@ -213,6 +213,14 @@ __device__ inline uint32_t unpack_pair<8>(uint32_t w, int k) {
   return __byte_perm(w, 0x64646464u, k == 0 ? 0x4240u : 0x4341u);
 }
 
+// fp16 pair (1024 + 2^(b-1), same): subtracted from an unpacked pair it gives
+// the centred codes (code - 2^(b-1)), exactly.
+template <int B>
+__device__ inline uint32_t centre_bits() {
+  constexpr uint32_t h = 0x6400u + (1u << (B - 1));
+  return h | (h << 16);
+}
+
 // fp16 pair (-(1024 + 2^(b-1)), same), exact in fp16: the constant A operand
 // that turns the products of (1024 + code) into products of the centred code.
 template <int B>

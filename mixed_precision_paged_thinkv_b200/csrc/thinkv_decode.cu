@@ -476,11 +476,18 @@ __device__ __forceinline__ void lane_words(const uint8_t* base, int w0, uint32_t
 }
 
 // One live page-head block (in shared memory) of a class with B-bit codes.
-//   QK: S^T[16 slots x 8 heads] = K(codes) x Q^T per group, with codes as
-//       fp16 (1024 + code); the 1024 offset folds into the group's zero term:
-//       q.k = s * sum q (1024 + c) + (z - 1024 s) * sum q.
+//   QK: S^T[16 slots x 8 heads] = K(codes) x Q^T per group.  8-bit codes enter
+//       as fp16 (1024 + code) and the offset folds into the group's zero term:
+//       q.k = s * sum q (1024 + c) + (z - 1024 s) * sum q.  4- and 2-bit codes
+//       have scales large enough that the cancellation of the 1024 s term
+//       would cost precision: they enter centred, (code - 2^(b-1)), exactly,
+//       and q.k = s * sum q (c - 2^(b-1)) + (z + 2^(b-1) s) * sum q.
 //   PV: O^T[16 channels x 8 heads] += V^T(codes - 2^(b-1)) x W per m-tile,
 //       W = p * s_V * 2^sigma rounded to fp16, plus sum p (z + 2^(b-1) s) in fp32.
+//       8-bit codes: the MMA takes (1024 + code) and a constant-row product
+//       removes the offset; 4- and 2-bit codes are centred in the operand (a
+//       centred code of 1 or 2 next to a 1024 offset would lose 9-10 bits of
+//       the running accumulator on every page).
 template <int D, int G, int B>
 __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
                                  float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
@@ -532,6 +539,7 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
             } else {
               constexpr int PAIRS = (PB == 2 ? 4 : 16 / B);  // pairs per (spread) word
               a[hi * 2 + r] = unpack_pair<B>(w[r][u / PAIRS], u % PAIRS);
+              if constexpr (B != 8) a[hi * 2 + r] = hsub2_bits(a[hi * 2 + r], centre_bits<B>());
             }
           }
         }
@@ -544,7 +552,8 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
         const uint32_t p0 = kpar[gr * 16 + g], p1 = kpar[gr * 16 + g + 8];
         const float2 sz0 = __half22float2(*reinterpret_cast<const __half2*>(&p0));  // (s, z)
         const float2 sz1 = __half22float2(*reinterpret_cast<const __half2*>(&p1));
-        const float zc0 = fmaf(-1024.f, sz0.x, sz0.y), zc1 = fmaf(-1024.f, sz1.x, sz1.y);
+        constexpr float off = B == 8 ? -1024.f : (float)(1 << (B - 1));   // see above
+        const float zc0 = fmaf(off, sz0.x, sz0.y), zc1 = fmaf(off, sz1.x, sz1.y);
         lg[0] = fmaf(sz0.x, c[0], fmaf(zc0, S.qsum[gr][0], lg[0]));
         lg[1] = fmaf(sz0.x, c[1], fmaf(zc0, S.qsum[gr][1], lg[1]));
         lg[2] = fmaf(sz1.x, c[2], fmaf(zc1, S.qsum[gr][0], lg[2]));
@@ -702,8 +711,8 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
     }
   }
 
-  // ---------------- O^T += V^T(codes - 2^(b-1)) x W, per m-tile: V^T(1024 + codes) x W
-  //                  plus one constant-row product that removes 1024 + 2^(b-1) ----------------
+  // ---------------- O^T += V^T(codes - 2^(b-1)) x W, per m-tile (8-bit: V^T(1024 + codes) x W
+  //                  plus one constant-row product that removes 1024 + 2^(b-1)) ----------------
   {
     constexpr int Q = (B == 16) ? D / 8 : D * B / 128;   // words per token pair
     constexpr int PER = (B == 16) ? 1 : 16 / B;          // codes per half-word
@@ -745,11 +754,12 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
               a[P * 2 + r] = vr[P][wq] & (P ? dm1 : dm0);   // raw values of dead slots: zero
             } else {
               a[P * 2 + r] = unpack_pair<B>(vr[P][wq], e % PER);   // 1024 + code
+              if constexpr (B != 8) a[P * 2 + r] = hsub2_bits(a[P * 2 + r], centre_bits<B>());
             }
           }
         }
         mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
-        if constexpr (B != 16) {
+        if constexpr (B == 8) {
           // centre at once: + (-(1024 + 2^(b-1))) * sum of W over the page's
           // tokens, so the segment's accumulators never carry the offset
           const uint32_t kc = neg_centre_bits<B>();
