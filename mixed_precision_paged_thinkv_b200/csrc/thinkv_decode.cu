@@ -321,6 +321,7 @@ struct SegState {
   float z[NG][2];                     // zero-term accumulators (heads 2t, 2t+1)
   float acc[MT][4];                   // PV accumulators (centred codes), units of 2^-sigma
   int sigma;                          // W = p * s_V * 2^sigma is the fp16 PV operand
+  float th[2];                        // top-k thresholds of heads 2t, 2t+1 (copies)
 };
 
 template <int D, int G>
@@ -352,6 +353,7 @@ __device__ inline void seg_begin(SegState<D, G>& S, const DecodeParams& p, const
   S.sigma = kSigmaInit;               // the first page sets sigma
   S.m[0] = S.m[1] = -INFINITY;
   S.lp[0] = S.lp[1] = 0.f;
+  S.th[0] = S.th[1] = -INFINITY;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) S.acc[mt][0] = S.acc[mt][1] = S.acc[mt][2] = S.acc[mt][3] = 0.f;
   if (tk.topk > 0) {
@@ -568,23 +570,32 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
 
   // ---------------- top-k candidates (logits above the head's threshold) ----------------
   if (tk.topk > 0) {
+    // the thresholds are register copies; they change only when a buffer is cut
+    bool ins = false;
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       const int hd = 2 * t + (x & 1);
-      if (hd < Gq && lg[x] > tk.theta[hd]) {
+      if (hd < Gq && lg[x] > S.th[x & 1]) {
         const int at = atomicAdd(&tk.cnt[hd], 1);
         tk.cand[hd * kCandCap + at] = lg[x];
+        ins = true;
       }
     }
-    __syncwarp();
-    // a head whose buffer could overflow on the next page is cut back
-    unsigned full = __ballot_sync(0xFFFFFFFFu, lane < Gq && tk.cnt[lane] > kCandCap - 16);
-    while (full) {
-      const int hf = __ffs(full) - 1;
-      if (tk.topk <= 32) cand_prune(tk, hf);
-      // ties can keep too many: then the exact cut, which keeps topk
-      if (tk.cnt[hf] > kCandCap - 16) cand_compact(tk, hf);
-      full &= full - 1;
+    if (__any_sync(0xFFFFFFFFu, ins)) {
+      __syncwarp();
+      // a head whose buffer could overflow on the next page is cut back
+      unsigned full = __ballot_sync(0xFFFFFFFFu, lane < Gq && tk.cnt[lane] > kCandCap - 16);
+      if (full) {
+        while (full) {
+          const int hf = __ffs(full) - 1;
+          if (tk.topk <= 32) cand_prune(tk, hf);
+          // ties can keep too many: then the exact cut, which keeps topk
+          if (tk.cnt[hf] > kCandCap - 16) cand_compact(tk, hf);
+          full &= full - 1;
+        }
+        S.th[0] = 2 * t < Gq ? tk.theta[2 * t] : INFINITY;
+        S.th[1] = 2 * t + 1 < Gq ? tk.theta[2 * t + 1] : INFINITY;
+      }
     }
   }
 
@@ -1010,6 +1021,8 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   const int np = (int)(by_unit ? nl : w1 - w0 + 1);
   if (np <= 1) return;                          // finished inside one split warp
   const int Gq = p.Gq, k = p.topk, kpad = (k + 3) / 4 * 4;
+  // the top-k warps' live count, requested now and used after the merge
+  const int live_i = (p.mass && threadIdx.x < 32 * Gq) ? p.live_count[p.seq[i]] : 0;
   const int64_t rb = record_bytes(Gq, D, k);
   const uint8_t* recs = reinterpret_cast<const uint8_t*>(p.rec);
   auto rec = [&](int j) -> const uint8_t* {
@@ -1107,7 +1120,7 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   if (warp >= Gq) return;
   const int r = warp;
   const int64_t mrow = (int64_t)i * p.Hq + h * Gq + r;
-  if (p.live_count[p.seq[i]] <= k) {
+  if (live_i <= k) {
     if (lane == 0) p.mass[mrow] = 1.f;
     return;
   }
