@@ -1194,13 +1194,14 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
   const int Gq0 = L.num_q_heads / L.num_kv_heads;
   const int q_bytes = Gq0 * D * 2;
   const int stage_bytes = (int)((maxphb + 127) / 128 * 128) + (q_bytes + 127) / 128 * 128;
-  // ~15 KB of page-head stages per warp keeps three 4-warp CTAs per SM
-  int nstage = (int)(15360 / stage_bytes);
+  // ~15 KB of page-head stages and top-k buffers per warp keeps three 4-warp
+  // CTAs per SM (at 8 warps per SM the top-k path ran 12-19 % slower)
+  const int Gq = L.num_q_heads / L.num_kv_heads;
+  const int topk_bytes = topk > 0 ? kTopkHdrBytes + Gq * kCandCap * 4 : 0;
+  int nstage = (int)((15360 - topk_bytes) / stage_bytes);
   if (nstage < 2) nstage = 2;
   if (nstage > kMaxStages) nstage = kMaxStages;
-  const int Gq = L.num_q_heads / L.num_kv_heads;
-  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes +
-                        (topk > 0 ? kTopkHdrBytes + Gq * kCandCap * 4 : 0);
+  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes + topk_bytes;
   const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)kDecWarps * warp_smem;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
