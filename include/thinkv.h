@@ -3,16 +3,18 @@
  *
  * What the library computes follows "ThinKV: Thought-Adaptive KV Cache
  * Compression for Efficient Reasoning Models":
- *   - arXiv abstract: a kernel that extends PagedAttention so that evicted
- *     tokens' memory slots are reused without compaction;
+ *   - arXiv abstract: decode attention over paged KV memory in the style of
+ *     PagedAttention, where slots freed by eviction go to later tokens and
+ *     nothing is compacted;
  *   - explainer, Resume Technique > Methodologie > "Quantification Adaptative
  *     a la Pensee (TBQ)": token precision set by thought type, R > E > T, by
  *     group quantisation;
  *   - explainer, Methodologie > "Eviction Adaptative a la Pensee (TBE)":
  *     tokens of less important thoughts are evicted;
  *   - explainer, Methodologie > "Implementation Systeme: Pensee Continue (CT)":
- *     a modified block table tracking thought type, start index and eviction
- *     mask; new tokens of the same thought type overwrite evicted slots.
+ *     a block table extended with each slot's thought type, start index and
+ *     eviction state; an evicted slot is refilled in place by a later token of
+ *     the same type.
  * Where the pages leave a choice open (integer code format, rounding of the
  * fp16 scale/zero, free-list discipline, eviction order, the attention-mass
  * statistic) this header states the choice made.

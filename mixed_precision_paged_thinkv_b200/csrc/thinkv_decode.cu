@@ -1,7 +1,7 @@
 // thinkv_decode.cu -- decode attention over mixed-precision, slot-reusing pages.
 //
 // "ThinKV: Thought-Adaptive KV Cache Compression for Efficient Reasoning
-// Models": the arXiv abstract's kernel "that extends PagedAttention" to read a
+// Models": the arXiv abstract's PagedAttention-based decode kernel, reading a
 // cache whose tokens carry per-thought-type precision (explainer, Methodologie,
 // TBQ) and whose evicted slots are holes that are never compacted (explainer,
 // "Implementation Systeme: Pensee Continue (CT)").  The pages print no kernel

@@ -13,10 +13,10 @@
  *   [TBE]  explainer, Methodologie > "Eviction Adaptative a la Pensee (TBE)":
  *          tokens of less important thoughts are evicted.
  *   [CT]   explainer, Methodologie > "Implementation Systeme: Pensee Continue
- *          (CT)" and the arXiv abstract: a PagedAttention extension whose
- *          block table records thought type, start index and eviction mask;
- *          new tokens of the same thought type overwrite evicted slots in
- *          place, so nothing is ever compacted.
+ *          (CT)" and the arXiv abstract: paged attention memory whose
+ *          block table also records each slot's thought type, start index
+ *          and eviction state; an evicted slot is refilled in place by a
+ *          later token of the same type, so nothing is ever compacted.
  * Readings where the pages are silent (code format, rounding of the fp16
  * scale/zero, free-list discipline, eviction order, ...) are listed with the
  * design notes; each is marked "reading" below where it is used.

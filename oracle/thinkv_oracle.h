@@ -7,14 +7,14 @@
  * tables) and is written to be checked by eye against the method it follows:
  *
  *   "ThinKV: Thought-Adaptive KV Cache Compression for Efficient Reasoning
- *   Models" -- arXiv abstract (kernel extending PagedAttention that reuses
- *   evicted tokens' memory slots without compaction) and the explainer's
+ *   Models" -- arXiv abstract (paged decode attention in the PagedAttention
+ *   style, slots freed by eviction reused, nothing compacted) and the explainer's
  *   "Resume Technique / Methodologie" sections: TBQ (precision assigned by
  *   thought type, R > E > T, group quantisation), TBE (eviction of tokens of
  *   less important thoughts) and "Implementation Systeme: Pensee Continue
- *   (CT)" (a modified block table tracking thought type, start index and
- *   eviction mask; new tokens of the same thought type overwrite evicted
- *   slots in place).
+ *   (CT)" (a block table extended with each slot's thought type, start
+ *   index and eviction state; an evicted slot is refilled in place by a later
+ *   token of the same type).
  *
  * Every place where the pages are silent is filled by one stated reading;
  * the list is kept with the design notes of this repository.
