@@ -323,8 +323,8 @@ def workload_config(w, live):
 def thinkv_arm(args, w, world, rank, local):
     import torch
     from mixed_precision_paged_thinkv_b200 import build as B
-    from mixed_precision_paged_thinkv_b200.runner import (WorkloadRun, make_steps, run_step,
-                                                          run_step_from_host)
+    from mixed_precision_paged_thinkv_b200.runner import (PackedStep, WorkloadRun, make_steps,
+                                                          run_step, run_step_from_host)
     B.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -387,8 +387,10 @@ def thinkv_arm(args, w, world, rank, local):
     value = tokens / max_s
 
     # end to end through host buffers (pinned), copies inside the timed region
-    host = [steps[Wm + K + k].to("cpu", pin=True) for k in range(e2e_steps)]
-    dbuf = steps[Wm + K]  # device staging tensors, overwritten by the copies
+    # each step's inputs packed in one pinned buffer: one copy per step
+    host = [PackedStep(steps[Wm + K + k], "cpu", pin=True).fill(steps[Wm + K + k])
+            for k in range(e2e_steps)]
+    dbuf = PackedStep(steps[Wm + K], dev)  # device staging, overwritten by the copies
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     mass_h = torch.empty(mass.shape, dtype=mass.dtype).pin_memory() if w.topk else None
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -115,6 +115,35 @@ class StepInputs:
         return StepInputs(**out)
 
 
+class PackedStep:
+    """A step's inputs as views into one contiguous byte buffer (host, pinned
+    host or device), so that moving a step between host and device is a
+    single copy.  Every field starts on a 256-byte boundary."""
+
+    ALIGN = 256
+
+    def __init__(self, like: StepInputs, device, pin: bool = False):
+        layout, off = [], 0
+        for f in StepInputs.FIELDS:
+            t = getattr(like, f)
+            n = t.numel() * t.element_size()
+            layout.append((f, off, n, t.dtype, tuple(t.shape)))
+            off += (n + self.ALIGN - 1) // self.ALIGN * self.ALIGN
+        buf = torch.empty(max(off, self.ALIGN), dtype=torch.uint8, device=device)
+        self.buf = buf.pin_memory() if pin else buf
+        self.inputs = StepInputs(**{f: self.buf[o:o + n].view(dt).view(shape)
+                                    for f, o, n, dt, shape in layout})
+
+    def fill(self, src: StepInputs) -> "PackedStep":
+        """Copies ``src`` in, field by field (synchronous; for setup only)."""
+        for f in StepInputs.FIELDS:
+            getattr(self.inputs, f).copy_(getattr(src, f))
+        return self
+
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+
 def make_steps(run: "WorkloadRun", nsteps: int, first_step: int = 0, device=None):
     """Inputs of the next ``nsteps`` steps of ``run`` (does not advance it)."""
     w = run.w
@@ -141,16 +170,15 @@ def run_step(cache: ThinKVCache, inp: StepInputs, out: torch.Tensor, topk: Optio
     return cache.decode(inp.seqs, inp.q, topk=topk, out=out, mass=mass)
 
 
-def run_step_from_host(cache: ThinKVCache, host: StepInputs, dev: StepInputs,
+def run_step_from_host(cache: ThinKVCache, host: PackedStep, dev: PackedStep,
                        out_dev: torch.Tensor, out_host: torch.Tensor, topk: Optional[int] = None,
                        mass_dev: Optional[torch.Tensor] = None,
                        mass_host: Optional[torch.Tensor] = None):
     """One step whose inputs start in pinned host memory and whose outputs end
-    there: host->device copies, the three library calls, device->host copies,
-    all queued on the current stream."""
-    for f in StepInputs.FIELDS:
-        getattr(dev, f).copy_(getattr(host, f), non_blocking=True)
-    run_step(cache, dev, out_dev, topk=topk, mass=mass_dev)
+    there: one host->device copy of the packed inputs, the three library
+    calls, device->host copies, all queued on the current stream."""
+    dev.buf.copy_(host.buf, non_blocking=True)
+    run_step(cache, dev.inputs, out_dev, topk=topk, mass=mass_dev)
     out_host.copy_(out_dev, non_blocking=True)
     if topk:
         mass_host.copy_(mass_dev, non_blocking=True)

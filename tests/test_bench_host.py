@@ -96,3 +96,29 @@ def test_before_eviction_workloads_keep_the_shape_and_history():
         assert "state" not in bench.workload_config(base, None)
     with pytest.raises(KeyError):
         W.get("no-such-workload")
+
+
+def test_packed_step_round_trips_every_field_through_one_buffer():
+    """The end-to-end leg moves a step's inputs with one copy of a packed
+    buffer: every field survives the copy, starts on a 256-byte boundary, and
+    the views are what the library calls receive."""
+    from mixed_precision_paged_thinkv_b200.runner import PackedStep, StepInputs
+    g = torch.Generator().manual_seed(3)
+    B, H, d, Hq = 5, 2, 64, 8
+    src = StepInputs(seqs=torch.arange(B, dtype=torch.int32),
+                     pos=torch.randint(0, 1000, (B,), dtype=torch.int32, generator=g),
+                     tags=torch.randint(0, 3, (B,), dtype=torch.uint8, generator=g),
+                     k=torch.randn(B, H, d, generator=g).half(),
+                     v=torch.randn(B, H, d, generator=g).half(),
+                     budgets=torch.randint(1, 50, (B,), dtype=torch.int32, generator=g),
+                     q=torch.randn(B, Hq, d, generator=g).half())
+    host = PackedStep(src, "cpu").fill(src)
+    dev = PackedStep(src, "cpu")
+    dev.buf.copy_(host.buf)
+    base = dev.buf.data_ptr()
+    for f in StepInputs.FIELDS:
+        a, b = getattr(src, f), getattr(dev.inputs, f)
+        assert b.dtype == a.dtype and b.shape == a.shape and b.is_contiguous(), f
+        assert torch.equal(a, b), f
+        assert (b.data_ptr() - base) % PackedStep.ALIGN == 0, f
+    assert host.nbytes() >= src.nbytes() and host.nbytes() % PackedStep.ALIGN == 0
