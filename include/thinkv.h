@@ -36,6 +36,16 @@
  *     decode still runs (it only reads state that every operation leaves
  *     consistent).  thinkv_get_status / thinkv_clear_status read and reset it.
  *   - Nothing traps or spins without a bound.
+ *   - Small appends, small evicts and decode launch their kernels with
+ *     programmatic stream serialisation: a kernel may start while the
+ *     previous kernel on the stream is finishing.  Before waiting for that
+ *     kernel it reads only the call's own input arrays (token ids,
+ *     positions, tags, K/V rows, budgets, sequence ids); cache state is read
+ *     after the wait.  The library's kernels never write a call's inputs.  A
+ *     caller whose own kernel writes a call's inputs, directly before the
+ *     call, must not release its dependents early
+ *     (griddepcontrol.launch_dependents); a copy or an ordinary kernel
+ *     completes before the call's kernels start.
  */
 #ifndef THINKV_H
 #define THINKV_H
