@@ -26,6 +26,7 @@ import math
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -347,8 +348,9 @@ def thinkv_arm(args, w, world, rank, local):
     alg_bytes, live, pages = algorithmic_decode_bytes(w, snap)
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    clocks = ClockSampler(os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/clocks{rank}.csv")
+    # the raw nvidia-smi samples go to THINKV_CLOCK_LOG_DIR (default: the temp dir)
+    clocks = ClockSampler(os.path.join(os.environ.get("THINKV_CLOCK_LOG_DIR", tempfile.gettempdir()),
+                                       f"thinkv_clocks_rank{rank}.csv"))
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
