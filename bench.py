@@ -121,8 +121,9 @@ def launches_per_step(batch: int) -> int:
 
 def algorithmic_decode_bytes(w, snap) -> int:
     """Bytes one decode call must move: codes + params of every live token for
-    every kv-head, the table entry and live-list entry of every live page, Q,
-    O and (if asked) the fp32 top-k mass."""
+    every kv-head, the table entry and live-list entry (8 B each) of every
+    live page, the sequence id and live-page count (4 B each) of every
+    sequence, Q, O and (if asked) the fp32 top-k mass."""
     H, d, G = w.num_kv_heads, w.head_dim, w.group_size
 
     def entry_class(e):  # block-table entry: page | class << 32 | live_mask << 48
@@ -145,7 +146,8 @@ def algorithmic_decode_bytes(w, snap) -> int:
         b = w.bits[c]
         per = 2 * d * b // 8 + (2 * (d // G) * 4 if b < 16 else 0)
         total += live_by_class[c] * H * per
-    total += pages * (8 + 4)
+    total += pages * (8 + 8)
+    total += w.batch * (4 + 4)
     total += 2 * w.batch * w.num_q_heads * d * 2
     if w.topk:
         total += w.batch * w.num_q_heads * 4

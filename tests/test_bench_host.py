@@ -122,3 +122,30 @@ def test_packed_step_round_trips_every_field_through_one_buffer():
         assert torch.equal(a, b), f
         assert (b.data_ptr() - base) % PackedStep.ALIGN == 0, f
     assert host.nbytes() >= src.nbytes() and host.nbytes() % PackedStep.ALIGN == 0
+
+
+def test_algorithmic_decode_bytes_counts_live_tokens_pages_and_rows():
+    """Byte accounting on a hand-made state: sequence 0 has one 8-bit page with
+    3 live slots and one 2-bit page with 16; sequence 1 has one 4-bit page with
+    1 live slot.  d = 128, G = 64, 2 kv-heads, 4 q-heads, top-k on."""
+    import numpy as np
+    from mixed_precision_paged_thinkv_b200 import workloads as W
+    w = W.scaled(W.WORKLOADS["tiny"], batch=2, num_q_heads=4, num_kv_heads=2, head_dim=128,
+                 group_size=64, topk=32)
+    def ent(page, cls, mask):
+        return np.uint64(page | (cls << 32) | (mask << 48))
+    table = np.zeros((2, 4), dtype=np.uint64)
+    table[0, 0] = ent(7, 0, 0b111)
+    table[0, 1] = ent(3, 2, 0xFFFF)
+    table[1, 2] = ent(5, 1, 0b1000)
+    live = np.zeros((2, 4), dtype=np.uint64)
+    live[0, 0] = np.uint64(7 | (0 << 32) | (0 << 40))
+    live[0, 1] = np.uint64(3 | (2 << 32) | (1 << 40))
+    live[1, 0] = np.uint64(5 | (1 << 32) | (2 << 40))
+    snap = {"num_live": np.array([2, 1], dtype=np.int32), "live_list": live, "table": table}
+    total, by_class, pages = bench.algorithmic_decode_bytes(w, snap)
+    assert by_class == [3, 1, 16] and pages == 3
+    per = {8: 2 * 128 + 2 * 2 * 4, 4: 128 + 16, 2: 64 + 16}      # 272 / 144 / 80 B
+    want = 2 * (3 * per[8] + 1 * per[4] + 16 * per[2])            # x kv-heads
+    want += 3 * 16 + 2 * 8 + 2 * 2 * 4 * 128 * 2 + 2 * 4 * 4     # pages, seqs, Q+O, mass
+    assert total == want
