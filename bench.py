@@ -282,7 +282,8 @@ def reference_arm(args, w, world, rank):
         "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": r["steps"], "warmup": args.warmup,
         "ms_per_step": 1000.0 * r["seconds"] / max(1, r["steps"]), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (attention), f32 (quantiser)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "dtype_detail": "attention in f64; the quantiser in the f32 operations it is defined with",
         "data": "synthetic", "config": workload_config(w, None),
         "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": r["cores"],
                          "kind": "oracle",
@@ -430,7 +431,8 @@ def thinkv_arm(args, w, world, rank, local):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": Wm, "ms_per_step": 1000.0 * max_s / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8/4/2 codes, f16 mma, f32 accumulate",
+            "dtype": "f16",
+            "dtype_detail": "8/4/2-bit integer codes dequantised into f16 mma operands, f32 accumulate",
             "data": "synthetic (seeded counter-hash normals, segment tags)",
             "config": workload_config(w, live),
             "decode_ms": sum(dec_ms) / len(dec_ms),
