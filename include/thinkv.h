@@ -25,6 +25,11 @@
  *     no global state, apart from the fixed scratch array of
  *     thinkv_decode_attention_noalloc.  fp16 values travel as uint16_t bit
  *     patterns.
+ *   - Alignment: pool[c], k, v, q, out and every workspace start on a 16-byte
+ *     boundary (they are moved by bulk copies and 16-byte vector accesses);
+ *     block_table and live_list on an 8-byte boundary; every other array on
+ *     the boundary of its element type.  A pointer that breaks this is
+ *     rejected with THINKV_ERR_INVALID before anything is launched.
  *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous
  *     on it.
  *   - Host-checkable errors (bad layout, null pointers, sizes) return a
@@ -281,7 +286,9 @@ THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs
  * that size returns THINKV_ERR_WORKSPACE before launching anything.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  Calls share the array: two calls that overlap on the GPU
+ * capture.  The looked-up address belongs to the device's context of that
+ * moment: after cudaDeviceReset() on a device, this entry point must not be
+ * called on that device again in the same process.  Calls share the array: two calls that overlap on the GPU
  * (different streams, or different host threads) race and must not be
  * issued.  Nothing is allocated or freed. */
 THINKV_API int thinkv_decode_attention_noalloc(const thinkv_cache* cache, int32_t n_seqs,

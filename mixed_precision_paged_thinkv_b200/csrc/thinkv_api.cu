@@ -43,11 +43,21 @@ namespace thinkv {
 
 bool cache_ok(const thinkv_cache* C) {
   if (!C || !layout_ok(&C->L)) return false;
-  for (int c = 0; c < 3; ++c)
+  for (int c = 0; c < 3; ++c) {
     if (C->L.pool_pages[c] > 0 && (!C->pool[c] || !C->slot_pos[c])) return false;
-  return C->block_table && C->num_blocks && C->free_slots && C->free_top && C->fifo &&
-         C->fifo_head && C->fifo_tail && C->live_count && C->live_list && C->live_index &&
-         C->num_live && C->page_bump && C->status;
+    // page-head blocks are moved by bulk copies and 16-byte vector stores
+    if (!aligned(C->pool[c], 16) || !aligned(C->slot_pos[c], 4)) return false;
+  }
+  if (!(C->block_table && C->num_blocks && C->free_slots && C->free_top && C->fifo &&
+        C->fifo_head && C->fifo_tail && C->live_count && C->live_list && C->live_index &&
+        C->num_live && C->page_bump && C->status))
+    return false;
+  // 64-bit words are updated with 64-bit atomics; the rest are int32 arrays
+  return aligned(C->block_table, 8) && aligned(C->live_list, 8) && aligned(C->num_blocks, 4) &&
+         aligned(C->free_slots, 4) && aligned(C->free_top, 4) && aligned(C->fifo, 4) &&
+         aligned(C->fifo_head, 4) && aligned(C->fifo_tail, 4) && aligned(C->live_count, 4) &&
+         aligned(C->live_index, 4) && aligned(C->num_live, 4) && aligned(C->page_bump, 4) &&
+         aligned(C->status, 4);
 }
 
 CacheView view_of(const thinkv_cache* C) {
@@ -90,13 +100,17 @@ int num_sms_current() {
   return cached[dev];
 }
 
+}  // namespace
+
+namespace thinkv {
+
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return THINKV_OK;
   if (getenv("THINKV_VERBOSE")) fprintf(stderr, "libthinkv: %s\n", cudaGetErrorString(e));
   return THINKV_ERR_CUDA;
 }
 
-}  // namespace
+}  // namespace thinkv
 
 extern "C" {
 
@@ -179,6 +193,9 @@ int thinkv_append_quantize(const thinkv_cache* C, int32_t n, const int32_t* seq,
   if (!cache_ok(C) || n < 0) return THINKV_ERR_INVALID;
   if (n == 0) return THINKV_OK;
   if (!seq || !pos || !tag || !k || !v) return THINKV_ERR_INVALID;
+  if (!aligned(seq, 4) || !aligned(pos, 4) || !aligned(k, 16) || !aligned(v, 16))
+    return THINKV_ERR_INVALID;
+  if (workspace && !aligned(workspace, 16)) return THINKV_ERR_INVALID;
   if (!workspace || workspace_bytes < append_workspace_bytes(n)) return THINKV_ERR_WORKSPACE;
   const int sms = num_sms_current();
   if (sms <= 0) return THINKV_ERR_CUDA;
@@ -200,6 +217,7 @@ int thinkv_evict(const thinkv_cache* C, int32_t n, const int32_t* seq, const int
   }
   if (n == 0) return THINKV_OK;
   if (!seq || !budget) return THINKV_ERR_INVALID;
+  if (!aligned(seq, 4) || !aligned(budget, 4)) return THINKV_ERR_INVALID;
   return cuda_status(launch_evict(view_of(C), n, seq, budget, o, static_cast<cudaStream_t>(stream)));
 }
 
@@ -219,6 +237,8 @@ int thinkv_decode_attention(const thinkv_cache* C, int32_t n, const int32_t* seq
   if (!cache_ok(C) || n < 1 || n > 16384) return THINKV_ERR_INVALID;
   if (!seq || !q || !out) return THINKV_ERR_INVALID;
   if (topk_mass && (topk < 1 || topk > 64)) return THINKV_ERR_INVALID;
+  if (!decode_args_aligned(seq, q, out, topk_mass)) return THINKV_ERR_INVALID;
+  if (workspace && !aligned(workspace, 16)) return THINKV_ERR_INVALID;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return THINKV_ERR_CUDA;
   DecodeLaunch dl;

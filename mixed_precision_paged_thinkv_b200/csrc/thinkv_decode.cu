@@ -28,6 +28,7 @@
 //   head for the top-k lists -- and writes fp16 O and the top-k mass.
 #include <cuda_fp16.h>
 #include <limits.h>
+#include <mutex>
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
@@ -1159,17 +1160,24 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
 
 template <int D, int G>
 cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
-  // raise the dynamic shared-memory limit of this instantiation once per device
+  // raise the dynamic shared-memory limit of this instantiation once per
+  // device (and again whenever a launch needs more); host threads that decode
+  // at the same time serialise on the lock, so the recorded size never runs
+  // ahead of the attribute actually set
+  static std::mutex lock;
   static size_t configured[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (dl.smem_bytes > configured[dev]) {
-    e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)dl.smem_bytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = dl.smem_bytes;
+  {
+    std::lock_guard<std::mutex> guard(lock);
+    if (dl.smem_bytes > configured[dev]) {
+      e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)dl.smem_bytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = dl.smem_bytes;
+    }
   }
   e = launch_pdl(decode_split_kernel<D, G>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
                  stream, p);

@@ -55,8 +55,16 @@ cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, cons
                          const uint8_t order[3], cudaStream_t stream);
 
 // host-side checks shared by the entry points
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool cache_ok(const thinkv_cache* C);
 CacheView view_of(const thinkv_cache* C);
+// q rows and out rows are moved with bulk copies / 8-byte vector stores;
+// seq and mass are plain 4-byte arrays
+inline bool decode_args_aligned(const void* seq, const void* q, const void* out, const void* mass) {
+  return aligned(seq, 4) && aligned(q, 16) && aligned(out, 16) && aligned(mass, 4);
+}
+// THINKV_OK, or THINKV_ERR_CUDA (printed to stderr when THINKV_VERBOSE is set)
+int cuda_status(cudaError_t e);
 
 // decode
 struct DecodeLaunch {

@@ -53,6 +53,7 @@ extern "C" int thinkv_decode_attention_noalloc(const thinkv_cache* C, int32_t n,
   if (!cache_ok(C) || n < 1 || n > 16384) return THINKV_ERR_INVALID;
   if (!seq || !q || !out) return THINKV_ERR_INVALID;
   if (topk_mass && (topk < 1 || topk > 64)) return THINKV_ERR_INVALID;
+  if (!decode_args_aligned(seq, q, out, topk_mass)) return THINKV_ERR_INVALID;
   const int k = topk_mass ? topk : 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return THINKV_ERR_CUDA;
@@ -60,10 +61,8 @@ extern "C" int thinkv_decode_attention_noalloc(const thinkv_cache* C, int32_t n,
   if (!plan_decode_launch(C->L, n, k, dev, &dl)) return THINKV_ERR_INVALID;
   if (decode_workspace_bytes(C->L, n, k, dl) > kScratchBytes) return THINKV_ERR_WORKSPACE;
   void* ws = nullptr;
-  if (scratch_address(&ws) != cudaSuccess) return THINKV_ERR_CUDA;
+  const cudaError_t e = scratch_address(&ws);
+  if (e != cudaSuccess) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launch_decode(view_of(C), n, seq, q, out, topk_mass, k, softmax_scale, ws, dl, s) ==
-                 cudaSuccess
-             ? THINKV_OK
-             : THINKV_ERR_CUDA;
+  return cuda_status(launch_decode(view_of(C), n, seq, q, out, topk_mass, k, softmax_scale, ws, dl, s));
 }

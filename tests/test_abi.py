@@ -116,3 +116,48 @@ def test_layout_decoder_is_a_bijection():
                 assert bits.min() == 0 and bits.max() == 16 * d * w - w
                 assert len(np.unique(bits)) == 16 * d
                 assert np.all(bits % w == 0)
+
+
+def test_misaligned_pointers_rejected_without_launch(lib):
+    """Pointers off the documented boundaries are refused before any CUDA call
+    (bulk copies and vector accesses would otherwise fault on the device)."""
+    from mixed_precision_paged_thinkv_b200 import binding
+    cs = binding.CacheStruct()
+    cs.L = _layout()
+    for name, _ in binding.CacheStruct._fields_[1:]:
+        v = getattr(cs, name)
+        if isinstance(v, C.Array):
+            for i in range(3):
+                v[i] = 4096
+        else:
+            setattr(cs, name, 4096)
+    ok = C.c_void_p(4096)
+    odd = C.c_void_p(4096 + 2)
+    word = C.c_void_p(4096 + 4)       # 4-byte aligned, not 16
+    # a misaligned k, v, q, out or workspace
+    assert lib.thinkv_append_quantize(C.byref(cs), 4, ok, ok, ok, word, ok, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_append_quantize(C.byref(cs), 4, ok, ok, ok, ok, word, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_append_quantize(C.byref(cs), 4, odd, ok, ok, ok, ok, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_append_quantize(C.byref(cs), 4, ok, ok, ok, ok, ok, word, 10 ** 6, None) == 1
+    assert lib.thinkv_evict(C.byref(cs), 1, odd, ok, None, None) == 1
+    assert lib.thinkv_evict(C.byref(cs), 1, ok, odd, None, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, ok, word, ok, None, 0, 0.0, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, ok, ok, word, None, 0, 0.0, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, odd, ok, ok, None, 0, 0.0, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, ok, ok, ok, odd, 8, 0.0, ok, 10 ** 6, None) == 1
+    assert lib.thinkv_decode_attention(C.byref(cs), 1, ok, ok, ok, None, 0, 0.0, word, 10 ** 6, None) == 1
+    f = lib.thinkv_decode_attention_noalloc
+    f.argtypes = [C.POINTER(binding.CacheStruct), C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
+                  C.c_void_p, C.c_int32, C.c_float, C.c_void_p]
+    f.restype = C.c_int
+    assert f(C.byref(cs), 1, ok, word, ok, None, 0, 0.0, None) == 1
+    # a misaligned cache buffer makes every operation refuse the cache
+    cs.pool[1] = 4096 + 8
+    assert lib.thinkv_cache_reset(C.byref(cs), None) == 1
+    assert lib.thinkv_evict(C.byref(cs), 1, ok, ok, None, None) == 1
+    cs.pool[1] = 4096
+    cs.block_table = 4096 + 4
+    assert lib.thinkv_cache_reset(C.byref(cs), None) == 1
+    cs.block_table = 4096
+    cs.num_live = 4096 + 2
+    assert lib.thinkv_cache_reset(C.byref(cs), None) == 1
