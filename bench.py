@@ -5,11 +5,14 @@
 One step = one token appended (quantised) per sequence, eviction back to the
 budget, and decode attention (+ the top-k mass when the workload asks for
 it) over every sequence -- the whole hot path over one batch.  The workload
-defaults to the R1-Distill-Llama-8B-shaped layer (16 sequences x 16384
-generated tokens, 32/8 heads, head_dim 128, 8/4/2-bit R/E/T codes, group 64,
-5% budget).  Inputs are synthetic and seeded; the per-step inputs are
-resident on the GPU before timing; L2 is flushed (512 MiB write) between
-steps, outside the timed events.
+defaults to the serving-churn layer, the largest single-GPU configuration
+(128 sequences with lengths log-uniform over 2k-64k, 1000 churn steps before
+timing, 32/8 heads, head_dim 128, 8/4/2-bit R/E/T codes, group 64, 5%
+budget).  In the same run the three other budgeted layer shapes
+(R1-Distill-Llama-8B, R1-Distill-Qwen-14B, GPT-OSS-20B) are set up and timed
+the same way; their lines go to `per_config`.  Inputs are synthetic and
+seeded; the per-step inputs are resident on the GPU before timing; L2 is
+flushed (512 MiB write) between steps, outside the timed events.
 
 The metric is decode tokens/s (one token per sequence per step); the
 roofline block reports the decode kernel's achieved HBM bandwidth from its
@@ -36,7 +39,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "decode-attention tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
-DEFAULT_WORKLOAD = "r1-llama-8b"
+DEFAULT_WORKLOAD = "churn"
+PER_CONFIG = ["r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b"]
 FLUSH_BYTES = 512 << 20
 DECODE_SRC = [os.path.join(ROOT, "mixed_precision_paged_thinkv_b200", "csrc", f)
               for f in ("thinkv_decode.cu", "thinkv_common.cuh", "thinkv_internal.h")]
@@ -230,65 +234,171 @@ def barrier(world):
 # --------------------------------------------------------------------------- #
 # oracle timing (CPU baseline and the reference arm)
 # --------------------------------------------------------------------------- #
-def time_oracle(w, steps: int, warmup: int, budget_s: float, gen_device: str):
-    """Replays the workload's setup in the oracle (untimed), then times oracle
-    steps (append + evict + decode over every sequence).  Returns a dict."""
-    import torch
-    from mixed_precision_paged_thinkv_b200 import workloads as W
-    from mixed_precision_paged_thinkv_b200.runner import geometry
-    from oracle import oracle as O
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
-    sched = W.Schedule(w, extra=warmup + steps + 2)
-    geom = geometry(w, sched)
-    o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
-                 geom["max_seqs"], geom["max_blocks_per_seq"], geom["pool_pages"])
+
+def sample_sequences(w, n_sample: int):
+    """An evenly spaced sample of the workload's sequences (all if it has fewer):
+    the CPU legs replay only these, so their cost stays bounded."""
+    if w.batch <= n_sample:
+        return list(range(w.batch))
+    return [int(x) for x in np.linspace(0, w.batch - 1, n_sample).round().astype(int)]
+
+
+class OracleReplay:
+    """The oracle replaying a sample of a workload's sequences: the same
+    prefill calls, setup evict, churn steps and timed steps as the GPU run,
+    restricted to those sequences.  Sequences never interact (except through
+    the numbering of pages), so each step's work per sequence is the work of
+    the full-batch run; throughput scales by sequences."""
+
+    def __init__(self, w, seqs, extra: int, gen_device: str):
+        import math as _m
+        from mixed_precision_paged_thinkv_b200 import workloads as W
+        from oracle import oracle as O
+        self.W, self.O = W, O
+        self.w, self.seqs, self.gen_device = w, list(seqs), gen_device
+        self.sched = W.Schedule(w, extra)
+        pool, mb = [0, 0, 0], 1
+        for s in self.seqs:
+            cnt = np.bincount(self.sched.tags(s), minlength=3)
+            pages = [int(_m.ceil(int(cnt[c]) / 16)) for c in range(3)]
+            pool = [a + b for a, b in zip(pool, pages)]
+            mb = max(mb, sum(pages))
+        self.o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
+                          len(self.seqs), mb, [max(1, p) for p in pool])
+        self.generated = self.sched.lengths[self.seqs].astype(np.int64).copy()
+        self.ids = np.arange(len(self.seqs), dtype=np.int32)
+
+    def _append(self, runs):
+        W, O = self.W, self.O
+        if not runs:
+            return
+        S, P, T, orig = [], [], [], []
+        for (j, p0, c) in runs:
+            s = self.seqs[j]
+            S.append(np.full(c, j, dtype=np.int32))
+            P.append(np.arange(p0, p0 + c, dtype=np.int32))
+            T.append(self.sched.tags(s)[p0:p0 + c])
+            orig.append(np.full(c, s, dtype=np.int64))
+        S, P, T, orig = map(np.concatenate, (S, P, T, orig))
+        k, v = W.kv_for_tokens(self.w, orig, P.astype(np.int64), device=self.gen_device)
+        assert self.o.append(S, P, T.astype(np.uint8), k.cpu(), v.cpu()) == O.OK
+
+    def setup(self):
+        where = {s: j for j, s in enumerate(self.seqs)}
+        for call in self.sched.prefill_calls():
+            self._append([(where[s], p0, c) for (s, p0, c) in call.runs if s in where])
+        assert self.o.evict(self.ids, self.sched.budgets(self.generated)) == self.O.OK
+        if self.w.post_evict_append:
+            n = self.w.post_evict_append
+            self._append([(j, int(self.generated[j]), n) for j in range(len(self.seqs))])
+            self.generated += n
+        for _ in range(self.w.churn_steps):
+            self.step_inputs_and_run(0, decode=False)
+
+    def step_inputs(self, step: int):
+        """The next step's inputs: one token per sampled sequence, budgets, Q rows."""
+        W = self.W
+        pos = self.generated.astype(np.int32)
+        tags = np.array([self.sched.tags(s)[int(p)] for s, p in zip(self.seqs, pos)], np.uint8)
+        k, v = W.kv_for_tokens(self.w, np.asarray(self.seqs, np.int64), pos.astype(np.int64),
+                               device=self.gen_device)
+        budgets = self.sched.budgets(self.generated + 1)
+        q = W.q_values(self.w, step, device=self.gen_device)[self.seqs].cpu()
+        return pos, tags, k.cpu(), v.cpu(), budgets, q
+
+    def run_step(self, inp, threads: int, decode: bool = True):
+        """append + evict (+ decode); returns (step seconds, decode seconds)."""
+        O = self.O
+        pos, tags, k, v, budgets, q = inp
+        t0 = time.perf_counter()
+        assert self.o.append(self.ids, pos, tags, k, v) == O.OK
+        assert self.o.evict(self.ids, budgets) == O.OK
+        t1 = time.perf_counter()
+        if decode:
+            self.o.decode(self.ids, q, topk=self.w.topk, threads=threads)
+        t2 = time.perf_counter()
+        self.generated += 1
+        return t2 - t0, t2 - t1
+
+    def step_inputs_and_run(self, step, decode=True, threads=1):
+        return self.run_step(self.step_inputs(step), threads, decode)
+
+
+def time_oracle(w, steps: int, warmup: int, budget_s: float, gen_device: str,
+                n_sample: int = 0, repeats: int = 5):
+    """The oracle as it stands, on a bounded sample of the workload: the
+    sampled sequences' setup is replayed untimed, then steps (append 1 token
+    per sequence + evict + decode) are timed.  Each step is timed with the
+    decode on all host cores and, on a copy of the same inputs, the decode
+    alone single-threaded is timed too.  Medians over up to `repeats` steps
+    (at least one), stopping once `budget_s` of timed work is spent."""
+    # one sampled sequence per host core at least: decode parallelises over sequences
+    seqs = sample_sequences(w, n_sample or max(8, os.cpu_count() or 1))
+    rep = OracleReplay(w, seqs, extra=warmup + steps + repeats + 4, gen_device=gen_device)
     t0 = time.time()
-    for call in sched.prefill_calls():
-        k, v = W.call_kv(w, call, device=gen_device)
-        assert o.append(call.seqs, call.pos, call.tags, k.cpu(), v.cpu()) == O.OK
-    gen = sched.lengths.astype(np.int64).copy()
-    allseq = np.arange(w.batch, dtype=np.int32)
-    assert o.evict(allseq, sched.budgets(gen)) == O.OK
+    rep.setup()
     setup_s = time.time() - t0
     threads = os.cpu_count() or 1
-    times = []
-    for k in range(warmup + steps):
-        call = sched.one_token_call(gen)
-        kk, vv = W.call_kv(w, call, device=gen_device)
-        kk, vv = kk.cpu(), vv.cpu()
-        q = W.q_values(w, k, device=gen_device).cpu()
-        gen = gen + 1
-        b = sched.budgets(gen)
+    for k in range(warmup):
+        rep.step_inputs_and_run(k, threads=threads)
+    step_s, dec_s, dec1_s = [], [], []
+    spent = 0.0
+    for k in range(max(1, min(steps, repeats))):
+        inp = rep.step_inputs(warmup + k)
+        st, dt = rep.run_step(inp, threads)
+        # the same decode again, single-threaded (the state did not change)
         t = time.perf_counter()
-        assert o.append(call.seqs, call.pos, call.tags, kk, vv) == O.OK
-        assert o.evict(allseq, b) == O.OK
-        o.decode(allseq, q, topk=w.topk, threads=threads)
-        dt = time.perf_counter() - t
-        if k >= warmup:
-            times.append(dt)
-        if k >= warmup and sum(times) > budget_s:
+        rep.o.decode(rep.ids, inp[5], topk=w.topk, threads=1)
+        d1 = time.perf_counter() - t
+        step_s.append(st)
+        dec_s.append(dt)
+        dec1_s.append(d1)
+        spent += st + d1
+        if spent > budget_s:
             break
-    total = sum(times)
-    return {"seconds": total, "steps": len(times), "tokens": w.batch * len(times),
-            "value": w.batch * len(times) / total, "cores": threads, "setup_s": setup_s}
+    med = lambda x: float(np.median(x))
+    n = len(seqs)
+    return {"value": n / med(step_s), "decode_tokens_per_s": n / med(dec_s),
+            "decode_tokens_per_s_1thread": n / med(dec1_s),
+            "step_ms": 1000 * med(step_s), "steps": len(step_s), "cores": threads,
+            "seqs": n, "setup_s": setup_s, "seconds": float(sum(step_s))}
+
+
+def _oracle_sample_text(w, r) -> str:
+    return (f"oracle (C, fp64 attention) on {r['seqs']} of {w.batch} sequences (evenly spaced), "
+            f"their setup replayed untimed; median of {r['steps']} steps of append 1 token/seq + "
+            f"evict + decode (decode on {r['cores']} OpenMP threads); tokens/s scaled per sequence; "
+            f"host CPU: {cpu_model()}")
 
 
 def reference_arm(args, w, world, rank):
     if rank != 0:
         return 0
     gen_device = "cuda" if _cuda_ok() else "cpu"
-    r = time_oracle(w, args.steps, args.warmup, budget_s=120.0, gen_device=gen_device)
+    r = time_oracle(w, max(args.steps, 1), min(args.warmup, 3), budget_s=60.0,
+                    gen_device=gen_device)
     line = {
         "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": r["steps"], "warmup": args.warmup,
-        "ms_per_step": 1000.0 * r["seconds"] / max(1, r["steps"]), "higher_is_better": True,
+        "ms_per_step": r["step_ms"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "dtype_detail": "attention in f64; the quantiser in the f32 operations it is defined with",
         "data": "synthetic", "config": workload_config(w, None),
         "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": r["cores"],
-                         "kind": "oracle",
-                         "sample": f"oracle replays the setup untimed, then {r['steps']} steps "
-                                   f"(append 1 token/seq + evict + decode over all {w.batch} seqs)"},
+                         "kind": "oracle", "sample": _oracle_sample_text(w, r),
+                         "cpu_model": cpu_model(),
+                         "decode_tokens_per_s": r["decode_tokens_per_s"],
+                         "decode_tokens_per_s_1thread": r["decode_tokens_per_s_1thread"]},
         "e2e": {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -308,7 +418,9 @@ def workload_config(w, live):
     cfg = {"workload": f"{w.name}: layer {w.num_q_heads}q/{w.num_kv_heads}kv heads, "
                        f"head_dim {w.head_dim}, batch {w.batch}, lengths {w.lengths}, "
                        f"R/E/T {w.bits[0]}/{w.bits[1]}/{w.bits[2]}-bit, group {w.group_size}, "
-                       f"budget {w.budget}",
+                       f"budget {w.budget}"
+                       + (f", {w.churn_steps} churn steps before timing" if w.churn_steps else "")
+                       + (f", top-{w.topk} mass" if w.topk else ""),
            "batch": w.batch, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
            "head_dim": w.head_dim, "group_size": w.group_size, "page_size": w.page_size,
            "bits_RET": list(w.bits), "topk": w.topk,
@@ -324,24 +436,21 @@ def workload_config(w, live):
 # --------------------------------------------------------------------------- #
 # the library arm
 # --------------------------------------------------------------------------- #
-def thinkv_arm(args, w, world, rank, local):
+def measure_workload(w, K: int, Wm: int, dev, flush, e2e_steps: int = 0, clocks=None,
+                     world: int = 1):
+    """Sets the workload up on the GPU, then times K steps (append + evict +
+    decode, one event pair per step, L2 flushed before each), the decode call
+    alone K times on the state the steps left, and (if e2e_steps) steps from
+    pinned host buffers.  Returns the measurements of this rank."""
     import torch
-    from mixed_precision_paged_thinkv_b200 import build as B
     from mixed_precision_paged_thinkv_b200.runner import (PackedStep, WorkloadRun, make_steps,
                                                           run_step, run_step_from_host)
-    B.build()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    K, Wm = args.steps, args.warmup
-    e2e_steps = max(3, min(K, 20))
     run = WorkloadRun(w, extra=Wm + K + e2e_steps + 2, device=str(dev))
     run.setup()
     torch.cuda.synchronize()
     steps = make_steps(run, Wm + K + e2e_steps, device=dev)
     out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float16, device=dev)
     mass = torch.empty(w.batch, w.num_q_heads, dtype=torch.float32, device=dev) if w.topk else None
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
     for k in range(Wm):
         flush.zero_()
         run_step(run.cache, steps[k], out, topk=w.topk, mass=mass)
@@ -349,15 +458,14 @@ def thinkv_arm(args, w, world, rank, local):
     assert run.cache.status() == 0, "device status after warm-up"
     snap = run.cache.snapshot()
     alg_bytes, live, pages = algorithmic_decode_bytes(w, snap)
+    del snap
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    # the raw nvidia-smi samples go to THINKV_CLOCK_LOG_DIR (default: the temp dir)
-    clocks = ClockSampler(os.path.join(os.environ.get("THINKV_CLOCK_LOG_DIR", tempfile.gettempdir()),
-                                       f"thinkv_clocks_rank{rank}.csv"))
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.4)
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.4)
     t_wall = time.time()
     for k in range(K):
         flush.zero_()
@@ -372,11 +480,11 @@ def thinkv_arm(args, w, world, rank, local):
     torch.cuda.synchronize()
     t_wall = time.time() - t_wall
     barrier(world)
-    clk = clocks.stop(str(torch.cuda.get_device_properties(dev).uuid))
+    clk = clocks.stop(str(torch.cuda.get_device_properties(dev).uuid)) if clocks is not None else None
     assert run.cache.status() == 0, "device status after the timed steps"
     step_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
-    # the decode kernel alone, for its roofline: the same launch on the state
-    # the timed steps left, L2 flushed before each
+    # the decode call alone, for its roofline: the same launch on the state the
+    # timed steps left, L2 flushed before each
     dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
     last = steps[Wm + K - 1]
@@ -387,46 +495,99 @@ def thinkv_arm(args, w, world, rank, local):
         dev_ev[k][1].record()
     torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in dev_ev]
-    step_s = sum(step_ms) / 1000.0
-    max_s, tokens = dist_max_sum(step_s, float(w.batch * K), world, dev)
-    value = tokens / max_s
+    res = {"step_s": sum(step_ms) / 1000.0, "steps": K, "tokens": float(w.batch * K),
+           "step_ms": step_ms, "dec_ms": dec_ms, "alg_bytes": alg_bytes, "live": live,
+           "pages": pages, "clocks": clk, "wall_s": t_wall}
 
-    # end to end through host buffers (pinned), copies inside the timed region
-    # each step's inputs packed in one pinned buffer: one copy per step
-    host = [PackedStep(steps[Wm + K + k], "cpu", pin=True).fill(steps[Wm + K + k])
-            for k in range(e2e_steps)]
-    dbuf = PackedStep(steps[Wm + K], dev)  # device staging, overwritten by the copies
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    mass_h = torch.empty(mass.shape, dtype=mass.dtype).pin_memory() if w.topk else None
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(e2e_steps)]
-    torch.cuda.synchronize()
-    for k in range(e2e_steps):
-        flush.zero_()
-        e2e_ev[k][0].record()
-        run_step_from_host(run.cache, host[k], dbuf, out, out_h, topk=w.topk,
-                           mass_dev=mass, mass_host=mass_h)
-        e2e_ev[k][1].record()
-    torch.cuda.synchronize()
-    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1000.0
-    e2e_max, e2e_tok = dist_max_sum(e2e_s, float(w.batch * e2e_steps), world, dev)
-    h2d = host[0].nbytes()
-    d2h = out_h.numel() * 2 + (mass_h.numel() * 4 if w.topk else 0)
+    if e2e_steps:
+        # end to end through host buffers (pinned), copies inside the timed
+        # region; each step's inputs packed in one pinned buffer: one copy
+        host = [PackedStep(steps[Wm + K + k], "cpu", pin=True).fill(steps[Wm + K + k])
+                for k in range(e2e_steps)]
+        dbuf = PackedStep(steps[Wm + K], dev)  # device staging, overwritten by the copies
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        mass_h = torch.empty(mass.shape, dtype=mass.dtype).pin_memory() if w.topk else None
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(e2e_steps)]
+        torch.cuda.synchronize()
+        for k in range(e2e_steps):
+            flush.zero_()
+            e2e_ev[k][0].record()
+            run_step_from_host(run.cache, host[k], dbuf, out, out_h, topk=w.topk,
+                               mass_dev=mass, mass_host=mass_h)
+            e2e_ev[k][1].record()
+        torch.cuda.synchronize()
+        res["e2e_s"] = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1000.0
+        res["e2e_tokens"] = float(w.batch * e2e_steps)
+        res["e2e_steps"] = e2e_steps
+        res["h2d"] = host[0].nbytes()
+        res["d2h"] = out_h.numel() * 2 + (mass_h.numel() * 4 if w.topk else 0)
+    del run, steps
+    torch.cuda.empty_cache()
+    return res
 
-    # roofline of the decode kernel (one launch per decode call)
-    dec_avg_s = sum(dec_ms) / len(dec_ms) / 1000.0
-    achieved = alg_bytes / dec_avg_s / 1e9
+
+def roofline_block(w, res):
+    """Roofline of the decode call from its algorithmic bytes and event time."""
+    dec_avg_s = sum(res["dec_ms"]) / len(res["dec_ms"]) / 1000.0
+    achieved = res["alg_bytes"] / dec_avg_s / 1e9
     peak, peak_kind = peak_hbm_gbs()
-    traffic = traffic_per_launch(w.name)
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": traffic_per_launch(w.name),
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+            "kernel": DECODE_KERNELS,
+            "algorithmic_bytes_per_launch": res["alg_bytes"], "live_pages": res["pages"]}
+
+
+DECODE_KERNELS = "decode call: decode_split_kernel + decode_combine_kernel"
+
+
+def thinkv_arm(args, w, world, rank, local):
+    import torch
+    from mixed_precision_paged_thinkv_b200 import build as B
+    from mixed_precision_paged_thinkv_b200 import workloads as W
+    B.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    K, Wm = args.steps, args.warmup
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    # the raw nvidia-smi samples go to THINKV_CLOCK_LOG_DIR (default: the temp dir)
+    clocks = ClockSampler(os.path.join(os.environ.get("THINKV_CLOCK_LOG_DIR", tempfile.gettempdir()),
+                                       f"thinkv_clocks_rank{rank}.csv"))
+    e2e_steps = max(3, min(K, 20))
+    res = measure_workload(w, K, Wm, dev, flush, e2e_steps=e2e_steps, clocks=clocks, world=world)
+    max_s, tokens = dist_max_sum(res["step_s"], res["tokens"], world, dev)
+    value = tokens / max_s
+    e2e_max, e2e_tok = dist_max_sum(res["e2e_s"], res["e2e_tokens"], world, dev)
+
+    # the other budgeted configurations, same run (single-GPU runs only)
+    per_config = {}
+    if world == 1 and not args.no_per_config and w.name == DEFAULT_WORKLOAD:
+        for name in PER_CONFIG:
+            wc = W.get(name)
+            Kc = max(3, min(K, 20))
+            rc = measure_workload(wc, Kc, 3, dev, flush)
+            dec = sum(rc["dec_ms"]) / len(rc["dec_ms"])
+            per_config[name] = {
+                "config": workload_config(wc, rc["live"]),
+                "steps": Kc, "warmup": 3,
+                "ms_per_step": 1000.0 * rc["step_s"] / Kc,
+                "value": rc["tokens"] / rc["step_s"], "unit": "tokens/s",
+                "decode_ms": dec,
+                "decode_kv_tokens_per_s": float(sum(rc["live"])) / (dec / 1000.0),
+                "roofline": roofline_block(wc, rc)}
+
     result = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            r = time_oracle(w, steps=200, warmup=1, budget_s=15.0, gen_device=str(dev))
+            r = time_oracle(w, steps=5, warmup=1, budget_s=20.0, gen_device=str(dev))
             cpu = {"value": r["value"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
-                   "sample": f"oracle (C, fp64 attention) replays the setup untimed, then "
-                             f"{r['steps']} steps of append 1 token/seq + evict + decode over all "
-                             f"{w.batch} seqs (~15 s cap); decode on {r['cores']} OpenMP threads"}
+                   "sample": _oracle_sample_text(w, r), "cpu_model": cpu_model(),
+                   "decode_tokens_per_s": r["decode_tokens_per_s"],
+                   "decode_tokens_per_s_1thread": r["decode_tokens_per_s_1thread"],
+                   "setup_replay_s": r["setup_s"]}
+        dec = sum(res["dec_ms"]) / len(res["dec_ms"])
         result = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": Wm, "ms_per_step": 1000.0 * max_s / K,
@@ -434,21 +595,18 @@ def thinkv_arm(args, w, world, rank, local):
             "dtype": "f16",
             "dtype_detail": "8/4/2-bit integer codes dequantised into f16 mma operands, f32 accumulate",
             "data": "synthetic (seeded counter-hash normals, segment tags)",
-            "config": workload_config(w, live),
-            "decode_ms": sum(dec_ms) / len(dec_ms),
-            "decode_hbm_gbs": achieved,
-            "decode_kv_tokens_per_s": float(sum(live)) / dec_avg_s,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
-                         "kernel": "decode call: decode_split_kernel + decode_combine_kernel",
-                         "algorithmic_bytes_per_launch": alg_bytes, "live_pages": pages},
+            "config": workload_config(w, res["live"]),
+            "decode_ms": dec,
+            "decode_hbm_gbs": res["alg_bytes"] / (dec / 1000.0) / 1e9,
+            "decode_kv_tokens_per_s": float(sum(res["live"])) / (dec / 1000.0),
+            "roofline": roofline_block(w, res),
+            "per_config": per_config or None,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_tok / e2e_max, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "e2e": {"value": e2e_tok / e2e_max, "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
+                    "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},
             "gpu_launches": launches_per_step(w.batch) * K,
-            "clocks": clk,
-            "wall_s_timed_loop": t_wall,
+            "clocks": res["clocks"],
+            "wall_s_timed_loop": res["wall_s"],
         }
     return result
 
@@ -461,6 +619,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="thinkv", choices=["thinkv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the chosen workload (skip the per_config block)")
     args = ap.parse_args()
     from mixed_precision_paged_thinkv_b200 import workloads as W
     w = W.get(args.workload)

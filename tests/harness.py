@@ -271,6 +271,47 @@ def compare_codes_by_pos(cache, gl: dict, oracle: O.Oracle, ol: dict):
             assert np.array_equal(vp[n, :, gslots], op[opages, :, 1, oslots]), f"V params class {c}"
 
 
+def compare_seq_structure(g: dict, s: int, o: dict, j: int):
+    """Bit-exact comparison of GPU sequence s with oracle sequence j, where the
+    two runs number pool pages differently (the oracle replays a subset of the
+    batch).  Everything the state holds per sequence is in per-sequence terms
+    (table entry indices, slot ids entry*16 + slot, counters) and must match
+    exactly; page ids are compared through the entry -> page map each side's
+    table defines, which must be a bijection."""
+    for key in ("num_blocks", "live_count", "num_live"):
+        assert int(g[key][s]) == int(o[key][j]), f"{key} of seq {s}"
+    for key in ("free_top", "fifo_head", "fifo_tail"):
+        assert np.array_equal(g[key][s], o[key][j]), f"{key} of seq {s}"
+    nb = int(o["num_blocks"][j])
+    gt, ot = g["table"][s, :nb], o["table"][j, :nb]
+    assert np.array_equal(O.entry_class(gt), O.entry_class(ot)), f"entry classes of seq {s}"
+    assert np.array_equal(O.entry_mask(gt), O.entry_mask(ot)), f"entry masks of seq {s}"
+    gp, op = O.entry_page(gt).astype(np.int64), O.entry_page(ot).astype(np.int64)
+    assert len(set(gp.tolist())) == nb, f"GPU pages of seq {s} repeat"
+    # slot positions of every slot of every entry, through the page map
+    for c in range(3):
+        sel = np.flatnonzero(O.entry_class(ot) == c)
+        if sel.size:
+            gsp = g["slot_pos"][c][gp[sel]]
+            osp = o["slot_pos"][c][op[sel]]
+            assert np.array_equal(gsp, osp), f"slot_pos of seq {s} class {c}"
+    cap = g["fifo"].shape[2]
+    for c in range(3):
+        top = int(o["free_top"][j, c])
+        assert np.array_equal(g["free_slots"][s, c, :top], o["free_slots"][j, c, :top]), \
+            f"free stack of seq {s} class {c}"
+        h, t = int(o["fifo_head"][j, c]), int(o["fifo_tail"][j, c])
+        idx = np.arange(h, t) % cap
+        assert np.array_equal(g["fifo"][s, c, idx], o["fifo"][j, c, idx]), f"fifo of seq {s} class {c}"
+    nl = int(o["num_live"][j])
+    gl, ol = g["live_list"][s, :nl], o["live_list"][j, :nl]
+    assert np.array_equal(O.live_entry(gl), O.live_entry(ol)), f"live list order of seq {s}"
+    assert np.array_equal(O.entry_class(gl), O.entry_class(ol)), f"live list classes of seq {s}"
+    assert np.array_equal(O.entry_page(gl).astype(np.int64), gp[O.live_entry(gl)]), \
+        f"live list pages of seq {s}"
+    assert np.array_equal(g["live_index"][s, :nb], o["live_index"][j, :nb]), f"live index of seq {s}"
+
+
 def check_slot_invariants(snap, ns):
     """Free-slot invariants of every sequence (no oracle needed): per (sequence,
     class) the allocated slots are exactly the live ones plus the free-stack

@@ -31,7 +31,9 @@ def _check(g, osub, step, topk):
     assert g.cache.status() == 0
     snap = g.cache.snapshot()
     Hn.check_slot_invariants(snap, g.w.batch)
+    ost = osub.o.state()
     for j, s in enumerate(osub.seqs):
+        Hn.compare_seq_structure(snap, s, ost, j)
         gl = Hn.gpu_live_by_pos(snap, s)
         ol = osub.live_by_pos(j)
         assert sorted(gl) == sorted(ol), f"live positions of seq {s}"

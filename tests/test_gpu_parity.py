@@ -186,3 +186,73 @@ def test_topk_mass_long_pieces_and_tied_logits(k):
     assert err <= Hn.TOL, err
     assert merr <= Hn.MASS_TOL, merr
     assert np.allclose(m[:4], k / L, rtol=1e-3, atol=0), m[:4].min()
+
+
+@pytest.mark.parametrize("order", [(0, 1, 2), (1, 2, 0), (2, 0, 1), (0, 2, 1)])
+def test_eviction_class_orders(order):
+    """A non-default class order for eviction (the `order` argument): the
+    victims, freed slots and live lists must match the oracle's, through a
+    first evict that reaches into every class and churn steps after it."""
+    w = W.Workload(name="x", batch=3, num_q_heads=8, num_kv_heads=2, head_dim=128, group_size=64,
+                   lengths=("uniform", 300, 900), budget=("frac", 0.2), seed=13)
+    g, o = _pair(w, extra=12)
+    for call in g.sched.prefill_calls():
+        g.append_call(call)
+        o.append_call(call)
+    dev = torch.device("cuda")
+    seqs = torch.arange(w.batch, dtype=torch.int32, device=dev)
+    for step in range(4):
+        b = g.sched.budgets(g.generated)
+        g.cache.evict(seqs, torch.as_tensor(b, device=dev), order=order)
+        assert o.o.evict(o.all_seqs, b, order=order) == 0
+        _check_all(g, o, step=step, topk=4, codes=(step == 0))
+        call = g.sched.one_token_call(g.generated)
+        g.append_call(call)
+        o.append_call(call)
+        g.generated += 1
+        o.generated += 1
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.5])
+def test_explicit_softmax_scale(scale):
+    """softmax_scale > 0 replaces 1/sqrt(d): a flat (0.02) and a sharp (0.5)
+    softmax against the oracle with the same scale."""
+    w = W.Workload(name="x", batch=3, num_q_heads=16, num_kv_heads=4, head_dim=64, group_size=32,
+                   lengths=("uniform", 200, 1200), budget=("frac", 0.3), seed=17)
+    g, o = _pair(w)
+    g.setup()
+    o.setup()
+    torch.cuda.synchronize()
+    q = W.q_values(w, 0, device="cuda")
+    out, mass = g.cache.decode(g.all_seqs, q, topk=8, softmax_scale=scale)
+    ref, rmass = o.o.decode(o.all_seqs, W.q_values(w, 0), softmax_scale=scale, topk=8, threads=8)
+    err = Hn.attn_error(out.cpu().numpy(), ref)
+    merr = float(np.abs(mass.cpu().numpy().astype(np.float64) - rmass).max())
+    print(f"scale {scale}: attention error {err:.3e}, top-k mass error {merr:.3e}")
+    assert err <= Hn.TOL and merr <= Hn.MASS_TOL, (err, merr)
+
+
+def test_decode_shuffled_subset_with_repeated_ids():
+    """decode over a permuted subset of the sequences with one id twice: row i
+    of the output belongs to seq[i], whatever the order, and a repeated id
+    gives the same row twice."""
+    w = W.Workload(name="x", batch=6, num_q_heads=16, num_kv_heads=4, head_dim=128, group_size=64,
+                   lengths=("uniform", 100, 1500), budget=("frac", 0.25), seed=19)
+    g, o = _pair(w)
+    g.setup()
+    o.setup()
+    torch.cuda.synchronize()
+    ids = np.array([4, 1, 5, 1, 0], dtype=np.int32)
+    qall = W.q_values(w, 3)
+    q = qall[[0, 1, 2, 3, 4]].contiguous()           # one query row set per call slot
+    out, mass = g.cache.decode(torch.as_tensor(ids, device="cuda"), q.cuda(), topk=6)
+    ref, rmass = o.o.decode(ids, q, topk=6, threads=8)
+    err = Hn.attn_error(out.cpu().numpy(), ref)
+    merr = float(np.abs(mass.cpu().numpy().astype(np.float64) - rmass).max())
+    print(f"shuffled subset: attention error {err:.3e}, top-k mass error {merr:.3e}")
+    assert err <= Hn.TOL and merr <= Hn.MASS_TOL, (err, merr)
+    # the repeated id with the same query gives the same row
+    q2 = q.clone()
+    q2[3] = q2[1]
+    out2, _ = g.cache.decode(torch.as_tensor(ids, device="cuda"), q2.cuda())
+    assert torch.equal(out2[1], out2[3])

@@ -34,9 +34,12 @@ def test_subset_replay_equals_full_replay():
     sub = Hn.OracleSubset(w, seqs, extra=0, gen_device="cpu")
     sub.setup()
     fs = full.o.state()
+    ss = sub.o.state()
     Hn.check_slot_invariants(fs, w.batch)
-    Hn.check_slot_invariants(sub.o.state(), len(seqs))
+    Hn.check_slot_invariants(ss, len(seqs))
     for j, s in enumerate(seqs):
+        # the whole per-sequence state, through the entry -> page map
+        Hn.compare_seq_structure(fs, s, ss, j)
         a, b = _by_pos(fs, s), sub.live_by_pos(j)
         assert sorted(a) == sorted(b)
         for c in range(3):
@@ -70,3 +73,59 @@ def test_slot_invariants_catch_a_lost_slot():
     except AssertionError:
         return
     raise AssertionError("a slot missing from the free stack went unnoticed")
+
+
+def test_structure_comparison_catches_planted_differences():
+    """compare_seq_structure (used on the full-size GPU states) must notice a
+    swapped FIFO pair, a flipped mask bit, a reordered free stack, a moved
+    live-list entry and a wrong slot position."""
+    import copy
+    w = W.scaled(W.WORKLOADS["churn"], batch=3, lengths=("fixed", 700), churn_steps=5,
+                 budget=("frac", 0.2))
+    sched = W.Schedule(w, 0)
+    full = Hn.OracleRun(w, geometry(w, sched), extra=0)
+    full.setup()
+    sub = Hn.OracleSubset(w, [2], extra=0, gen_device="cpu")
+    sub.setup()
+    fs, ss = full.o.state(), sub.o.state()
+    Hn.compare_seq_structure(fs, 2, ss, 0)
+    cap = ss["fifo"].shape[2]
+
+    def plant(edit):
+        st = copy.deepcopy(ss)
+        edit(st)
+        try:
+            Hn.compare_seq_structure(fs, 2, st, 0)
+        except AssertionError:
+            return
+        raise AssertionError("a planted difference went unnoticed")
+
+    c = int(np.argmax(ss["fifo_tail"][0] - ss["fifo_head"][0]))
+    h = int(ss["fifo_head"][0, c])
+
+    def swap_fifo(st):
+        a, b = h % cap, (h + 1) % cap
+        st["fifo"][0, c, [a, b]] = st["fifo"][0, c, [b, a]]
+    plant(swap_fifo)
+
+    def flip_mask(st):
+        st["table"][0, 0] ^= np.uint64(1 << 48)
+    plant(flip_mask)
+
+    cf = int(np.argmax(ss["free_top"][0]))
+
+    def reorder_stack(st):
+        st["free_slots"][0, cf, [0, 1]] = st["free_slots"][0, cf, [1, 0]]
+    assert ss["free_top"][0, cf] >= 2
+    plant(reorder_stack)
+
+    def move_live(st):
+        st["live_list"][0, [0, 1]] = st["live_list"][0, [1, 0]]
+    assert ss["num_live"][0] >= 2
+    plant(move_live)
+
+    def wrong_pos(st):
+        e = st["table"][0, 0]
+        cls, page = int(O.entry_class(e)), int(O.entry_page(e))
+        st["slot_pos"][cls][page, 3] += 1
+    plant(wrong_pos)
