@@ -277,7 +277,7 @@ def compare_seq_structure(g: dict, s: int, o: dict, j: int):
     batch).  Everything the state holds per sequence is in per-sequence terms
     (table entry indices, slot ids entry*16 + slot, counters) and must match
     exactly; page ids are compared through the entry -> page map each side's
-    table defines, which must be a bijection."""
+    table defines, which must be one-to-one on (class, page)."""
     for key in ("num_blocks", "live_count", "num_live"):
         assert int(g[key][s]) == int(o[key][j]), f"{key} of seq {s}"
     for key in ("free_top", "fifo_head", "fifo_tail"):
@@ -287,7 +287,9 @@ def compare_seq_structure(g: dict, s: int, o: dict, j: int):
     assert np.array_equal(O.entry_class(gt), O.entry_class(ot)), f"entry classes of seq {s}"
     assert np.array_equal(O.entry_mask(gt), O.entry_mask(ot)), f"entry masks of seq {s}"
     gp, op = O.entry_page(gt).astype(np.int64), O.entry_page(ot).astype(np.int64)
-    assert len(set(gp.tolist())) == nb, f"GPU pages of seq {s} repeat"
+    # page ids number each class pool separately: (class, page) is the key
+    gkey = (O.entry_class(gt).astype(np.int64) << 32) | gp
+    assert len(set(gkey.tolist())) == nb, f"GPU pages of seq {s} repeat"
     # slot positions of every slot of every entry, through the page map
     for c in range(3):
         sel = np.flatnonzero(O.entry_class(ot) == c)
