@@ -72,12 +72,14 @@ def lib():
             L.or_f16_to_f32.restype = C.c_float
             L.or_f16_round_array.argtypes = [P, C.c_int64, C.c_int32, P]
             L.or_quantize_group.argtypes = [P, C.c_int32, C.c_int32, P, P, P]
+            L.or_classify.argtypes = [C.c_int32, C.c_int32, P, C.c_float, C.c_float, P]
+            L.or_tbe.argtypes = [P, C.c_int32, P, P, P, C.c_int32, P]
             for f in ("or_codes", "or_params", "or_slot_pos"):
                 getattr(L, f).argtypes = [P, C.c_int]
                 getattr(L, f).restype = P
             for f in ("or_table", "or_num_blocks", "or_free_slots", "or_free_top", "or_fifo",
                       "or_fifo_head", "or_fifo_tail", "or_live_count", "or_live_list",
-                      "or_live_index", "or_num_live", "or_page_bump"):
+                      "or_live_index", "or_num_live", "or_page_bump", "or_seg", "or_nseg"):
                 getattr(L, f).argtypes = [P]
                 getattr(L, f).restype = P
             _lib = L
@@ -132,6 +134,15 @@ def quantize_group(x, bits: int):
     return codes, int(s[0]), int(z[0])
 
 
+def classify(mass, theta_t: float, theta_r: float) -> np.ndarray:
+    """R/E/T tags (uint8 [n]) from top-k masses (float32 [n, hq])."""
+    m = np.ascontiguousarray(mass, dtype=np.float32)
+    n, hq = m.shape
+    tags = np.zeros(n, dtype=np.uint8)
+    lib().or_classify(n, hq, _ptr(m), C.c_float(theta_t), C.c_float(theta_r), _ptr(tags))
+    return tags
+
+
 # -- one oracle cache ---------------------------------------------------------- #
 class Oracle:
     """One oracle state with the given geometry."""
@@ -179,6 +190,15 @@ class Oracle:
         o = None if order is None else np.ascontiguousarray(order, dtype=np.uint8)
         return int(lib().or_evict(self._h, seq.shape[0], _ptr(seq), _ptr(budget),
                                   None if o is None else _ptr(o)))
+
+    def tbe(self, seq, pos, tag, t_min: int = 0, schedule: Optional[Sequence[int]] = None) -> int:
+        """TBE after an append of the same tokens (see or_tbe)."""
+        seq = np.ascontiguousarray(seq, dtype=np.int32)
+        pos = np.ascontiguousarray(pos, dtype=np.int32)
+        tag = np.ascontiguousarray(tag, dtype=np.uint8)
+        sch = None if schedule is None else np.ascontiguousarray(schedule, dtype=np.int32)
+        return int(lib().or_tbe(self._h, seq.shape[0], _ptr(seq), _ptr(pos), _ptr(tag),
+                                int(t_min), None if sch is None else _ptr(sch)))
 
     def decode(self, seq, q, softmax_scale: float = 0.0, topk: Optional[int] = None,
                threads: int = 1):
@@ -233,6 +253,8 @@ class Oracle:
             "live_index": self._arr("or_live_index", np.int32, (ns, nb)),
             "num_live": self._arr("or_num_live", np.int32, (ns,)),
             "page_bump": self._arr("or_page_bump", np.int32, (3,)),
+            "seg": self._arr("or_seg", np.int32, (ns, nb * PAGE, 5)),
+            "nseg": self._arr("or_nseg", np.int32, (ns,)),
             "slot_pos": [self.slot_pos(c) for c in range(3)],
         }
 

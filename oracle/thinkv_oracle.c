@@ -165,7 +165,13 @@ struct or_state {
   int32_t* live_index;
   int32_t* num_live;
   int32_t page_bump[3];
+  /* TBE segments: per sequence, up to cap records of SEG_FIELDS ints */
+  int32_t* seg;
+  int32_t* nseg;
 };
+
+/* fields of one TBE segment record */
+enum { SEG_CLS = 0, SEG_LEVEL = 1, SEG_LO = 2, SEG_LEN = 3, SEG_TRIM = 4, SEG_FIELDS = 5 };
 
 #define ENTRY_PAGE(e) ((int32_t)((e) & 0xFFFFFFFFull))
 #define ENTRY_CLASS(e) ((int32_t)(((e) >> 32) & 0xFF))
@@ -226,6 +232,9 @@ or_state* or_create(const or_layout* L) {
   S->live_list = (uint64_t*)calloc(ns * nb, sizeof(uint64_t));
   S->live_index = (int32_t*)malloc(ns * nb * sizeof(int32_t));
   S->num_live = (int32_t*)calloc(ns, sizeof(int32_t));
+  S->seg = (int32_t*)calloc(ns * (size_t)S->cap * SEG_FIELDS + 1, sizeof(int32_t));
+  S->nseg = (int32_t*)calloc(ns, sizeof(int32_t));
+  if (!S->seg || !S->nseg) fail = 1;
   if (!S->table || !S->num_blocks || !S->free_slots || !S->free_top || !S->fifo ||
       !S->fifo_head || !S->fifo_tail || !S->live_count || !S->live_list ||
       !S->live_index || !S->num_live)
@@ -241,6 +250,7 @@ void or_destroy(or_state* S) {
   free(S->table); free(S->num_blocks); free(S->free_slots); free(S->free_top);
   free(S->fifo); free(S->fifo_head); free(S->fifo_tail); free(S->live_count);
   free(S->live_list); free(S->live_index); free(S->num_live);
+  free(S->seg); free(S->nseg);
   free(S);
 }
 
@@ -364,10 +374,36 @@ int or_append(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos,
 /* ====================================================================== */
 /* evict to budget [TBE][CT]                                               */
 /* ====================================================================== */
+/* One victim: table slot ts (entry*16 + slot) of class c in sequence s.  Its
+ * mask bit is cleared (an entry left with no live token leaves the live-page
+ * list by swap-with-last), its start index set to -1, its slot pushed onto
+ * its class's free stack, and the live count drops.  Nothing is moved. */
+static void evict_token(or_state* S, int s, int c, int32_t ts) {
+  const or_layout* L = &S->L;
+  int32_t e = ts / OR_PAGE, slot = ts % OR_PAGE;
+  uint64_t* ent = &table_row(S, s)[e];
+  *ent &= ~((uint64_t)1 << (48 + slot));
+  if (ENTRY_MASK(*ent) == 0) {                 /* page emptied: swap-remove */
+    uint64_t* list = S->live_list + (size_t)s * L->max_blocks_per_seq;
+    int32_t* index = S->live_index + (size_t)s * L->max_blocks_per_seq;
+    int32_t at = index[e], last = --S->num_live[s];
+    uint64_t moved = list[last];
+    list[at] = moved;
+    index[LIVE_ENTRY(moved)] = at;
+    index[e] = -1;
+  }
+  S->slot_pos[c][(size_t)ENTRY_PAGE(*ent) * OR_PAGE + slot] = -1;
+  int32_t* top = &S->free_top[s * 3 + c];
+  free_stack(S, s, c)[(*top)++] = ts;
+  S->live_count[s]--;
+}
+
 /* Reading: n = max(0, live - budget) victims, taken oldest first from the
  * class FIFOs in the given class order (default T, then E, then R).  Each
  * victim's mask bit is cleared, its start index set to -1 and its slot pushed
- * onto its class's free stack, in victim order.  Pages are never released. */
+ * onto its class's free stack, in victim order.  Pages are never released.
+ * A FIFO entry of -1 is a tombstone (a token TBE already evicted): taking a
+ * victim from a class first steps its head over the tombstones there. */
 int or_evict(or_state* S, int32_t n, const int32_t* seq, const int32_t* budget,
              const uint8_t* order) {
   const or_layout* L = &S->L;
@@ -391,30 +427,153 @@ int or_evict(or_state* S, int32_t n, const int32_t* seq, const int32_t* budget,
       int c = -1;
       for (int o = 0; o < 3; ++o) {
         int cc = order[o];
-        if (S->fifo_head[s * 3 + cc] < S->fifo_tail[s * 3 + cc]) { c = cc; break; }
+        int32_t* head = &S->fifo_head[s * 3 + cc];
+        while (*head < S->fifo_tail[s * 3 + cc] && fifo_ring(S, s, cc)[(*head) % S->cap] < 0)
+          (*head)++;                             /* tombstone */
+        if (*head < S->fifo_tail[s * 3 + cc]) { c = cc; break; }
       }
       if (c < 0) break;                          /* unreachable: live > budget >= 0 */
       int32_t* head = &S->fifo_head[s * 3 + c];
       int32_t ts = fifo_ring(S, s, c)[(*head) % S->cap];
       (*head)++;
-      int32_t e = ts / OR_PAGE, slot = ts % OR_PAGE;
-      uint64_t* ent = &table_row(S, s)[e];
-      *ent &= ~((uint64_t)1 << (48 + slot));
-      if (ENTRY_MASK(*ent) == 0) {               /* page emptied: swap-remove */
-        uint64_t* list = S->live_list + (size_t)s * L->max_blocks_per_seq;
-        int32_t* index = S->live_index + (size_t)s * L->max_blocks_per_seq;
-        int32_t at = index[e], last = --S->num_live[s];
-        uint64_t moved = list[last];
-        list[at] = moved;
-        index[LIVE_ENTRY(moved)] = at;
-        index[e] = -1;
-      }
-      S->slot_pos[c][(size_t)ENTRY_PAGE(*ent) * OR_PAGE + slot] = -1;
-      int32_t* top = &S->free_top[s * 3 + c];
-      free_stack(S, s, c)[(*top)++] = ts;
-      S->live_count[s]--;
+      evict_token(S, s, c, ts);
     }
   }
+  return OR_OK;
+}
+
+/* ====================================================================== */
+/* TBE: segment-level eviction on Transition thoughts                      */
+/* ====================================================================== */
+/* Explainer, Methodologie, "Eviction Adaptative a la Pensee (TBE)": when a
+ * Transition thought appears, tokens of the earlier, less critical Reasoning
+ * and Execution segments are evicted progressively along an annealing
+ * schedule (retention 64, then 32, then 16), a segment at a time rather than
+ * token by token; and (the explainer's "Astuce B") a small safety net of
+ * Transition tokens is always kept.  Readings:
+ *   - a segment is a maximal run of consecutive tokens of one sequence with
+ *     the same tag, in append order; a T event is the first token of a new T
+ *     segment;
+ *   - at a T event each earlier R or E segment takes the next step of the
+ *     schedule (its k-th event keeps at most schedule[min(k,3)-1] tokens) and
+ *     each earlier T segment keeps only its share of the t_min most recent
+ *     live tokens of all earlier T segments;
+ *   - a segment gives up its oldest live tokens first (the segment's live
+ *     tokens are always a suffix of it); victims go in segment order, then
+ *     token order;
+ *   - an evicted token's FIFO entry becomes a tombstone (-1), since it need
+ *     not be at the FIFO head.
+ * A segment record holds its class, schedule level, the FIFO counter of its
+ * first token (lo), its length, and trim: how far from lo TBE has passed.
+ * Its live tokens are the FIFO entries [max(lo + trim, head), lo + len). */
+static int32_t* seg_rec(or_state* S, int s, int32_t j) {
+  return S->seg + (((size_t)s * S->cap) + (size_t)j) * SEG_FIELDS;
+}
+
+static int32_t seg_first_live(const or_state* S, int s, const int32_t* g) {
+  int32_t a = g[SEG_LO] + g[SEG_TRIM], head = S->fifo_head[s * 3 + g[SEG_CLS]];
+  return a > head ? a : head;
+}
+
+static int32_t seg_live(const or_state* S, int s, const int32_t* g) {
+  int32_t live = g[SEG_LO] + g[SEG_LEN] - seg_first_live(S, s, g);
+  return live > 0 ? live : 0;
+}
+
+/* the x oldest live tokens of segment g, tombstoned in the FIFO */
+static void trim_segment(or_state* S, int s, int32_t* g, int32_t x) {
+  int c = g[SEG_CLS];
+  int32_t first = seg_first_live(S, s, g);
+  for (int32_t k = 0; k < x; ++k) {
+    int32_t* entry = &fifo_ring(S, s, c)[(first + k) % S->cap];
+    evict_token(S, s, c, *entry);
+    *entry = -1;
+  }
+  g[SEG_TRIM] = first + x - g[SEG_LO];
+}
+
+/* the T event that opens segment e of sequence s */
+static void tbe_event(or_state* S, int s, int32_t e, int32_t t_min, const int32_t* schedule) {
+  int32_t* keep_t = (int32_t*)calloc((size_t)e + 1, sizeof(int32_t));
+  int32_t net = t_min;                           /* safety net, newest T tokens first */
+  for (int32_t j = e - 1; j >= 0; --j) {
+    int32_t* g = seg_rec(S, s, j);
+    if (g[SEG_CLS] != OR_T) continue;
+    int32_t live = seg_live(S, s, g), k = live < net ? live : net;
+    keep_t[j] = k;
+    net -= k;
+  }
+  for (int32_t j = 0; j < e; ++j) {
+    int32_t* g = seg_rec(S, s, j);
+    int32_t live = seg_live(S, s, g), x;
+    if (g[SEG_CLS] == OR_T) {
+      x = live - keep_t[j];
+    } else {
+      if (g[SEG_LEVEL] < 3) g[SEG_LEVEL]++;
+      x = live - schedule[g[SEG_LEVEL] - 1];
+    }
+    if (x > 0) trim_segment(S, s, g, x);
+  }
+  free(keep_t);
+}
+
+int or_tbe(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos, const uint8_t* tag,
+           int32_t t_min, const int32_t* schedule) {
+  const or_layout* L = &S->L;
+  static const int32_t default_schedule[3] = {64, 32, 16};
+  if (!schedule) schedule = default_schedule;
+  if (n < 0 || t_min < 0 || schedule[0] < 0 || schedule[1] < 0 || schedule[2] < 0)
+    return OR_ERR_INVALID;
+  if (n == 0) return OR_OK;
+  int ns = L->max_seqs;
+  /* the same token runs as the append that has just stored them */
+  char* seen = (char*)calloc((size_t)ns, 1);
+  int64_t* cnt = (int64_t*)calloc((size_t)ns * 3, sizeof(int64_t));
+  int32_t* newseg = (int32_t*)calloc((size_t)ns, sizeof(int32_t));
+  int bad = 0;
+  for (int32_t i = 0; i < n && !bad; ++i) {
+    int s = seq[i];
+    if (s < 0 || s >= ns || tag[i] > 2 || pos[i] < 0) { bad = 1; break; }
+    int new_run = (i == 0 || seq[i - 1] != s);
+    if (new_run) {
+      if (seen[s]) bad = 1;
+      seen[s] = 1;
+    } else if (pos[i] <= pos[i - 1]) bad = 1;
+    cnt[(size_t)s * 3 + tag[i]]++;
+    int32_t last_cls = new_run ? (S->nseg[s] > 0 ? seg_rec(S, s, S->nseg[s] - 1)[SEG_CLS] : -1)
+                               : tag[i - 1];
+    if (tag[i] != last_cls) newseg[s]++;
+  }
+  for (int s = 0; s < ns && !bad; ++s)
+    if ((int64_t)S->nseg[s] + newseg[s] > S->cap) bad = 1;
+  free(seen);
+  free(newseg);
+  if (bad) { free(cnt); return OR_ERR_INVALID; }
+  /* the append pushed sequence s's class-c tokens of the call, in call order,
+   * onto FIFO counters tail - cnt .. tail - 1 */
+  int32_t* next = (int32_t*)calloc((size_t)ns * 3, sizeof(int32_t));
+  for (int s = 0; s < ns; ++s)
+    for (int c = 0; c < 3; ++c)
+      next[s * 3 + c] = S->fifo_tail[s * 3 + c] - (int32_t)cnt[(size_t)s * 3 + c];
+  for (int32_t i = 0; i < n; ++i) {
+    int s = seq[i], c = tag[i];
+    int32_t idx = next[s * 3 + c]++;
+    int32_t ns_s = S->nseg[s];
+    if (ns_s > 0 && seg_rec(S, s, ns_s - 1)[SEG_CLS] == c) {
+      seg_rec(S, s, ns_s - 1)[SEG_LEN]++;
+      continue;
+    }
+    int32_t* g = seg_rec(S, s, ns_s);
+    g[SEG_CLS] = c;
+    g[SEG_LEVEL] = 0;
+    g[SEG_LO] = idx;
+    g[SEG_LEN] = 1;
+    g[SEG_TRIM] = 0;
+    S->nseg[s] = ns_s + 1;
+    if (c == OR_T) tbe_event(S, s, ns_s, t_min, schedule);
+  }
+  free(next);
+  free(cnt);
   return OR_OK;
 }
 
@@ -530,6 +689,28 @@ int or_decode(const or_state* S, int32_t n, const int32_t* seq, const uint16_t* 
 }
 
 /* ====================================================================== */
+/* thought decomposition from attention sparsity (mechanism only)          */
+/* ====================================================================== */
+/* Explainer, Methodologie, "Decomposition de la Pensee via la Parcimonie de
+ * l'Attention": thoughts are told apart by how sparse their attention is --
+ * Transition the sparsest, then Reasoning, Execution the least sparse.
+ * Reading: the sparsity of one decode step of sequence i is the mean over
+ * query heads of the top-k attention mass (a head whose probability sits on a
+ * few tokens has a mass near 1).  The mean is an fp32 sum in head order
+ * divided by the head count (both rounded to nearest), so that the tag -- an
+ * integer decided by floating point -- is reproducible exactly.  The two
+ * thresholds are the calibration the pages leave to a real model. */
+void or_classify(int32_t n, int32_t hq, const float* mass, float theta_t, float theta_r,
+                 uint8_t* tags) {
+  for (int32_t i = 0; i < n; ++i) {
+    float sum = 0.0f;
+    for (int32_t h = 0; h < hq; ++h) sum = sum + mass[(size_t)i * hq + h];
+    float score = sum / (float)hq;
+    tags[i] = score >= theta_t ? OR_T : (score >= theta_r ? OR_R : OR_E);
+  }
+}
+
+/* ====================================================================== */
 /* state export                                                            */
 /* ====================================================================== */
 const void* or_codes(const or_state* S, int c) { return S->codes[c]; }
@@ -547,3 +728,5 @@ const uint64_t* or_live_list(const or_state* S) { return S->live_list; }
 const int32_t* or_live_index(const or_state* S) { return S->live_index; }
 const int32_t* or_num_live(const or_state* S) { return S->num_live; }
 const int32_t* or_page_bump(const or_state* S) { return S->page_bump; }
+const int32_t* or_seg(const or_state* S) { return S->seg; }
+const int32_t* or_nseg(const or_state* S) { return S->nseg; }

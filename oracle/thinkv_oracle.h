@@ -58,6 +58,20 @@ int or_decode(const or_state* S, int32_t n, const int32_t* seq,
               double* out /* [n][Hq][d] */, double* mass /* [n][Hq] or NULL */,
               int32_t threads);
 
+/* TBE, segment-level eviction on Transition thoughts: called after or_append
+ * with the same token arrays.  Each new T segment anneals the earlier
+ * segments (R/E: keep schedule[level-1] tokens, level 1..3; T: keep the t_min
+ * most recent earlier T tokens); evicted FIFO entries become tombstones (-1).
+ * schedule: 3 retentions, NULL = {64, 32, 16}. */
+int or_tbe(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos, const uint8_t* tag,
+           int32_t t_min, const int32_t* schedule);
+
+/* Thought decomposition from attention sparsity (mechanism only): per
+ * sequence i, score = (sum over heads, in head order, of mass[i][h]) / hq in
+ * fp32; tag T if score >= theta_t, else R if score >= theta_r, else E. */
+void or_classify(int32_t n, int32_t hq, const float* mass, float theta_t, float theta_r,
+                 uint8_t* tags);
+
 /* ---- building blocks, exposed for the pin tests ---------------------- */
 uint16_t or_f16_round_down(float x);
 uint16_t or_f16_round_up(float x);
@@ -81,6 +95,10 @@ void or_quantize_group(const uint16_t* x, int32_t G, int32_t bits,
  *                of the entries with a non-zero mask (first num_live[s] valid)
  *   live_index : [max_seqs][max_blocks]               int32 position in live_list or -1
  *   page_bump : [3]                                   int32
+ *   seg        : [max_seqs][max_blocks*16][5]         int32 TBE segments:
+ *                class, level, lo (FIFO counter of the first token), len, trim
+ *   nseg       : [max_seqs]                           int32 segments per sequence
+ * A FIFO entry of -1 is a tombstone (evicted by TBE, not yet popped).
  */
 const void* or_codes(const or_state* S, int c);
 const uint16_t* or_params(const or_state* S, int c);
@@ -97,6 +115,8 @@ const uint64_t* or_live_list(const or_state* S);
 const int32_t* or_live_index(const or_state* S);
 const int32_t* or_num_live(const or_state* S);
 const int32_t* or_page_bump(const or_state* S);
+const int32_t* or_seg(const or_state* S);
+const int32_t* or_nseg(const or_state* S);
 
 #ifdef __cplusplus
 }

@@ -343,4 +343,5 @@ def check_slot_invariants(snap, ns):
             assert np.array_equal(mark, own.astype(np.int32)), f"free/live slots, seq {s} class {c}"
             h, t = int(snap["fifo_head"][s, c]), int(snap["fifo_tail"][s, c])
             win = snap["fifo"][s, c, np.arange(h, t) % cap]
+            win = win[win >= 0]                            # -1: tombstones of TBE evictions
             assert np.array_equal(np.sort(win), live_ids)

@@ -67,12 +67,14 @@ def test_noalloc_matches_workspace_decode_on_two_calls(name, topk):
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
+    """A call whose scratch need exceeds the fixed array is refused before
+    anything is launched (q and out are never touched, so small buffers do)."""
     from mixed_precision_paged_thinkv_b200 import binding, build
     build.build()
-    n = 4096
-    cache = binding.ThinKVCache(64, 8, 128, 64, (8, 4, 2), n, 1, (1, 1, 1))
+    n = 16384
+    cache = binding.ThinKVCache(2048, 256, 128, 64, (8, 4, 2), n, 1, (1, 1, 1))
     seqs = torch.arange(n, dtype=torch.int32, device="cuda")
-    q = torch.zeros(n, 64, 128, dtype=torch.float16, device="cuda")
+    q = torch.zeros(16, 128, dtype=torch.float16, device="cuda")
     out = torch.zeros_like(q)
     need = cache.decode_workspace_bytes(n, 0)
     assert need > binding_scratch_bytes()
