@@ -245,6 +245,56 @@ THINKV_API int thinkv_append_quantize(const thinkv_cache* cache, int32_t n_token
 THINKV_API int thinkv_evict(const thinkv_cache* cache, int32_t n_seqs, const int32_t* seq,
                  const int32_t* budget, const uint8_t* order, void* stream);
 
+/* TBE segment state of a cache (caller-owned device buffers, sizes from
+ * thinkv_tbe_buffer_bytes, cleared by thinkv_tbe_reset together with a
+ * thinkv_cache_reset of the cache):
+ *   seg      int32 [max_seqs][max_blocks_per_seq*16][4]  one record per
+ *            segment: class | level << 8, lo (FIFO counter of its first
+ *            token), len (tokens), trim (how far from lo TBE has evicted)
+ *   nseg     int32 [max_seqs]   segments recorded per sequence
+ *   settled  int32 [max_seqs]   segments before it no T event can change
+ *            any more (a speed-up: they are not visited again) */
+typedef struct {
+  int32_t* seg;
+  int32_t* nseg;
+  int32_t* settled;
+} thinkv_tbe;
+
+enum { THINKV_TBE_SEG = 0, THINKV_TBE_NSEG = 1, THINKV_TBE_SETTLED = 2, THINKV_TBE_NUM_BUFFERS = 3 };
+
+/* Bytes of TBE buffer `which` (THINKV_TBE_*); 0 for a bad layout or id. */
+THINKV_API size_t thinkv_tbe_buffer_bytes(const thinkv_layout* L, int32_t which);
+
+/* Empties the TBE state (no segments) on `stream`. */
+THINKV_API int thinkv_tbe_reset(const thinkv_layout* L, const thinkv_tbe* tbe, void* stream);
+
+/* Workspace bytes thinkv_evict_tbe needs for n_tokens tokens. */
+THINKV_API size_t thinkv_tbe_workspace_bytes(int32_t n_tokens);
+
+/* TBE: segment-level eviction on Transition thoughts (explainer, Resume
+ * Technique > Methodologie > "Eviction Adaptative a la Pensee (TBE)", and
+ * "Astuce B": a small safety net of Transition tokens is always kept).
+ * Call it right after thinkv_append_quantize with the same token arrays
+ * (n_tokens, seq, pos, tag).  Readings: a segment is a maximal run of
+ * consecutive tokens of a sequence with one tag; the first token of a new T
+ * segment is a T event.  At each T event, in call order, every earlier R or
+ * E segment takes the next step of `schedule` (its k-th event keeps at most
+ * schedule[min(k,3)-1] of its tokens) and the earlier T segments keep only
+ * the t_min most recent live T tokens among them.  A segment gives up its
+ * oldest tokens first; victims go in segment order, then token order: each
+ * one's live bit is cleared, its slot_pos set to -1, its slot pushed on its
+ * class's free stack (CT: refilled in place later), and its FIFO entry
+ * becomes a tombstone (-1) that thinkv_evict steps over.
+ * schedule: HOST array of 3 retentions >= 0, or NULL for {64, 32, 16};
+ * t_min >= 0.  Bad token data or a full segment table -> *status = INVALID
+ * and nothing changes; while *status != 0 the call does nothing.
+ * workspace: device, >= thinkv_tbe_workspace_bytes(n_tokens) bytes, no
+ * initialisation needed.  One kernel. */
+THINKV_API int thinkv_evict_tbe(const thinkv_cache* cache, const thinkv_tbe* tbe, int32_t n_tokens,
+                                const int32_t* seq, const int32_t* pos, const uint8_t* tag,
+                                int32_t t_min, const int32_t* schedule, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* Workspace bytes thinkv_decode_attention needs on the CURRENT device. */
 THINKV_API size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t n_seqs, int32_t topk);
 
@@ -300,6 +350,22 @@ THINKV_API int thinkv_decode_attention_noalloc(const thinkv_cache* cache, int32_
                                                const int32_t* seq, const uint16_t* q,
                                                uint16_t* out, float* topk_mass, int32_t topk,
                                                float softmax_scale, void* stream);
+
+/* Thought tags from attention sparsity (mechanism only).
+ * Explainer, Resume Technique > Methodologie > "Decomposition de la Pensee
+ * via la Parcimonie de l'Attention": Transition thoughts have the sparsest
+ * attention, then Reasoning, and Execution the least sparse.
+ * For each i < n: score = (mass[i][0] + mass[i][1] + ... + mass[i][hq-1]) /
+ * hq, the sum taken left to right and the division in fp32 (round to
+ * nearest); tags[i] = THINKV_T if score >= theta_t, else THINKV_R if
+ * score >= theta_r, else THINKV_E.
+ * mass: device fp32 [n][num_q_heads], e.g. the topk_mass output of
+ * thinkv_decode_attention; tags: device uint8 [n].  The thresholds are the
+ * calibration (the pages leave it to a real model); NaN thresholds or
+ * n < 0 or num_q_heads < 1 -> THINKV_ERR_INVALID.  One kernel, no state. */
+THINKV_API int thinkv_classify_thoughts(int32_t n, int32_t num_q_heads, const float* mass,
+                                        float theta_t, float theta_r, uint8_t* tags,
+                                        void* stream);
 
 /* Synchronises `stream`, then copies *status to *out (host). */
 THINKV_API int thinkv_get_status(const thinkv_cache* cache, void* stream, int32_t* out);

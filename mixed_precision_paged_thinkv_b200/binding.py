@@ -33,8 +33,11 @@ EXPORTED = [
     "thinkv_cache_reset", "thinkv_append_workspace_bytes", "thinkv_append_quantize",
     "thinkv_evict", "thinkv_decode_workspace_bytes", "thinkv_decode_attention",
     "thinkv_get_status", "thinkv_clear_status", "thinkv_status_string",
-    "thinkv_decode_attention_noalloc",
+    "thinkv_decode_attention_noalloc", "thinkv_classify_thoughts",
+    "thinkv_tbe_buffer_bytes", "thinkv_tbe_reset", "thinkv_tbe_workspace_bytes", "thinkv_evict_tbe",
 ]
+
+TBE_BUFFERS = ["seg", "nseg", "settled"]
 
 
 class ThinkvError(RuntimeError):
@@ -59,6 +62,10 @@ class CacheStruct(C.Structure):
                 ("live_count", C.c_void_p), ("live_list", C.c_void_p),
                 ("live_index", C.c_void_p), ("num_live", C.c_void_p),
                 ("page_bump", C.c_void_p), ("status", C.c_void_p)]
+
+
+class TbeStruct(C.Structure):
+    _fields_ = [("seg", C.c_void_p), ("nseg", C.c_void_p), ("settled", C.c_void_p)]
 
 
 _lock = threading.Lock()
@@ -98,6 +105,17 @@ def lib():
             L.thinkv_get_status.restype = C.c_int
             L.thinkv_clear_status.argtypes = [C.POINTER(CacheStruct), P]
             L.thinkv_clear_status.restype = C.c_int
+            L.thinkv_classify_thoughts.argtypes = [I32, I32, P, C.c_float, C.c_float, P, P]
+            L.thinkv_tbe_buffer_bytes.argtypes = [C.POINTER(Layout), I32]
+            L.thinkv_tbe_buffer_bytes.restype = SZ
+            L.thinkv_tbe_reset.argtypes = [C.POINTER(Layout), C.POINTER(TbeStruct), P]
+            L.thinkv_tbe_reset.restype = C.c_int
+            L.thinkv_tbe_workspace_bytes.argtypes = [I32]
+            L.thinkv_tbe_workspace_bytes.restype = SZ
+            L.thinkv_evict_tbe.argtypes = [C.POINTER(CacheStruct), C.POINTER(TbeStruct), I32, P, P, P,
+                                           I32, P, P, SZ, P]
+            L.thinkv_evict_tbe.restype = C.c_int
+            L.thinkv_classify_thoughts.restype = C.c_int
             L.thinkv_status_string.argtypes = [I32]
             L.thinkv_status_string.restype = C.c_char_p
             _lib = L
@@ -106,6 +124,19 @@ def lib():
 
 def status_string(code: int) -> str:
     return lib().thinkv_status_string(int(code)).decode()
+
+
+def classify_thoughts(mass: torch.Tensor, theta_t: float, theta_r: float,
+                      tags: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """R/E/T tags (uint8 [n]) from top-k attention masses (fp32 [n, Hq], device)."""
+    assert mass.dtype == torch.float32 and mass.dim() == 2 and mass.is_contiguous()
+    n, hq = mass.shape
+    if tags is None:
+        tags = torch.empty(n, dtype=torch.uint8, device=mass.device)
+    _check(lib().thinkv_classify_thoughts(int(n), int(hq), _ptr(mass), float(theta_t),
+                                          float(theta_r), _ptr(tags), _stream(stream)),
+           "classify_thoughts")
+    return tags
 
 
 def make_layout(num_q_heads, num_kv_heads, head_dim, group_size, bits, max_seqs,
@@ -138,7 +169,7 @@ class ThinKVCache:
 
     def __init__(self, num_q_heads: int, num_kv_heads: int, head_dim: int, group_size: int,
                  bits: Sequence[int], max_seqs: int, max_blocks_per_seq: int,
-                 pool_pages: Sequence[int], device: str = "cuda"):
+                 pool_pages: Sequence[int], device: str = "cuda", tbe: bool = False):
         self.layout = make_layout(num_q_heads, num_kv_heads, head_dim, group_size, bits,
                                   max_seqs, max_blocks_per_seq, pool_pages)
         L = lib()
@@ -161,6 +192,13 @@ class ThinKVCache:
         for name in BUFFERS[6:]:
             setattr(self.cs, name, _ptr(self.buf[name]))
         self._ws = {}
+        self.tbe = None
+        if tbe:
+            self.tbe_buf = {}
+            for i, name in enumerate(TBE_BUFFERS):
+                nbytes = int(L.thinkv_tbe_buffer_bytes(C.byref(self.layout), i))
+                self.tbe_buf[name] = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            self.tbe = TbeStruct(*[_ptr(self.tbe_buf[n]) for n in TBE_BUFFERS])
         self.reset()
 
     # -- helpers --
@@ -179,6 +217,23 @@ class ThinKVCache:
     # -- operations --
     def reset(self, stream=None):
         _check(lib().thinkv_cache_reset(C.byref(self.cs), _stream(stream)), "reset")
+        if self.tbe is not None:
+            _check(lib().thinkv_tbe_reset(C.byref(self.layout), C.byref(self.tbe), _stream(stream)),
+                   "tbe_reset")
+
+    def evict_tbe(self, seq: torch.Tensor, pos: torch.Tensor, tag: torch.Tensor, t_min: int = 0,
+                  schedule: Optional[Sequence[int]] = None, stream=None):
+        """TBE after an append of the same tokens (needs tbe=True)."""
+        assert self.tbe is not None, "cache created without TBE buffers"
+        n = int(seq.numel())
+        assert seq.dtype == torch.int32 and pos.dtype == torch.int32 and tag.dtype == torch.uint8
+        sch = None if schedule is None else (C.c_int32 * 3)(*[int(x) for x in schedule])
+        nbytes = int(lib().thinkv_tbe_workspace_bytes(n))
+        ws = self._workspace("tbe", nbytes)
+        _check(lib().thinkv_evict_tbe(C.byref(self.cs), C.byref(self.tbe), n, _ptr(seq), _ptr(pos),
+                                      _ptr(tag), int(t_min),
+                                      None if sch is None else C.cast(sch, C.c_void_p),
+                                      _ptr(ws), ws.numel(), _stream(stream)), "evict_tbe")
 
     def append(self, seq: torch.Tensor, pos: torch.Tensor, tag: torch.Tensor,
                k: torch.Tensor, v: torch.Tensor, stream=None):
@@ -261,6 +316,12 @@ class ThinKVCache:
             "slot_pos": [self._host(f"slot_pos_{n}", np.int32, (self.pool_pages[c], PAGE))
                          for c, n in enumerate("RET")],
         }
+        if self.tbe is not None:
+            seg = self.tbe_buf["seg"].cpu().numpy().view(np.int32).reshape(ns, cap, 4)
+            # (class | level << 8, lo, len, trim) -> (class, level, lo, len, trim)
+            st["seg"] = np.stack([seg[..., 0] & 0xFF, (seg[..., 0] >> 8) & 0xFF, seg[..., 1],
+                                  seg[..., 2], seg[..., 3]], axis=-1)
+            st["nseg"] = self.tbe_buf["nseg"].cpu().numpy().view(np.int32).copy()
         return st
 
     def pool_bytes(self, c: int) -> np.ndarray:

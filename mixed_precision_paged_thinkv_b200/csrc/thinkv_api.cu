@@ -4,6 +4,7 @@
 // handling; every operation itself runs in the kernels of thinkv_append.cu,
 // thinkv_evict.cu and thinkv_decode.cu.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
@@ -221,6 +222,56 @@ int thinkv_evict(const thinkv_cache* C, int32_t n, const int32_t* seq, const int
   return cuda_status(launch_evict(view_of(C), n, seq, budget, o, static_cast<cudaStream_t>(stream)));
 }
 
+size_t thinkv_tbe_buffer_bytes(const thinkv_layout* L, int32_t which) {
+  if (!layout_ok(L)) return 0;
+  const size_t ns = (size_t)L->max_seqs, cap = (size_t)L->max_blocks_per_seq * kPage;
+  switch (which) {
+    case THINKV_TBE_SEG: return ns * cap * 16;
+    case THINKV_TBE_NSEG: return ns * 4;
+    case THINKV_TBE_SETTLED: return ns * 4;
+    default: return 0;
+  }
+}
+
+static bool tbe_ok(const thinkv_tbe* T) {
+  return T && T->seg && T->nseg && T->settled && aligned(T->seg, 16) && aligned(T->nseg, 4) &&
+         aligned(T->settled, 4);
+}
+
+int thinkv_tbe_reset(const thinkv_layout* L, const thinkv_tbe* T, void* stream) {
+  if (!layout_ok(L) || !tbe_ok(T)) return THINKV_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(T->nseg, 0, thinkv_tbe_buffer_bytes(L, THINKV_TBE_NSEG), s);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(T->settled, 0, thinkv_tbe_buffer_bytes(L, THINKV_TBE_SETTLED), s);
+  return cuda_status(e);
+}
+
+size_t thinkv_tbe_workspace_bytes(int32_t n_tokens) {
+  if (n_tokens < 0) return 0;
+  return ((size_t)(n_tokens > 0 ? n_tokens : 1) * 4 + 255) / 256 * 256;
+}
+
+int thinkv_evict_tbe(const thinkv_cache* C, const thinkv_tbe* T, int32_t n, const int32_t* seq,
+                     const int32_t* pos, const uint8_t* tag, int32_t t_min, const int32_t* schedule,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cache_ok(C) || !tbe_ok(T) || n < 0 || t_min < 0) return THINKV_ERR_INVALID;
+  int32_t sch[3] = {64, 32, 16};
+  if (schedule) {
+    for (int k = 0; k < 3; ++k) {
+      if (schedule[k] < 0) return THINKV_ERR_INVALID;
+      sch[k] = schedule[k];
+    }
+  }
+  if (n == 0) return THINKV_OK;
+  if (!seq || !pos || !tag || !aligned(seq, 4) || !aligned(pos, 4)) return THINKV_ERR_INVALID;
+  if (workspace && !aligned(workspace, 16)) return THINKV_ERR_INVALID;
+  if (!workspace || workspace_bytes < thinkv_tbe_workspace_bytes(n)) return THINKV_ERR_WORKSPACE;
+  return cuda_status(launch_tbe(view_of(C), reinterpret_cast<int4*>(T->seg), T->nseg, T->settled, n,
+                                seq, pos, tag, t_min, sch, static_cast<int32_t*>(workspace),
+                                static_cast<cudaStream_t>(stream)));
+}
+
 size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t n_seqs, int32_t topk) {
   if (!layout_ok(L) || n_seqs < 1 || n_seqs > 16384 || topk < 0 || topk > 64) return 0;
   int dev = 0;
@@ -247,6 +298,16 @@ int thinkv_decode_attention(const thinkv_cache* C, int32_t n, const int32_t* seq
     return THINKV_ERR_WORKSPACE;
   return cuda_status(launch_decode(view_of(C), n, seq, q, out, topk_mass, topk_mass ? topk : 0,
                                    softmax_scale, workspace, dl, static_cast<cudaStream_t>(stream)));
+}
+
+int thinkv_classify_thoughts(int32_t n, int32_t num_q_heads, const float* mass, float theta_t,
+                             float theta_r, uint8_t* tags, void* stream) {
+  if (n < 0 || num_q_heads < 1) return THINKV_ERR_INVALID;
+  if (isnan(theta_t) || isnan(theta_r)) return THINKV_ERR_INVALID;
+  if (n == 0) return THINKV_OK;
+  if (!mass || !tags || !aligned(mass, 4)) return THINKV_ERR_INVALID;
+  return cuda_status(launch_classify(n, num_q_heads, mass, theta_t, theta_r, tags,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 int thinkv_get_status(const thinkv_cache* C, void* stream, int32_t* out) {

@@ -6,13 +6,14 @@
 // only marked in the block table's eviction mask and becomes reusable by the
 // next token of its thought type -- nothing is moved or compacted.
 //
-// One CTA.  The call is validated first (sequence range, duplicates, budget
-// sign; all-or-nothing), then one warp per sequence takes its victims from the
-// class FIFO heads in `order`, 32 at a time: slot ids are read coalesced, the
-// bits of victims sharing a table entry are merged with __match_any_sync, an
-// entry that loses its last live token leaves the live-page list (in victim
-// order, by swap-with-last), and the victims are pushed on their class's free
-// stack in victim order.  Each sequence's state is touched by one warp only.
+// The call is validated first (sequence range, duplicates, budget sign;
+// all-or-nothing), then one warp per sequence takes its victims from the
+// class FIFO heads in `order`, 32 at a time: slot ids are read coalesced,
+// tombstones left by TBE are stepped over, the bits of victims sharing a table
+// entry are merged with __match_any_sync, an entry that loses its last live
+// token leaves the live-page list (in victim order, by swap-with-last), and
+// the victims are pushed on their class's free stack in victim order.  Each
+// sequence's state is touched by one warp only.
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
@@ -25,18 +26,17 @@ namespace {
 constexpr int kEvictThreads = 1024;
 constexpr int kEvictWarps = kEvictThreads / 32;
 
-struct Order {
-  uint8_t c[4];
-};
+__device__ void evict_seq(const CacheView& C, int s, int bud, uint32_t order, bool check_status);
 
+// Calls of any size: one CTA validates the call (all-or-nothing), then a warp
+// per sequence evicts it (evict_seq).
 __global__ void __launch_bounds__(kEvictThreads, 1)
     evict_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
-                 const int32_t* __restrict__ budget, Order order) {
+                 const int32_t* __restrict__ budget, uint32_t order) {
   extern __shared__ uint32_t seen[];  // max_seqs bits
   __shared__ int s_err;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int max_seqs = C.L.max_seqs, nb_max = C.L.max_blocks_per_seq;
-  const int64_t cap = (int64_t)nb_max * kPage;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int max_seqs = C.L.max_seqs;
   if (tid == 0) s_err = (*C.status != 0) ? -1 : 0;
   for (int i = tid; i < (max_seqs + 31) / 32; i += kEvictThreads) seen[i] = 0;
   __syncthreads();
@@ -55,81 +55,7 @@ __global__ void __launch_bounds__(kEvictThreads, 1)
     if (tid == 0) set_status(C.status, s_err);
     return;
   }
-
-  for (int i = warp; i < n; i += kEvictWarps) {
-    const int s = seq[i];
-    int remaining = C.live_count[s] - budget[i];
-    if (remaining <= 0) continue;
-    uint64_t* table = C.block_table + (int64_t)s * nb_max;
-    uint64_t* llist = C.live_list + (int64_t)s * nb_max;
-    int32_t* lidx = C.live_index + (int64_t)s * nb_max;
-    int nlive = C.num_live[s];
-    int evicted = 0;
-    for (int o = 0; o < 3 && remaining > 0; ++o) {
-      const int c = order.c[o];
-      const int head = C.fifo_head[s * 3 + c];
-      const int avail = C.fifo_tail[s * 3 + c] - head;
-      const int take = min(avail, remaining);
-      if (take <= 0) continue;
-      const int32_t* ring = C.fifo + ((int64_t)s * 3 + c) * cap;
-      int32_t* stack = C.free_slots + ((int64_t)s * 3 + c) * cap;
-      const int top = C.free_top[s * 3 + c];
-      for (int v0 = 0; v0 < take; v0 += 32) {
-        const int v = v0 + lane;
-        const bool valid = v < take;
-        int32_t ts = valid ? ring[((int64_t)head + v) % cap] : 0;
-        const int e = ts >> 4, slot = ts & 15;
-        // merge the bits of victims that share an entry; the highest such lane
-        // is the last victim of that entry in this batch
-        const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? e : -1 - lane);
-        const uint32_t mybit = valid ? (1u << slot) : 0u;
-        const uint32_t bits = __reduce_or_sync(grp, mybit);
-        const bool last = valid && (31 - __clz(grp)) == lane;
-        bool emptied = false;
-        uint32_t page = 0;
-        if (valid) {
-          uint64_t ent = table[e];
-          page = entry_page(ent);
-          if (last) {
-            uint32_t mask = entry_mask(ent) & ~bits;
-            table[e] = (ent & 0x0000FFFFFFFFFFFFull) | ((uint64_t)mask << 48);
-            emptied = (mask == 0);
-          }
-          C.slot_pos[c][(int64_t)page * kPage + slot] = -1;
-          stack[top + v] = ts;
-        }
-        // entries emptied in this batch leave the live list in victim order
-        unsigned ev = __ballot_sync(0xFFFFFFFFu, emptied);
-        __syncwarp();
-        while (ev) {
-          const int src = __ffs(ev) - 1;
-          const int ee = __shfl_sync(0xFFFFFFFFu, e, src);
-          if (lane == 0) {
-            const int at = lidx[ee];
-            const int lastpos = --nlive;
-            const uint64_t moved = llist[lastpos];
-            llist[at] = moved;
-            lidx[live_desc_entry(moved)] = at;
-            lidx[ee] = -1;
-          }
-          nlive = __shfl_sync(0xFFFFFFFFu, nlive, 0);
-          __syncwarp();
-          ev &= ev - 1;
-        }
-      }
-      if (lane == 0) {
-        C.fifo_head[s * 3 + c] = head + take;
-        C.free_top[s * 3 + c] = top + take;
-      }
-      remaining -= take;
-      evicted += take;
-    }
-    if (lane == 0) {
-      C.live_count[s] -= evicted;
-      C.num_live[s] = nlive;
-    }
-    __syncwarp();
-  }
+  for (int i = warp; i < n; i += kEvictWarps) evict_seq(C, seq[i], budget[i], order, false);
 }
 
 
@@ -145,10 +71,13 @@ constexpr int kSmallEvictWarps = kSmallEvictThreads / 32;
 
 // Evicts sequence s down to `bud` live tokens (one warp).  The class order is
 // packed one class per byte.  All of s's counters are loaded at once (with
-// the sticky status when check_status: a set status makes this a no-op); the
-// victims of all classes are then taken 32 at a time in victim order.
+// the sticky status when check_status: a set status makes this a no-op).
+// Victims are the oldest live entries of the first class in order that has
+// one, then the next class: each class FIFO is scanned from its head 32
+// entries at a time; -1 entries are tombstones (tokens TBE evicted away from
+// the head), stepped over and consumed like the victims before them.
 __device__ void evict_seq(const CacheView& C, int s, int bud, uint32_t order,
-                          bool check_status = false) {
+                          bool check_status) {
   const int lane = threadIdx.x & 31;
   const int nb_max = C.L.max_blocks_per_seq;
   const int64_t cap = (int64_t)nb_max * kPage;
@@ -169,73 +98,79 @@ __device__ void evict_seq(const CacheView& C, int s, int bud, uint32_t order,
   int nlive = __shfl_sync(0xFFFFFFFFu, val, 10);
   int remaining = live - bud;
   if (remaining <= 0) return;
-  int head[3], take[3], top[3], cum[3];
-  int total = 0;
-#pragma unroll
-  for (int o = 0; o < 3; ++o) {
-    head[o] = __shfl_sync(0xFFFFFFFFu, val, o);
-    const int tail = __shfl_sync(0xFFFFFFFFu, val, 3 + o);
-    top[o] = __shfl_sync(0xFFFFFFFFu, val, 6 + o);
-    take[o] = min(max(tail - head[o], 0), remaining);
-    remaining -= take[o];
-    total += take[o];
-    cum[o] = total;                                  // victims of classes 0..o
-  }
   uint64_t* table = C.block_table + (int64_t)s * nb_max;
   uint64_t* llist = C.live_list + (int64_t)s * nb_max;
   int32_t* lidx = C.live_index + (int64_t)s * nb_max;
-  for (int v0 = 0; v0 < total; v0 += 32) {
-    const int vv = v0 + lane;
-    const bool valid = vv < total;
-    const int o = vv < cum[0] ? 0 : (vv < cum[1] ? 1 : 2);
+  int total = 0;
+  int new_head = 0, new_top = 0;                     // lane o < 3 keeps class o's values
+  for (int o = 0; o < 3; ++o) {
     const int c = (int)((order >> (8 * o)) & 0xFFu);
-    const int r = vv - (o == 0 ? 0 : (o == 1 ? cum[0] : cum[1]));   // rank inside the class
-    const int hd = o == 0 ? head[0] : (o == 1 ? head[1] : head[2]);
-    const int tp = o == 0 ? top[0] : (o == 1 ? top[1] : top[2]);
-    int32_t ts = 0;
-    if (valid) ts = C.fifo[((int64_t)s * 3 + c) * cap + ((int64_t)hd + r) % cap];
-    const int e = ts >> 4, slot = ts & 15;
-    // merge the bits of victims that share an entry (entries are class-pure);
-    // the highest such lane writes the entry
-    const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? e : -1 - lane);
-    const uint32_t bits = __reduce_or_sync(grp, valid ? (1u << slot) : 0u);
-    const bool last = valid && (31 - __clz(grp)) == lane;
-    bool emptied = false;
-    if (valid) {
-      // through L2: an earlier batch may have rewritten this entry
-      const uint64_t ent = __ldcg(&table[e]);
-      const uint32_t page = entry_page(ent);
-      if (last) {
-        const uint32_t mask = entry_mask(ent) & ~bits;
-        table[e] = (ent & 0x0000FFFFFFFFFFFFull) | ((uint64_t)mask << 48);
-        emptied = (mask == 0);
+    int idx = __shfl_sync(0xFFFFFFFFu, val, o);
+    const int tail = __shfl_sync(0xFFFFFFFFu, val, 3 + o);
+    int top = __shfl_sync(0xFFFFFFFFu, val, 6 + o);
+    const int32_t* ring = C.fifo + ((int64_t)s * 3 + c) * cap;
+    int32_t* stack = C.free_slots + ((int64_t)s * 3 + c) * cap;
+    while (remaining > 0 && idx < tail) {
+      const int cnt = min(32, tail - idx);
+      const int32_t ts = lane < cnt ? ring[((int64_t)idx + lane) % cap] : -1;
+      const unsigned lbal = __ballot_sync(0xFFFFFFFFu, ts >= 0);
+      const int rank = __popc(lbal & ((1u << lane) - 1u));
+      const bool valid = ts >= 0 && rank < remaining;
+      const unsigned vbal = __ballot_sync(0xFFFFFFFFu, valid);
+      const int nv = __popc(vbal);
+      // the quota reached: consumed up to the last victim; else the whole chunk
+      const int consumed = (nv == remaining) ? 32 - __clz(vbal) : cnt;
+      const int e = valid ? (ts >> 4) : -1, slot = ts & 15;
+      // merge the bits of victims that share an entry (entries are class-pure);
+      // the highest such lane writes the entry
+      const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? e : -1 - lane);
+      const uint32_t bits = __reduce_or_sync(grp, valid ? (1u << slot) : 0u);
+      const bool last = valid && (31 - __clz(grp)) == lane;
+      bool emptied = false;
+      if (valid) {
+        // through L2: an earlier batch may have rewritten this entry
+        const uint64_t ent = __ldcg(&table[e]);
+        const uint32_t page = entry_page(ent);
+        if (last) {
+          const uint32_t mask = entry_mask(ent) & ~bits;
+          table[e] = (ent & 0x0000FFFFFFFFFFFFull) | ((uint64_t)mask << 48);
+          emptied = (mask == 0);
+        }
+        C.slot_pos[c][(int64_t)page * kPage + slot] = -1;
+        stack[top + rank] = ts;
       }
-      C.slot_pos[c][(int64_t)page * kPage + slot] = -1;
-      C.free_slots[((int64_t)s * 3 + c) * cap + tp + r] = ts;
-    }
-    // entries emptied in this batch leave the live list in victim order
-    unsigned ev = __ballot_sync(0xFFFFFFFFu, emptied);
-    __syncwarp();
-    while (ev) {
-      const int src = __ffs(ev) - 1;
-      const int ee = __shfl_sync(0xFFFFFFFFu, e, src);
-      if (lane == 0) {
-        const int lastpos = nlive - 1;
-        const int at = __ldcg(&lidx[ee]);
-        const uint64_t moved = __ldcg(&llist[lastpos]);
-        llist[at] = moved;
-        lidx[live_desc_entry(moved)] = at;
-        lidx[ee] = -1;
-      }
-      --nlive;
+      // entries emptied in this batch leave the live list in victim order
+      unsigned ev = __ballot_sync(0xFFFFFFFFu, emptied);
       __syncwarp();
-      ev &= ev - 1;
+      while (ev) {
+        const int src = __ffs(ev) - 1;
+        const int ee = __shfl_sync(0xFFFFFFFFu, e, src);
+        if (lane == 0) {
+          const int lastpos = nlive - 1;
+          const int at = __ldcg(&lidx[ee]);
+          const uint64_t moved = __ldcg(&llist[lastpos]);
+          llist[at] = moved;
+          lidx[live_desc_entry(moved)] = at;
+          lidx[ee] = -1;
+        }
+        --nlive;
+        __syncwarp();
+        ev &= ev - 1;
+      }
+      top += nv;
+      remaining -= nv;
+      total += nv;
+      idx += consumed;
+    }
+    if (lane == o) {
+      new_head = idx;
+      new_top = top;
     }
   }
   if (lane < 3) {
     const int c = (int)((order >> (8 * lane)) & 0xFFu);
-    C.fifo_head[s * 3 + c] = head[lane == 0 ? 0 : (lane == 1 ? 1 : 2)] + take[lane == 0 ? 0 : (lane == 1 ? 1 : 2)];
-    C.free_top[s * 3 + c] = top[lane == 0 ? 0 : (lane == 1 ? 1 : 2)] + take[lane == 0 ? 0 : (lane == 1 ? 1 : 2)];
+    C.fifo_head[s * 3 + c] = new_head;
+    C.free_top[s * 3 + c] = new_top;
   }
   if (lane == 0) {
     C.live_count[s] = live - total;
@@ -284,19 +219,14 @@ __global__ void __launch_bounds__(kSmallEvictThreads)
 
 cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
                          const uint8_t order[3], cudaStream_t stream) {
-  Order o;
-  o.c[0] = order[0];
-  o.c[1] = order[1];
-  o.c[2] = order[2];
-  o.c[3] = 0;
+  const uint32_t packed = (uint32_t)order[0] | ((uint32_t)order[1] << 8) | ((uint32_t)order[2] << 16);
   const size_t seen_bytes = (size_t)((C.L.max_seqs + 31) / 32) * 4;
   if (n <= kSmallEvict) {
-    const uint32_t packed = (uint32_t)order[0] | ((uint32_t)order[1] << 8) | ((uint32_t)order[2] << 16);
     const int grid = (n + kSmallEvictWarps - 1) / kSmallEvictWarps;
     return launch_pdl(evict_small_kernel, dim3(grid), dim3(kSmallEvictThreads), seen_bytes, stream,
                       C, n, seq, budget, packed);
   }
-  evict_kernel<<<1, kEvictThreads, seen_bytes, stream>>>(C, n, seq, budget, o);
+  evict_kernel<<<1, kEvictThreads, seen_bytes, stream>>>(C, n, seq, budget, packed);
   return cudaGetLastError();
 }
 

@@ -87,4 +87,13 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
                           uint16_t* out, float* mass, int32_t topk, float softmax_scale,
                           void* ws, const DecodeLaunch& dl, cudaStream_t stream);
 
+// TBE (segment-level eviction on Transition thoughts)
+cudaError_t launch_tbe(const CacheView& C, int4* seg, int32_t* nseg, int32_t* settled, int32_t n,
+                       const int32_t* seq, const int32_t* pos, const uint8_t* tag, int32_t t_min,
+                       const int32_t schedule[3], int32_t* run_start, cudaStream_t stream);
+
+// thought classifier (mechanism only)
+cudaError_t launch_classify(int32_t n, int32_t hq, const float* mass, float theta_t, float theta_r,
+                            uint8_t* tags, cudaStream_t stream);
+
 }  // namespace thinkv

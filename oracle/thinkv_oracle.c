@@ -544,8 +544,13 @@ int or_tbe(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos, const
                                : tag[i - 1];
     if (tag[i] != last_cls) newseg[s]++;
   }
-  for (int s = 0; s < ns && !bad; ++s)
+  for (int s = 0; s < ns && !bad; ++s) {
     if ((int64_t)S->nseg[s] + newseg[s] > S->cap) bad = 1;
+    /* the tokens must be the newest of their class FIFOs: the append that
+     * precedes this call put them there */
+    for (int c = 0; c < 3; ++c)
+      if (cnt[(size_t)s * 3 + c] > S->fifo_tail[s * 3 + c] - S->fifo_head[s * 3 + c]) bad = 1;
+  }
   free(seen);
   free(newseg);
   if (bad) { free(cnt); return OR_ERR_INVALID; }

@@ -161,3 +161,14 @@ def test_misaligned_pointers_rejected_without_launch(lib):
     cs.block_table = 4096
     cs.num_live = 4096 + 2
     assert lib.thinkv_cache_reset(C.byref(cs), None) == 1
+
+
+def test_classify_host_validation(lib):
+    ok = C.c_void_p(4096)
+    f = lib.thinkv_classify_thoughts
+    assert f(-1, 4, ok, C.c_float(0.5), C.c_float(0.2), ok, None) == 1
+    assert f(4, 0, ok, C.c_float(0.5), C.c_float(0.2), ok, None) == 1
+    assert f(4, 4, ok, C.c_float(float("nan")), C.c_float(0.2), ok, None) == 1
+    assert f(4, 4, None, C.c_float(0.5), C.c_float(0.2), ok, None) == 1
+    assert f(4, 4, C.c_void_p(4098), C.c_float(0.5), C.c_float(0.2), ok, None) == 1
+    assert f(0, 4, None, C.c_float(0.5), C.c_float(0.2), None, None) == 0

@@ -228,3 +228,18 @@ def test_tbe_rejects_bad_calls_and_changes_nothing():
             assert all(np.array_equal(a, b) for a, b in zip(before[key], after[key]))
         else:
             assert np.array_equal(before[key], after[key]), key
+
+
+def test_tbe_rejects_tokens_the_append_did_not_store():
+    """Class counts that exceed what the FIFOs hold: the call did not follow
+    an append of these tokens; rejected, nothing changes."""
+    o = O.Oracle(2, 1, 64, 32, (8, 4, 2), 1, 4, (4, 4, 4))
+    k, v = _kv(4, 1, 64, 2)
+    seq = np.zeros(2, np.int32)
+    assert o.append(seq, np.arange(2, dtype=np.int32), np.array([0, 0], np.uint8), k[:2], v[:2]) == O.OK
+    before = o.state()
+    assert o.tbe(np.zeros(3, np.int32), np.arange(3, dtype=np.int32),
+                 np.array([0, 0, 0], np.uint8)) == O.ERR_INVALID
+    assert o.tbe(seq, np.arange(2, dtype=np.int32), np.array([2, 2], np.uint8)) == O.ERR_INVALID
+    after = o.state()
+    assert np.array_equal(before["nseg"], after["nseg"])
