@@ -295,6 +295,33 @@ THINKV_API int thinkv_evict_tbe(const thinkv_cache* cache, const thinkv_tbe* tbe
                                 int32_t t_min, const int32_t* schedule, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Workspace bytes thinkv_compact needs for n_seqs sequences holding at most
+ * max_tokens live tokens together. */
+THINKV_API size_t thinkv_compact_workspace_bytes(int32_t n_seqs, int32_t max_tokens);
+
+/* Gather compaction: the step Continuous Thinking avoids, as a baseline to
+ * measure it by (explainer, Methodologie, "Implementation Systeme: Pensee
+ * Continue (CT)": evicting scattered tokens leaves holes that a gather-based
+ * compaction would close at a cost in time and HBM bandwidth; CT refills them
+ * in place; Resultats: the TPOT gain comes mainly from not compacting).
+ * The live tokens of seq[0..n_seqs) (distinct) in `src` move into fresh,
+ * hole-free pages of `dst`, a cache of the same geometry (pool sizes may
+ * differ) that holds nothing yet for those sequences: class by class (R, E,
+ * T), FIFO order within a class, 16 to a page, codes and params copied (not
+ * requantised), as if appended there in that order.  The last page of a class
+ * keeps its unused slots on the free stack; src's tombstones and free slots
+ * are not carried over; pages are granted in call order per class.  src is
+ * only read.  Decode over dst gives the same attention as over src.
+ * max_tokens: an upper bound of the live tokens of the listed sequences (a
+ * larger count sets dst's *status = INVALID).  A non-empty dst sequence or a
+ * repeated/out-of-range id -> INVALID, an exhausted dst pool -> OUT_OF_PAGES,
+ * both in dst's status with nothing changed.  workspace: device, >=
+ * thinkv_compact_workspace_bytes(n_seqs, max_tokens), no initialisation.
+ * Two kernels: the assignment (one CTA) and the copy (a warp per page-head). */
+THINKV_API int thinkv_compact(const thinkv_cache* src, const thinkv_cache* dst, int32_t n_seqs,
+                              const int32_t* seq, int32_t max_tokens, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* Workspace bytes thinkv_decode_attention needs on the CURRENT device. */
 THINKV_API size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t n_seqs, int32_t topk);
 

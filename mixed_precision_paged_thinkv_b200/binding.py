@@ -35,6 +35,7 @@ EXPORTED = [
     "thinkv_get_status", "thinkv_clear_status", "thinkv_status_string",
     "thinkv_decode_attention_noalloc", "thinkv_classify_thoughts",
     "thinkv_tbe_buffer_bytes", "thinkv_tbe_reset", "thinkv_tbe_workspace_bytes", "thinkv_evict_tbe",
+    "thinkv_compact_workspace_bytes", "thinkv_compact",
 ]
 
 TBE_BUFFERS = ["seg", "nseg", "settled"]
@@ -115,6 +116,11 @@ def lib():
             L.thinkv_evict_tbe.argtypes = [C.POINTER(CacheStruct), C.POINTER(TbeStruct), I32, P, P, P,
                                            I32, P, P, SZ, P]
             L.thinkv_evict_tbe.restype = C.c_int
+            L.thinkv_compact_workspace_bytes.argtypes = [I32, I32]
+            L.thinkv_compact_workspace_bytes.restype = SZ
+            L.thinkv_compact.argtypes = [C.POINTER(CacheStruct), C.POINTER(CacheStruct), I32, P, I32,
+                                         P, SZ, P]
+            L.thinkv_compact.restype = C.c_int
             L.thinkv_classify_thoughts.restype = C.c_int
             L.thinkv_status_string.argtypes = [I32]
             L.thinkv_status_string.restype = C.c_char_p
@@ -259,6 +265,16 @@ class ThinKVCache:
         _check(lib().thinkv_evict(C.byref(self.cs), n, _ptr(seq), _ptr(budget),
                                   None if o is None else C.cast(o, C.c_void_p),
                                   _stream(stream)), "evict")
+
+    def compact_into(self, dst: "ThinKVCache", seq: torch.Tensor, max_tokens: int, stream=None):
+        """Gather compaction of `seq`'s live tokens into the empty cache `dst`."""
+        n = int(seq.numel())
+        assert seq.dtype == torch.int32
+        nbytes = int(lib().thinkv_compact_workspace_bytes(n, int(max_tokens)))
+        ws = self._workspace("compact", nbytes)
+        _check(lib().thinkv_compact(C.byref(self.cs), C.byref(dst.cs), n, _ptr(seq),
+                                    int(max_tokens), _ptr(ws), ws.numel(), _stream(stream)),
+               "compact")
 
     def decode_workspace_bytes(self, n: int, topk: int = 0) -> int:
         return int(lib().thinkv_decode_workspace_bytes(C.byref(self.layout), n, topk))

@@ -15,7 +15,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libthinkv.so")
 SOURCES = ["thinkv_api.cu", "thinkv_append.cu", "thinkv_evict.cu", "thinkv_decode.cu",
-           "thinkv_noalloc.cu", "thinkv_classify.cu", "thinkv_tbe.cu"]
+           "thinkv_noalloc.cu", "thinkv_classify.cu", "thinkv_tbe.cu",
+           "thinkv_compact.cu"]
 HEADERS = ["thinkv_common.cuh", "thinkv_internal.h"]
 
 NVCC_FLAGS = [

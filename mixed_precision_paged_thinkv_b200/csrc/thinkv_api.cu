@@ -272,6 +272,30 @@ int thinkv_evict_tbe(const thinkv_cache* C, const thinkv_tbe* T, int32_t n, cons
                                 static_cast<cudaStream_t>(stream)));
 }
 
+size_t thinkv_compact_workspace_bytes(int32_t n_seqs, int32_t max_tokens) {
+  if (n_seqs < 0 || max_tokens < 0) return 0;
+  return compact_workspace_bytes(n_seqs, max_tokens);
+}
+
+int thinkv_compact(const thinkv_cache* src, const thinkv_cache* dst, int32_t n, const int32_t* seq,
+                   int32_t max_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cache_ok(src) || !cache_ok(dst) || n < 0 || max_tokens < 0) return THINKV_ERR_INVALID;
+  const thinkv_layout &A = src->L, &B = dst->L;
+  if (A.num_q_heads != B.num_q_heads || A.num_kv_heads != B.num_kv_heads ||
+      A.head_dim != B.head_dim || A.group_size != B.group_size || A.bits[0] != B.bits[0] ||
+      A.bits[1] != B.bits[1] || A.bits[2] != B.bits[2] || A.max_seqs != B.max_seqs ||
+      A.max_blocks_per_seq != B.max_blocks_per_seq || n > A.max_seqs)
+    return THINKV_ERR_INVALID;
+  if (n == 0) return THINKV_OK;
+  if (!seq || !aligned(seq, 4)) return THINKV_ERR_INVALID;
+  if (workspace && !aligned(workspace, 16)) return THINKV_ERR_INVALID;
+  if (!workspace || workspace_bytes < compact_workspace_bytes(n, max_tokens)) return THINKV_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return THINKV_ERR_CUDA;
+  return cuda_status(launch_compact(view_of(src), view_of(dst), n, seq, max_tokens, workspace, sms,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
 size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t n_seqs, int32_t topk) {
   if (!layout_ok(L) || n_seqs < 1 || n_seqs > 16384 || topk < 0 || topk > 64) return 0;
   int dev = 0;

@@ -74,6 +74,7 @@ def lib():
             L.or_quantize_group.argtypes = [P, C.c_int32, C.c_int32, P, P, P]
             L.or_classify.argtypes = [C.c_int32, C.c_int32, P, C.c_float, C.c_float, P]
             L.or_tbe.argtypes = [P, C.c_int32, P, P, P, C.c_int32, P]
+            L.or_compact.argtypes = [P, P, C.c_int32, P]
             for f in ("or_codes", "or_params", "or_slot_pos"):
                 getattr(L, f).argtypes = [P, C.c_int]
                 getattr(L, f).restype = P
@@ -199,6 +200,11 @@ class Oracle:
         sch = None if schedule is None else np.ascontiguousarray(schedule, dtype=np.int32)
         return int(lib().or_tbe(self._h, seq.shape[0], _ptr(seq), _ptr(pos), _ptr(tag),
                                 int(t_min), None if sch is None else _ptr(sch)))
+
+    def compact_into(self, dst: "Oracle", seq) -> int:
+        """Gather the live tokens of `seq` into the empty oracle `dst` (see or_compact)."""
+        seq = np.ascontiguousarray(seq, dtype=np.int32)
+        return int(lib().or_compact(self._h, dst._h, seq.shape[0], _ptr(seq)))
 
     def decode(self, seq, q, softmax_scale: float = 0.0, topk: Optional[int] = None,
                threads: int = 1):

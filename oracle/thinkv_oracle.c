@@ -583,6 +583,103 @@ int or_tbe(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos, const
 }
 
 /* ====================================================================== */
+/* gather compaction: the step CT avoids                                   */
+/* ====================================================================== */
+/* Explainer, Methodologie, "Implementation Systeme: Pensee Continue (CT)":
+ * without CT, evicting scattered tokens leaves holes that a gather-based
+ * compaction closes by moving the survivors together (at a cost in time and
+ * HBM bandwidth); CT instead refills the holes in place.  Reading of the
+ * compaction the pages compare against: each listed sequence's live tokens
+ * are gathered into fresh, hole-free pages of an empty cache dst of the same
+ * geometry -- class by class (R, E, T), in FIFO (arrival) order within a
+ * class, 16 to a page -- as if they were appended there in that order with
+ * their codes copied, not requantised.  The last page of a class keeps its
+ * unused slots on the free stack, as an append leaves them.  Tombstones and
+ * free slots are not carried over.  A token keeps its sequence id and
+ * position; dst's pages are granted in call order. */
+static void copy_token(const or_state* src, int c, int32_t sp, int ss, or_state* dst,
+                       int32_t dp, int ds) {
+  const or_layout* L = &src->L;
+  size_t rows = (size_t)L->num_kv_heads * 2, d = (size_t)L->head_dim;
+  size_t ng = (size_t)(L->head_dim / L->group_size);
+  for (size_t hk = 0; hk < rows; ++hk) {           /* (head, K|V) rows */
+    size_t a = (((size_t)sp * rows + hk) * OR_PAGE + ss), b = (((size_t)dp * rows + hk) * OR_PAGE + ds);
+    if (L->bits[c] == 16) {
+      memcpy((uint16_t*)dst->codes[c] + b * d, (const uint16_t*)src->codes[c] + a * d, d * 2);
+    } else {
+      memcpy((uint8_t*)dst->codes[c] + b * d, (const uint8_t*)src->codes[c] + a * d, d);
+      memcpy(dst->params[c] + b * ng * 2, src->params[c] + a * ng * 2, ng * 4);
+    }
+  }
+}
+
+int or_compact(const or_state* src, or_state* dst, int32_t n, const int32_t* seq) {
+  const or_layout* A = &src->L;
+  const or_layout* B = &dst->L;
+  if (n < 0) return OR_ERR_INVALID;
+  if (A->num_q_heads != B->num_q_heads || A->num_kv_heads != B->num_kv_heads ||
+      A->head_dim != B->head_dim || A->group_size != B->group_size ||
+      A->bits[0] != B->bits[0] || A->bits[1] != B->bits[1] || A->bits[2] != B->bits[2] ||
+      A->max_seqs != B->max_seqs || A->max_blocks_per_seq != B->max_blocks_per_seq)
+    return OR_ERR_INVALID;
+  char* seen = (char*)calloc((size_t)A->max_seqs, 1);
+  int64_t need[3] = {0, 0, 0};
+  int bad = 0;
+  for (int32_t i = 0; i < n && !bad; ++i) {
+    int s = seq[i];
+    if (s < 0 || s >= A->max_seqs || seen[s]) { bad = 1; break; }
+    seen[s] = 1;
+    if (dst->num_blocks[s] != 0) bad = 1;        /* dst must be empty for s */
+    for (int c = 0; c < 3; ++c) {
+      int64_t live = 0;
+      for (int32_t k = src->fifo_head[s * 3 + c]; k < src->fifo_tail[s * 3 + c]; ++k)
+        if (src->fifo[((size_t)s * 3 + c) * src->cap + (size_t)(k % src->cap)] >= 0) ++live;
+      need[c] += (live + OR_PAGE - 1) / OR_PAGE;
+    }
+  }
+  free(seen);
+  for (int c = 0; c < 3 && !bad; ++c)
+    if (need[c] > (int64_t)B->pool_pages[c] - dst->page_bump[c]) return OR_ERR_OUT_OF_PAGES;
+  if (bad) return OR_ERR_INVALID;
+  for (int32_t i = 0; i < n; ++i) {
+    int s = seq[i];
+    for (int c = 0; c < 3; ++c) {
+      int32_t used = OR_PAGE, e = -1, page = -1;
+      for (int32_t k = src->fifo_head[s * 3 + c]; k < src->fifo_tail[s * 3 + c]; ++k) {
+        int32_t ts = src->fifo[((size_t)s * 3 + c) * src->cap + (size_t)(k % src->cap)];
+        if (ts < 0) continue;                    /* tombstone */
+        int32_t se = ts / OR_PAGE, ss = ts % OR_PAGE;
+        int32_t sp = ENTRY_PAGE(table_row(src, s)[se]);
+        if (used == OR_PAGE) {                   /* a fresh page of class c */
+          page = dst->page_bump[c]++;
+          e = dst->num_blocks[s]++;
+          table_row(dst, s)[e] = (uint64_t)(uint32_t)page | ((uint64_t)c << 32);
+          for (int sl = 0; sl < OR_PAGE; ++sl) dst->slot_pos[c][(size_t)page * OR_PAGE + sl] = -1;
+          int32_t at = dst->num_live[s]++;
+          dst->live_list[(size_t)s * B->max_blocks_per_seq + at] = live_desc(page, c, e);
+          dst->live_index[(size_t)s * B->max_blocks_per_seq + e] = at;
+          used = 0;
+        }
+        int32_t slot = used++;
+        copy_token(src, c, sp, ss, dst, page, slot);
+        table_row(dst, s)[e] |= (uint64_t)1 << (48 + slot);
+        dst->slot_pos[c][(size_t)page * OR_PAGE + slot] =
+            src->slot_pos[c][(size_t)sp * OR_PAGE + ss];
+        int32_t* tail = &dst->fifo_tail[s * 3 + c];
+        fifo_ring(dst, s, c)[(*tail) % dst->cap] = e * OR_PAGE + slot;
+        (*tail)++;
+        dst->live_count[s]++;
+      }
+      /* the unused slots of the last page go on the free stack, the lowest on top */
+      if (page >= 0)
+        for (int sl = OR_PAGE - 1; sl >= used; --sl)
+          free_stack(dst, s, c)[dst->free_top[s * 3 + c]++] = e * OR_PAGE + sl;
+    }
+  }
+  return OR_OK;
+}
+
+/* ====================================================================== */
 /* decode attention over the mixed-precision pages                         */
 /* ====================================================================== */
 typedef struct { int32_t pos, cls, page, slot; } live_tok;

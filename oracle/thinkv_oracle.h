@@ -66,6 +66,11 @@ int or_decode(const or_state* S, int32_t n, const int32_t* seq,
 int or_tbe(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos, const uint8_t* tag,
            int32_t t_min, const int32_t* schedule);
 
+/* Gather compaction (what CT avoids): the live tokens of seq[0..n) move into
+ * fresh hole-free pages of the empty cache dst (same geometry), class by
+ * class, FIFO order within a class, codes copied. */
+int or_compact(const or_state* src, or_state* dst, int32_t n, const int32_t* seq);
+
 /* Thought decomposition from attention sparsity (mechanism only): per
  * sequence i, score = (sum over heads, in head order, of mass[i][h]) / hq in
  * fp32; tag T if score >= theta_t, else R if score >= theta_r, else E. */
