@@ -436,8 +436,61 @@ def workload_config(w, live):
 # --------------------------------------------------------------------------- #
 # the library arm
 # --------------------------------------------------------------------------- #
+def compaction_bytes(w, live_by_class) -> int:
+    """Bytes a gather compaction must move at least: every live token's codes
+    and params for every kv-head, read once and written once."""
+    H, d, G = w.num_kv_heads, w.head_dim, w.group_size
+    per = [2 * d * b // 8 + (2 * (d // G) * 4 if b < 16 else 0) for b in w.bits]
+    return 2 * sum(n * H * p for n, p in zip(live_by_class, per))
+
+
+def measure_compaction(w, run, last, out, mass, live, K: int, flush, dev):
+    """The step Continuous Thinking avoids: the state the timed steps left is
+    gathered into fresh hole-free pages of a second cache (thinkv_compact),
+    K times (the copy reset outside the events, L2 flushed), and the same
+    decode call is timed on the compacted copy."""
+    import torch
+    from mixed_precision_paged_thinkv_b200.binding import ThinKVCache
+    c = run.cache
+    pool = [n // 16 + w.batch + 1 for n in live]
+    dst = ThinKVCache(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
+                      c.max_seqs, c.max_blocks, pool, device=str(dev))
+    max_tok = int(sum(live)) + 16 * w.batch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for k in range(K):
+        dst.reset()
+        flush.zero_()
+        ev[k][0].record()
+        c.compact_into(dst, last.seqs, max_tok)
+        ev[k][1].record()
+    torch.cuda.synchronize()
+    assert dst.status() == 0, "device status after compaction"
+    comp_ms = [a.elapsed_time(b) for a, b in ev]
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    for k in range(K):
+        flush.zero_()
+        dev_ev[k][0].record()
+        dst.decode(last.seqs, last.q, topk=w.topk, out=out, mass=mass)
+        dev_ev[k][1].record()
+    torch.cuda.synchronize()
+    dec_ms = [a.elapsed_time(b) for a, b in dev_ev]
+    snap = dst.snapshot()
+    _, _, pages = algorithmic_decode_bytes(w, snap)
+    del dst, snap
+    torch.cuda.empty_cache()
+    cm = sum(comp_ms) / K
+    nbytes = compaction_bytes(w, live)
+    return {"kernels": "thinkv_compact (compact_assign_kernel + compact_copy_kernel)",
+            "ms": cm, "bytes_moved_min": nbytes, "gbs": nbytes / (cm / 1000.0) / 1e9,
+            "decode_ms_on_compacted": sum(dec_ms) / K, "live_pages_after": pages,
+            "note": "what one step would add if it compacted after each eviction (the step "
+                    "Continuous Thinking avoids), and the decode call on the compacted copy"}
+
+
 def measure_workload(w, K: int, Wm: int, dev, flush, e2e_steps: int = 0, clocks=None,
-                     world: int = 1):
+                     world: int = 1, compaction: bool = False):
     """Sets the workload up on the GPU, then times K steps (append + evict +
     decode, one event pair per step, L2 flushed before each), the decode call
     alone K times on the state the steps left, and (if e2e_steps) steps from
@@ -498,6 +551,8 @@ def measure_workload(w, K: int, Wm: int, dev, flush, e2e_steps: int = 0, clocks=
     res = {"step_s": sum(step_ms) / 1000.0, "steps": K, "tokens": float(w.batch * K),
            "step_ms": step_ms, "dec_ms": dec_ms, "alg_bytes": alg_bytes, "live": live,
            "pages": pages, "clocks": clk, "wall_s": t_wall}
+    if compaction:
+        res["compaction"] = measure_compaction(w, run, last, out, mass, live, K, flush, dev)
 
     if e2e_steps:
         # end to end through host buffers (pinned), copies inside the timed
@@ -555,7 +610,8 @@ def thinkv_arm(args, w, world, rank, local):
     clocks = ClockSampler(os.path.join(os.environ.get("THINKV_CLOCK_LOG_DIR", tempfile.gettempdir()),
                                        f"thinkv_clocks_rank{rank}.csv"))
     e2e_steps = max(3, min(K, 20))
-    res = measure_workload(w, K, Wm, dev, flush, e2e_steps=e2e_steps, clocks=clocks, world=world)
+    res = measure_workload(w, K, Wm, dev, flush, e2e_steps=e2e_steps, clocks=clocks, world=world,
+                           compaction=(world == 1))
     max_s, tokens = dist_max_sum(res["step_s"], res["tokens"], world, dev)
     value = tokens / max_s
     e2e_max, e2e_tok = dist_max_sum(res["e2e_s"], res["e2e_tokens"], world, dev)
@@ -601,6 +657,7 @@ def thinkv_arm(args, w, world, rank, local):
             "decode_kv_tokens_per_s": float(sum(res["live"])) / (dec / 1000.0),
             "roofline": roofline_block(w, res),
             "per_config": per_config or None,
+            "compaction_baseline": res.get("compaction"),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tok / e2e_max, "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
                     "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},

@@ -149,3 +149,12 @@ def test_algorithmic_decode_bytes_counts_live_tokens_pages_and_rows():
     want = 2 * (3 * per[8] + 1 * per[4] + 16 * per[2])            # x kv-heads
     want += 3 * 16 + 2 * 8 + 2 * 2 * 4 * 128 * 2 + 2 * 4 * 4     # pages, seqs, Q+O, mass
     assert total == want
+
+
+def test_compaction_bytes_counts_each_live_token_once_each_way():
+    import bench
+    from mixed_precision_paged_thinkv_b200 import workloads as W
+    w = W.WORKLOADS["r1-llama-8b"]          # 8 kv-heads, d 128, G 64, bits 8/4/2
+    # per (token, head): 272 / 144 / 80 bytes at 8 / 4 / 2 bits
+    assert bench.compaction_bytes(w, [10, 0, 0]) == 2 * 10 * 8 * 272
+    assert bench.compaction_bytes(w, [1, 2, 3]) == 2 * 8 * (272 + 2 * 144 + 3 * 80)

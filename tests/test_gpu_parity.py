@@ -251,8 +251,10 @@ def test_decode_shuffled_subset_with_repeated_ids():
     merr = float(np.abs(mass.cpu().numpy().astype(np.float64) - rmass).max())
     print(f"shuffled subset: attention error {err:.3e}, top-k mass error {merr:.3e}")
     assert err <= Hn.TOL and merr <= Hn.MASS_TOL, (err, merr)
-    # the repeated id with the same query gives the same row
+    # the repeated id with the same query gives the same row up to rounding
+    # (the two copies' pages fall at different stream-K split points, so
+    # their partial sums are merged in different orders)
     q2 = q.clone()
     q2[3] = q2[1]
     out2, _ = g.cache.decode(torch.as_tensor(ids, device="cuda"), q2.cuda())
-    assert torch.equal(out2[1], out2[3])
+    assert Hn.attn_error(out2[3:4].cpu().numpy(), out2[1:2].cpu().numpy().astype(np.float64)) <= Hn.TOL
