@@ -50,7 +50,7 @@ class _Layout(C.Structure):
                 ("head_dim", C.c_int32), ("page_size", C.c_int32),
                 ("group_size", C.c_int32), ("bits", C.c_int32 * 3),
                 ("max_seqs", C.c_int32), ("max_blocks_per_seq", C.c_int32),
-                ("pool_pages", C.c_int32 * 3)]
+                ("pool_pages", C.c_int32 * 3), ("fmt", C.c_int32 * 3)]
 
 
 def lib():
@@ -72,6 +72,13 @@ def lib():
             L.or_f16_to_f32.restype = C.c_float
             L.or_f16_round_array.argtypes = [P, C.c_int64, C.c_int32, P]
             L.or_quantize_group.argtypes = [P, C.c_int32, C.c_int32, P, P, P]
+            L.or_quantize_group_fmt.argtypes = [P, C.c_int32, C.c_int32, C.c_int32, P, P, P]
+            for f in ("or_e4m3_value", "or_e2m1_value"):
+                getattr(L, f).argtypes = [C.c_uint8]
+                getattr(L, f).restype = C.c_double
+            for f in ("or_e4m3_from_f32", "or_e2m1_from_f32"):
+                getattr(L, f).argtypes = [C.c_float]
+                getattr(L, f).restype = C.c_uint8
             L.or_classify.argtypes = [C.c_int32, C.c_int32, P, C.c_float, C.c_float, P]
             L.or_tbe.argtypes = [P, C.c_int32, P, P, P, C.c_int32, P]
             L.or_compact.argtypes = [P, P, C.c_int32, P]
@@ -124,15 +131,34 @@ def f16_round_array(x: np.ndarray, mode: str) -> np.ndarray:
     return out
 
 
-def quantize_group(x, bits: int):
+def quantize_group(x, bits: int, fmt: int = 0):
     """Quantise one group of fp16 values: returns (codes uint8, scale bits, zero bits)."""
     xs = _u16(x)
     G = xs.shape[0]
     codes = np.zeros(G, dtype=np.uint8)
     s = np.zeros(1, dtype=np.uint16)
     z = np.zeros(1, dtype=np.uint16)
-    lib().or_quantize_group(_ptr(xs), G, bits, _ptr(codes), _ptr(s), _ptr(z))
+    if fmt:
+        lib().or_quantize_group_fmt(_ptr(xs), G, bits, fmt, _ptr(codes), _ptr(s), _ptr(z))
+    else:
+        lib().or_quantize_group(_ptr(xs), G, bits, _ptr(codes), _ptr(s), _ptr(z))
     return codes, int(s[0]), int(z[0])
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().or_e4m3_value(int(code)))
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().or_e2m1_value(int(code)))
+
+
+def e4m3_from_f32(x: float) -> int:
+    return int(lib().or_e4m3_from_f32(float(x)))
+
+
+def e2m1_from_f32(x: float) -> int:
+    return int(lib().or_e2m1_from_f32(float(x)))
 
 
 def classify(mass, theta_t: float, theta_r: float) -> np.ndarray:
@@ -150,14 +176,16 @@ class Oracle:
 
     def __init__(self, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  group_size: int, bits: Sequence[int], max_seqs: int,
-                 max_blocks_per_seq: int, pool_pages: Sequence[int]):
+                 max_blocks_per_seq: int, pool_pages: Sequence[int],
+                 fmt: Sequence[int] = (0, 0, 0)):
         self.Hq, self.H, self.d, self.G = num_q_heads, num_kv_heads, head_dim, group_size
+        self.fmt = tuple(int(f) for f in fmt)
         self.bits = tuple(int(b) for b in bits)
         self.max_seqs, self.max_blocks = max_seqs, max_blocks_per_seq
         self.pool_pages = tuple(int(p) for p in pool_pages)
         lay = _Layout(num_q_heads, num_kv_heads, head_dim, PAGE, group_size,
                       (C.c_int32 * 3)(*self.bits), max_seqs, max_blocks_per_seq,
-                      (C.c_int32 * 3)(*self.pool_pages))
+                      (C.c_int32 * 3)(*self.pool_pages), (C.c_int32 * 3)(*self.fmt))
         self._lay = lay
         self._h = lib().or_create(C.byref(lay))
         if not self._h:

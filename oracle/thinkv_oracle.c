@@ -145,6 +145,98 @@ void or_quantize_group(const uint16_t* x, int32_t G, int32_t bits,
 }
 
 /* ====================================================================== */
+/* [TBQ] the pages' float formats: FP8 E4M3, FP4 E2M1, ternary             */
+/* ====================================================================== */
+/* The explainer's TBQ names 8-bit FP8 or 4-bit NVFP4 for Reasoning tokens
+ * and 2-bit ternary for Transition tokens.  Formats, from their definitions:
+ *   E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is
+ *         subnormal (m/8 * 2^-6); S.1111.111 is NaN, so the largest finite
+ *         value is 1.75 * 2^8 = 448; no infinities.
+ *   E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit: 0, 0.5, 1, 1.5, 2,
+ *         3, 4, 6 and their negatives.
+ * Rounding from fp32: to the nearest value, ties to the even mantissa, and
+ * magnitudes beyond the largest finite value saturate to it. */
+double or_e4m3_value(uint8_t c) {
+  int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);                  /* m/8 * 2^-6 */
+  else v = ldexp(8.0 + m, e - 10);                       /* (1 + m/8) * 2^(e-7) */
+  return s ? -v : v;
+}
+
+double or_e2m1_value(uint8_t c) {
+  int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  double v = e == 0 ? 0.5 * m : ldexp(2.0 + m, e - 2);   /* (1 + m/2) * 2^(e-1) */
+  return s ? -v : v;
+}
+
+/* nearest code of |x| among the finite non-negative codes 0..last of a
+ * format whose values grow with the code; ties go to the even code (the even
+ * mantissa bit) */
+static uint8_t nearest_code(double a, double (*val)(uint8_t), int last) {
+  if (a >= val((uint8_t)last)) return (uint8_t)last;      /* saturate */
+  int lo = 0;
+  while (lo < last && val((uint8_t)(lo + 1)) <= a) ++lo;  /* val(lo) <= a < val(lo + 1) */
+  double below = val((uint8_t)lo), above = val((uint8_t)(lo + 1));
+  if (a - below < above - a) return (uint8_t)lo;
+  if (a - below > above - a) return (uint8_t)(lo + 1);
+  return (uint8_t)((lo & 1) ? lo + 1 : lo);
+}
+
+uint8_t or_e4m3_from_f32(float x) {
+  if (isnan(x)) return 0x7F;
+  uint8_t c = nearest_code(fabs((double)x), or_e4m3_value, 0x7E);
+  return (uint8_t)(signbit(x) ? (c | 0x80) : c);
+}
+
+uint8_t or_e2m1_from_f32(float x) {
+  if (isnan(x)) return 0x7;                               /* no NaN in E2M1: saturate */
+  uint8_t c = nearest_code(fabs((double)x), or_e2m1_value, 0x7);
+  return (uint8_t)(signbit(x) ? (c | 0x8) : c);
+}
+
+/* One group in a float format (reading of TBQ's formats for the cache's
+ * per-group params):
+ *   FP8 (b = 8): scale = fp16 rounded UP of fp32(amax / 448), zero = 0,
+ *                code = E4M3 of fp32(x / scale);
+ *   FP4 (b = 4): scale = fp16 rounded UP of fp32(amax / 6), zero = 0,
+ *                code = E2M1 of fp32(x / scale) (NVFP4's element format; the
+ *                cache's group of G channels with an fp16 scale takes the
+ *                place of NVFP4's 16-element E4M3 micro-scales);
+ *   ternary (b = 2): scale = fp16 rounded UP of amax, zero = -scale,
+ *                code = clamp(rint_even(fp32(x / scale)), -1, 1) + 1,
+ *                so that zero + code * scale = scale * {-1, 0, +1}.
+ * amax = the largest |x| of the group (fp32).  A zero scale gives the code of
+ * 0 (E4M3/E2M1: 0; ternary: 1) for every element. */
+void or_quantize_group_fmt(const uint16_t* x, int32_t G, int32_t bits, int32_t fmt,
+                           uint8_t* codes, uint16_t* scale, uint16_t* zero) {
+  if (fmt == 0) { or_quantize_group(x, G, bits, codes, scale, zero); return; }
+  float amax = 0.0f;
+  for (int j = 0; j < G; ++j) {
+    float a = fabsf(or_f16_to_f32(x[j]));
+    if (a > amax) amax = a;
+  }
+  float top = bits == 8 ? 448.0f : (bits == 4 ? 6.0f : 1.0f);
+  uint16_t s = or_f16_round_up(amax / top);
+  float sf = or_f16_to_f32(s);
+  for (int j = 0; j < G; ++j) {
+    float v = or_f16_to_f32(x[j]);
+    if (bits == 2) {
+      float c = sf == 0.0f ? 0.0f : rintf(v / sf);
+      if (c < -1.0f) c = -1.0f;
+      if (c > 1.0f) c = 1.0f;
+      codes[j] = (uint8_t)((int)c + 1);
+    } else {
+      float t = sf == 0.0f ? 0.0f : v / sf;
+      codes[j] = bits == 8 ? or_e4m3_from_f32(t) : or_e2m1_from_f32(t);
+    }
+  }
+  *scale = s;
+  *zero = bits == 2 ? (uint16_t)(s ^ 0x8000) : 0;         /* -scale: exact in fp16 */
+}
+
+/* ====================================================================== */
 /* state                                                                   */
 /* ====================================================================== */
 struct or_state {
@@ -199,6 +291,7 @@ static int layout_ok(const or_layout* L) {
     int b = L->bits[c];
     if (b != 2 && b != 4 && b != 8 && b != 16) return 0;
     if (L->pool_pages[c] < 0) return 0;
+    if (L->fmt[c] != 0 && !(L->fmt[c] == 1 && b != 16)) return 0;
   }
   if (L->max_seqs <= 0 || L->max_blocks_per_seq <= 0) return 0;
   return 1;
@@ -286,7 +379,7 @@ static void write_token(or_state* S, int c, int32_t page, int slot,
       uint8_t* dst = (uint8_t*)S->codes[c] + row * d;
       uint16_t* prm = S->params[c] + row * ng * 2;
       for (int g = 0; g < ng; ++g)
-        or_quantize_group(x + g * G, G, b, dst + g * G, &prm[2 * g], &prm[2 * g + 1]);
+        or_quantize_group_fmt(x + g * G, G, b, L->fmt[c], dst + g * G, &prm[2 * g], &prm[2 * g + 1]);
     }
   }
 }
@@ -620,6 +713,7 @@ int or_compact(const or_state* src, or_state* dst, int32_t n, const int32_t* seq
   if (A->num_q_heads != B->num_q_heads || A->num_kv_heads != B->num_kv_heads ||
       A->head_dim != B->head_dim || A->group_size != B->group_size ||
       A->bits[0] != B->bits[0] || A->bits[1] != B->bits[1] || A->bits[2] != B->bits[2] ||
+      A->fmt[0] != B->fmt[0] || A->fmt[1] != B->fmt[1] || A->fmt[2] != B->fmt[2] ||
       A->max_seqs != B->max_seqs || A->max_blocks_per_seq != B->max_blocks_per_seq)
     return OR_ERR_INVALID;
   char* seen = (char*)calloc((size_t)A->max_seqs, 1);
@@ -702,8 +796,10 @@ static double deq(const or_state* S, int c, int32_t page, int h, int kv, int slo
   int ng = L->head_dim / L->group_size, g = j / L->group_size;
   const uint16_t* prm = S->params[c] + row * ng * 2 + 2 * g;
   double scale = or_f16_to_f32(prm[0]), zero = or_f16_to_f32(prm[1]);
-  double code = ((const uint8_t*)S->codes[c])[row * L->head_dim + j];
-  return zero + code * scale;
+  uint8_t code = ((const uint8_t*)S->codes[c])[row * L->head_dim + j];
+  if (L->fmt[c] == 1 && L->bits[c] == 8) return scale * or_e4m3_value(code);
+  if (L->fmt[c] == 1 && L->bits[c] == 4) return scale * or_e2m1_value(code);
+  return zero + (double)code * scale;                    /* integer codes; ternary */
 }
 
 static void decode_one(const or_state* S, int s, const uint16_t* q, double scale,

@@ -35,11 +35,17 @@ enum { OR_OK = 0, OR_ERR_INVALID = 1, OR_ERR_OUT_OF_PAGES = 2, OR_ERR_OUT_OF_BLO
 enum { OR_R = 0, OR_E = 1, OR_T = 2 };
 #define OR_PAGE 16
 
+/* code formats of a class (fmt[c]): integer asymmetric codes, or the float
+ * formats the pages name for the class's bit width (8: FP8 E4M3, 4: FP4
+ * E2M1, 2: ternary) */
+enum { OR_FMT_INT = 0, OR_FMT_FLOAT = 1 };
+
 typedef struct {
   int32_t num_q_heads, num_kv_heads, head_dim, page_size, group_size;
   int32_t bits[3];
   int32_t max_seqs, max_blocks_per_seq;
   int32_t pool_pages[3];
+  int32_t fmt[3];
 } or_layout;
 
 typedef struct or_state or_state;
@@ -85,6 +91,15 @@ float or_f16_to_f32(uint16_t h);
 void or_f16_round_array(const float* x, int64_t n, int32_t mode, uint16_t* out);
 void or_quantize_group(const uint16_t* x, int32_t G, int32_t bits,
                        uint8_t* codes, uint16_t* scale, uint16_t* zero);
+/* the same for any format (fmt OR_FMT_FLOAT: E4M3 / E2M1 / ternary) */
+void or_quantize_group_fmt(const uint16_t* x, int32_t G, int32_t bits, int32_t fmt,
+                           uint8_t* codes, uint16_t* scale, uint16_t* zero);
+/* E4M3 / E2M1: value of a code, and fp32 -> code rounded to nearest, ties to
+ * even, saturating to the largest finite value */
+double or_e4m3_value(uint8_t code);
+uint8_t or_e4m3_from_f32(float x);
+double or_e2m1_value(uint8_t code);
+uint8_t or_e2m1_from_f32(float x);
 
 /* ---- state export (for comparisons) ----------------------------------- */
 /* Natural layouts:
