@@ -274,7 +274,7 @@ class OracleReplay:
             pool = [a + b for a, b in zip(pool, pages)]
             mb = max(mb, sum(pages))
         self.o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
-                          len(self.seqs), mb, [max(1, p) for p in pool])
+                          len(self.seqs), mb, [max(1, p) for p in pool], fmt=w.fmt)
         self.generated = self.sched.lengths[self.seqs].astype(np.int64).copy()
         self.ids = np.arange(len(self.seqs), dtype=np.int32)
 
@@ -417,13 +417,15 @@ def _cuda_ok():
 def workload_config(w, live):
     cfg = {"workload": f"{w.name}: layer {w.num_q_heads}q/{w.num_kv_heads}kv heads, "
                        f"head_dim {w.head_dim}, batch {w.batch}, lengths {w.lengths}, "
-                       f"R/E/T {w.bits[0]}/{w.bits[1]}/{w.bits[2]}-bit, group {w.group_size}, "
+                       f"R/E/T {w.bits[0]}/{w.bits[1]}/{w.bits[2]}-bit"
+                       + (" (FP8 E4M3 / FP4 E2M1 / ternary)" if any(w.fmt) else "")
+                       + f", group {w.group_size}, "
                        f"budget {w.budget}"
                        + (f", {w.churn_steps} churn steps before timing" if w.churn_steps else "")
                        + (f", top-{w.topk} mass" if w.topk else ""),
            "batch": w.batch, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
            "head_dim": w.head_dim, "group_size": w.group_size, "page_size": w.page_size,
-           "bits_RET": list(w.bits), "topk": w.topk,
+           "bits_RET": list(w.bits), "fmt_RET": list(w.fmt), "topk": w.topk,
            "l2": "flushed between steps (512 MiB write, outside the timed events)",
            "parallelism": "replicas"}
     if live is not None:
@@ -454,7 +456,7 @@ def measure_compaction(w, run, last, out, mass, live, K: int, flush, dev):
     c = run.cache
     pool = [n // 16 + w.batch + 1 for n in live]
     dst = ThinKVCache(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
-                      c.max_seqs, c.max_blocks, pool, device=str(dev))
+                      c.max_seqs, c.max_blocks, pool, device=str(dev), fmt=w.fmt)
     max_tok = int(sum(live)) + 16 * w.batch
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]

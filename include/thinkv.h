@@ -88,13 +88,29 @@ enum { THINKV_R = 0, THINKV_E = 1, THINKV_T = 2 };
  *   head_dim in {64, 128}; group_size in {32, 64}, dividing head_dim;
  *   page_size == 16; bits[c] in {2, 4, 8, 16} for c = R, E, T;
  *   1 <= max_seqs <= 65536; 1 <= max_blocks_per_seq <= 2^21;
- *   num_kv_heads <= 256; 0 <= pool_pages[c] < 2^27. */
+ *   num_kv_heads <= 256; 0 <= pool_pages[c] < 2^27;
+ *   fmt[c] in {THINKV_FMT_INT, THINKV_FMT_FLOAT}, FLOAT only with bits 2, 4, 8. */
 typedef struct {
   int32_t num_q_heads, num_kv_heads, head_dim, page_size, group_size;
   int32_t bits[3];
   int32_t max_seqs, max_blocks_per_seq;
   int32_t pool_pages[3];
+  int32_t fmt[3];
 } thinkv_layout;
+
+/* Code formats of a class (fmt[c]).  THINKV_FMT_INT: integer asymmetric codes
+ * (the quantiser below).  THINKV_FMT_FLOAT: the formats the explainer's TBQ
+ * names, by bit width -- 8: FP8 E4M3, scale = fp16 rounded up of amax/448,
+ * zero 0, code = E4M3 of fp32(x/scale); 4: FP4 E2M1 (NVFP4's element format;
+ * the group of G channels with its fp16 scale stands in for NVFP4's
+ * 16-element E4M3 micro-scales), scale = fp16 rounded up of amax/6, zero 0;
+ * 2: ternary, scale = fp16 rounded up of amax, code = clamp(rint_even(fp32(x
+ * / scale)), -1, 1) + 1, zero = -scale.  amax: the group's largest |x|.
+ * E4M3/E2M1 rounding: to nearest, ties to even, saturating to 448 / 6.
+ * Dequantised value: scale * value(code) (E4M3/E2M1), zero + code * scale
+ * (ternary, as integer codes).  Same bytes and layout as the integer codes
+ * of that width.  A zero-filled fmt is all integer. */
+enum { THINKV_FMT_INT = 0, THINKV_FMT_FLOAT = 1 };
 
 /* The cache: device buffers, all allocated and owned by the caller with the
  * sizes thinkv_buffer_bytes() reports, and initialised by thinkv_cache_reset().

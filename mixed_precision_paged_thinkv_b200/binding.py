@@ -52,7 +52,7 @@ class Layout(C.Structure):
                 ("head_dim", C.c_int32), ("page_size", C.c_int32),
                 ("group_size", C.c_int32), ("bits", C.c_int32 * 3),
                 ("max_seqs", C.c_int32), ("max_blocks_per_seq", C.c_int32),
-                ("pool_pages", C.c_int32 * 3)]
+                ("pool_pages", C.c_int32 * 3), ("fmt", C.c_int32 * 3)]
 
 
 class CacheStruct(C.Structure):
@@ -146,10 +146,11 @@ def classify_thoughts(mass: torch.Tensor, theta_t: float, theta_r: float,
 
 
 def make_layout(num_q_heads, num_kv_heads, head_dim, group_size, bits, max_seqs,
-                max_blocks_per_seq, pool_pages) -> Layout:
+                max_blocks_per_seq, pool_pages, fmt=(0, 0, 0)) -> Layout:
     return Layout(int(num_q_heads), int(num_kv_heads), int(head_dim), PAGE, int(group_size),
                   (C.c_int32 * 3)(*[int(b) for b in bits]), int(max_seqs),
-                  int(max_blocks_per_seq), (C.c_int32 * 3)(*[int(p) for p in pool_pages]))
+                  int(max_blocks_per_seq), (C.c_int32 * 3)(*[int(p) for p in pool_pages]),
+                  (C.c_int32 * 3)(*[int(f) for f in fmt]))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -175,9 +176,11 @@ class ThinKVCache:
 
     def __init__(self, num_q_heads: int, num_kv_heads: int, head_dim: int, group_size: int,
                  bits: Sequence[int], max_seqs: int, max_blocks_per_seq: int,
-                 pool_pages: Sequence[int], device: str = "cuda", tbe: bool = False):
+                 pool_pages: Sequence[int], device: str = "cuda", tbe: bool = False,
+                 fmt: Sequence[int] = (0, 0, 0)):
         self.layout = make_layout(num_q_heads, num_kv_heads, head_dim, group_size, bits,
-                                  max_seqs, max_blocks_per_seq, pool_pages)
+                                  max_seqs, max_blocks_per_seq, pool_pages, fmt)
+        self.fmt = tuple(int(f) for f in fmt)
         L = lib()
         _check(L.thinkv_layout_check(C.byref(self.layout)), "layout")
         self.Hq, self.H, self.d, self.G = num_q_heads, num_kv_heads, head_dim, group_size

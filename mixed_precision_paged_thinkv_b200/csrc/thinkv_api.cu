@@ -31,6 +31,7 @@ bool layout_ok(const thinkv_layout* L) {
     const int b = L->bits[c];
     if (b != 2 && b != 4 && b != 8 && b != 16) return false;
     if (L->pool_pages[c] < 0 || L->pool_pages[c] >= (1 << 27)) return false;
+    if (L->fmt[c] != THINKV_FMT_INT && !(L->fmt[c] == THINKV_FMT_FLOAT && b != 16)) return false;
   }
   if (L->max_seqs < 1 || L->max_seqs > 65536) return false;
   if (L->max_blocks_per_seq < 1 || L->max_blocks_per_seq > (1 << 21)) return false;
@@ -283,7 +284,8 @@ int thinkv_compact(const thinkv_cache* src, const thinkv_cache* dst, int32_t n, 
   const thinkv_layout &A = src->L, &B = dst->L;
   if (A.num_q_heads != B.num_q_heads || A.num_kv_heads != B.num_kv_heads ||
       A.head_dim != B.head_dim || A.group_size != B.group_size || A.bits[0] != B.bits[0] ||
-      A.bits[1] != B.bits[1] || A.bits[2] != B.bits[2] || A.max_seqs != B.max_seqs ||
+      A.bits[1] != B.bits[1] || A.bits[2] != B.bits[2] || A.fmt[0] != B.fmt[0] ||
+      A.fmt[1] != B.fmt[1] || A.fmt[2] != B.fmt[2] || A.max_seqs != B.max_seqs ||
       A.max_blocks_per_seq != B.max_blocks_per_seq || n > A.max_seqs)
     return THINKV_ERR_INVALID;
   if (n == 0) return THINKV_OK;

@@ -345,7 +345,11 @@ __device__ inline RowVals<D> load_row(const uint16_t* __restrict__ x) {
 // Quantises one K or V row of one kv-head (values held by the warp, D/32
 // channels per lane) at bit width B (class c) and writes its codes and params
 // into slot pool_slot & 15 of page pool_slot >> 4's page-head block.
-template <int D, int G, int B>
+// F = 0: integer asymmetric codes.  F = 1: the float formats -- FP8 E4M3 (B =
+// 8) and FP4 E2M1 (B = 4) with scale = fp16 rounded up of amax / (largest
+// finite value) and zero 0; ternary (B = 2) with scale = fp16 rounded up of
+// amax, code = clamp(rint_even(x / scale), -1, 1) + 1 and zero = -scale.
+template <int D, int G, int B, int F>
 __device__ void scatter_unit_b(const CacheView& C, int c, uint32_t pool_slot, int h, int kv,
                                const RowVals<D>& vals, uint16_t* code_sm) {
   constexpr int PER = D / 32;          // channels per lane
@@ -359,6 +363,38 @@ __device__ void scatter_unit_b(const CacheView& C, int c, uint32_t pool_slot, in
   if constexpr (B == 16) {
 #pragma unroll
     for (int e = 0; e < PER; ++e) code_sm[lane * PER + e] = raw[e];
+  } else if constexpr (F == 1) {
+    float xf[PER], amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      xf[e] = __half2float(__ushort_as_half(raw[e]));
+      amax = fmaxf(amax, fabsf(xf[e]));
+    }
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    constexpr float top = B == 8 ? 448.f : (B == 4 ? 6.f : 1.f);
+    const __half sh = __float2half_ru(__fdiv_rn(amax, top));
+    const float sf = __half2float(sh);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      uint32_t cq;
+      if constexpr (B == 2) {
+        float r = sf == 0.f ? 0.f : rintf(__fdiv_rn(xf[e], sf));
+        r = fminf(fmaxf(r, -1.f), 1.f);
+        cq = (uint32_t)((int)r + 1);
+      } else {
+        const float t = sf == 0.f ? 0.f : __fdiv_rn(xf[e], sf);
+        cq = B == 8 ? e4m3_code(t) : e2m1_code(t);
+      }
+      code_sm[lane * PER + e] = (uint16_t)cq;
+    }
+    const int grp = (lane * PER) / G;
+    if ((lane % LPG) == 0) {
+      uint16_t* prm = reinterpret_cast<uint16_t*>(blk + 4LL * D * B + (kv ? 64LL * NG : 0));
+      const uint16_t zb = B == 2 ? (uint16_t)(__half_as_ushort(sh) ^ 0x8000u) : (uint16_t)0;
+      const uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)zb << 16);
+      *reinterpret_cast<uint32_t*>(prm + (grp * 16 + slot) * 2) = pair;
+    }
   } else {
     float xf[PER], mn = INFINITY, mx = -INFINITY;
 #pragma unroll
@@ -460,11 +496,14 @@ __device__ void scatter_unit_b(const CacheView& C, int c, uint32_t pool_slot, in
 template <int D, int G>
 __device__ inline void scatter_unit(const CacheView& C, int c, uint32_t pool_slot, int h, int kv,
                                     const RowVals<D>& vals, uint16_t* code_sm) {
-  switch (C.L.bits[c]) {
-    case 8: scatter_unit_b<D, G, 8>(C, c, pool_slot, h, kv, vals, code_sm); break;
-    case 4: scatter_unit_b<D, G, 4>(C, c, pool_slot, h, kv, vals, code_sm); break;
-    case 2: scatter_unit_b<D, G, 2>(C, c, pool_slot, h, kv, vals, code_sm); break;
-    default: scatter_unit_b<D, G, 16>(C, c, pool_slot, h, kv, vals, code_sm); break;
+  switch (C.L.bits[c] + (C.L.fmt[c] == 1 ? 256 : 0)) {
+    case 8: scatter_unit_b<D, G, 8, 0>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 4: scatter_unit_b<D, G, 4, 0>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 2: scatter_unit_b<D, G, 2, 0>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 256 + 8: scatter_unit_b<D, G, 8, 1>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 256 + 4: scatter_unit_b<D, G, 4, 1>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    case 256 + 2: scatter_unit_b<D, G, 2, 1>(C, c, pool_slot, h, kv, vals, code_sm); break;
+    default: scatter_unit_b<D, G, 16, 0>(C, c, pool_slot, h, kv, vals, code_sm); break;
   }
 }
 

@@ -229,4 +229,58 @@ __device__ inline uint32_t neg_centre_bits() {
   return h | (h << 16);
 }
 
+// ---------------------------------------------------------------------------
+// the float code formats (a class with fmt 1): FP8 E4M3 and FP4 E2M1, converted
+// by the hardware's cvt (round to nearest even, saturating to the largest
+// finite value); both are exact in fp16.
+// ---------------------------------------------------------------------------
+// E4M3 code of x.
+__device__ inline uint32_t e4m3_code(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(x));
+  return r & 0xFFu;
+}
+// E2M1 code of x (4 bits).
+__device__ inline uint32_t e2m1_code(float x) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(x));
+  return r & 0xFu;
+}
+// Two E4M3 codes (lo: bits 0-7, hi: bits 8-15) as the half2 (value(lo), value(hi)).
+__device__ inline uint32_t e4m3x2_to_half2(uint32_t pair) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\t"
+      "cvt.u16.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(r)
+      : "r"(pair));
+  return r;
+}
+// Two E2M1 codes (lo: bits 0-3, hi: bits 4-7) as the half2 (value(lo), value(hi)).
+__device__ inline uint32_t e2m1x2_to_half2(uint32_t pair) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.u8.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(r)
+      : "r"(pair));
+  return r;
+}
+// Float-format operand pair k of word w, laid out like unpack_pair: element k
+// of the low half-word (even channel / first token) in the low fp16 half,
+// element k of the high half-word in the high half.
+template <int B>
+__device__ inline uint32_t unpack_float_pair(uint32_t w, int k) {
+  if constexpr (B == 8) {
+    return e4m3x2_to_half2(__byte_perm(w, 0u, k == 0 ? 0x0020u : 0x0031u));
+  } else {
+    const uint32_t t = w >> (4 * k);
+    return e2m1x2_to_half2((t & 0xFu) | ((t >> 12) & 0xF0u));
+  }
+}
+
 }  // namespace thinkv

@@ -495,7 +495,10 @@ __device__ __forceinline__ void lane_words(const uint8_t* base, int w0, uint32_t
 //       removes the offset; 4- and 2-bit codes are centred in the operand (a
 //       centred code of 1 or 2 next to a 1024 offset would lose 9-10 bits of
 //       the running accumulator on every page).
-template <int D, int G, int B>
+//   Float codes (FP8 E4M3 at b = 8, FP4 E2M1 at b = 4; F = 1) enter as their
+//   exact fp16 values with no offset and a zero of 0; ternary codes are the
+//   2-bit integer path (zero = -scale).
+template <int D, int G, int B, int F = 0>
 __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
                                  float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
   const uint2* qfrag = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(pbuf) + kQfragOff);
@@ -545,8 +548,12 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
               a[hi * 2 + r] = w[r][u];
             } else {
               constexpr int PAIRS = (PB == 2 ? 4 : 16 / B);  // pairs per (spread) word
-              a[hi * 2 + r] = unpack_pair<B>(w[r][u / PAIRS], u % PAIRS);
-              if constexpr (B != 8) a[hi * 2 + r] = hsub2_bits(a[hi * 2 + r], centre_bits<B>());
+              if constexpr (F == 1) {
+                a[hi * 2 + r] = unpack_float_pair<B>(w[r][u / PAIRS], u % PAIRS);
+              } else {
+                a[hi * 2 + r] = unpack_pair<B>(w[r][u / PAIRS], u % PAIRS);
+                if constexpr (B != 8) a[hi * 2 + r] = hsub2_bits(a[hi * 2 + r], centre_bits<B>());
+              }
             }
           }
         }
@@ -559,7 +566,7 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
         const uint32_t p0 = kpar[gr * 16 + g], p1 = kpar[gr * 16 + g + 8];
         const float2 sz0 = __half22float2(*reinterpret_cast<const __half2*>(&p0));  // (s, z)
         const float2 sz1 = __half22float2(*reinterpret_cast<const __half2*>(&p1));
-        constexpr float off = B == 8 ? -1024.f : (float)(1 << (B - 1));   // see above
+        constexpr float off = F == 1 ? 0.f : (B == 8 ? -1024.f : (float)(1 << (B - 1)));   // see above
         const float zc0 = fmaf(off, sz0.x, sz0.y), zc1 = fmaf(off, sz1.x, sz1.y);
         lg[0] = fmaf(sz0.x, c[0], fmaf(zc0, S.qsum[gr][0], lg[0]));
         lg[1] = fmaf(sz0.x, c[1], fmaf(zc0, S.qsum[gr][1], lg[1]));
@@ -637,8 +644,9 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
       const uint32_t p0 = vpar[gr * 16 + g], p1 = vpar[gr * 16 + g + 8];
       const float2 sz0 = __half22float2(*reinterpret_cast<const __half2*>(&p0));
       const float2 sz1 = __half22float2(*reinterpret_cast<const __half2*>(&p1));
-      const float zv0 = live0 ? fmaf((float)(1 << (B - 1)), sz0.x, sz0.y) : 0.f;
-      const float zv1 = live1 ? fmaf((float)(1 << (B - 1)), sz1.x, sz1.y) : 0.f;
+      constexpr float voff = F == 1 ? 0.f : (float)(1 << (B - 1));
+      const float zv0 = live0 ? fmaf(voff, sz0.x, sz0.y) : 0.f;
+      const float zv1 = live1 ? fmaf(voff, sz1.x, sz1.y) : 0.f;
       S.z[gr][0] = fmaf(S.z[gr][0], a0, fmaf(pr[0], zv0, pr[2] * zv1));
       S.z[gr][1] = fmaf(S.z[gr][1], a1, fmaf(pr[1], zv0, pr[3] * zv1));
     }
@@ -769,13 +777,17 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
             if constexpr (B == 16) {
               a[P * 2 + r] = vr[P][wq] & (P ? dm1 : dm0);   // raw values of dead slots: zero
             } else {
-              a[P * 2 + r] = unpack_pair<B>(vr[P][wq], e % PER);   // 1024 + code
-              if constexpr (B != 8) a[P * 2 + r] = hsub2_bits(a[P * 2 + r], centre_bits<B>());
+              if constexpr (F == 1) {
+                a[P * 2 + r] = unpack_float_pair<B>(vr[P][wq], e % PER);   // value(code)
+              } else {
+                a[P * 2 + r] = unpack_pair<B>(vr[P][wq], e % PER);   // 1024 + code
+                if constexpr (B != 8) a[P * 2 + r] = hsub2_bits(a[P * 2 + r], centre_bits<B>());
+              }
             }
           }
         }
         mma_16816(S.acc[mt], a, wf[gr][0], wf[gr][1]);
-        if constexpr (B == 8) {
+        if constexpr (B == 8 && F == 0) {
           // centre at once: + (-(1024 + 2^(b-1))) * sum of W over the page's
           // tokens, so the segment's accumulators never carry the offset
           const uint32_t kc = neg_centre_bits<B>();
@@ -787,10 +799,13 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   }
 }
 
+// bits: the class's code width, plus 256 for the float formats at 8 and 4 bits
 template <int D, int G>
 __device__ inline void page_dispatch(SegState<D, G>& S, const uint8_t* blk, int bits, uint32_t mask,
                                      float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
   switch (bits) {
+    case 256 + 8: page_step<D, G, 8, 1>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 256 + 4: page_step<D, G, 4, 1>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
     case 8: page_step<D, G, 8>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
     case 4: page_step<D, G, 4>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
     case 2: page_step<D, G, 2>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
@@ -1360,7 +1375,8 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   for (int c = 0; c < 3; ++c) {
     p.pool[c] = C.pool[c];
     p.phb[c] = (int32_t)page_head_bytes(D, G, L.bits[c]);
-    p.bits[c] = L.bits[c];
+    // the float formats take their own page steps (ternary is the 2-bit path)
+    p.bits[c] = L.bits[c] + ((L.fmt[c] == 1 && L.bits[c] != 2) ? 256 : 0);
   }
   p.table = C.block_table;
   p.live_list = C.live_list;

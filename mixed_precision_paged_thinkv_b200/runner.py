@@ -51,7 +51,7 @@ class WorkloadRun:
         self.cache = ThinKVCache(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size,
                                  bits or w.bits, self.geom["max_seqs"],
                                  self.geom["max_blocks_per_seq"], self.geom["pool_pages"],
-                                 device=device)
+                                 device=device, fmt=w.fmt)
         self.generated = self.sched.lengths.astype(np.int64).copy()
         self.all_seqs = torch.arange(w.batch, dtype=torch.int32, device=self.device)
 

@@ -54,6 +54,9 @@ class Workload:
     head_dim: int
     group_size: int
     bits: Tuple[int, int, int] = (8, 4, 2)
+    # code format per class: 0 integer asymmetric codes, 1 the float formats
+    # (FP8 E4M3 / FP4 E2M1 / ternary at 8 / 4 / 2 bits)
+    fmt: Tuple[int, int, int] = (0, 0, 0)
     page_size: int = PAGE_SIZE
     # sequence lengths: ("fixed", n) | ("uniform", lo, hi) | ("loguniform", lo, hi)
     lengths: tuple = ("fixed", 512)
@@ -118,9 +121,18 @@ def before_eviction(w: Workload) -> Workload:
                                check_every=0)
 
 
+def float_formats(w: Workload) -> Workload:
+    """The same layer and history with the pages' own code formats: FP8 E4M3
+    for R, FP4 E2M1 for E, ternary for T (the explainer's TBQ)."""
+    return dataclasses.replace(w, name=w.name + "-float", fmt=(1, 1, 1))
+
+
 # Supplementary measurements (not the headline configurations).
 SUPPLEMENTARY = {n + "-mixed": before_eviction(WORKLOADS[n])
                  for n in ("r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b", "churn")}
+SUPPLEMENTARY.update({n + "-float": float_formats(WORKLOADS[n])
+                      for n in ("r1-llama-8b", "churn")})
+SUPPLEMENTARY["r1-llama-8b-mixed-float"] = float_formats(before_eviction(WORKLOADS["r1-llama-8b"]))
 
 
 def get(name: str) -> Workload:

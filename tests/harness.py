@@ -26,7 +26,7 @@ class OracleRun:
         self.sched = W.Schedule(w, extra)
         self.o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size,
                           bits or w.bits, geom["max_seqs"], geom["max_blocks_per_seq"],
-                          geom["pool_pages"])
+                          geom["pool_pages"], fmt=w.fmt)
         self.generated = self.sched.lengths.astype(np.int64).copy()
         self.all_seqs = np.arange(w.batch, dtype=np.int32)
 
@@ -171,7 +171,7 @@ class OracleSubset:
                 pool[c] += pages[c]
             mb = max(mb, sum(pages))
         self.o = O.Oracle(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
-                          len(self.seqs), mb, [max(1, p) for p in pool])
+                          len(self.seqs), mb, [max(1, p) for p in pool], fmt=w.fmt)
         self.generated = self.sched.lengths[self.seqs].astype(np.int64).copy()
 
     def _append(self, runs):

@@ -258,3 +258,48 @@ def test_decode_shuffled_subset_with_repeated_ids():
     q2[3] = q2[1]
     out2, _ = g.cache.decode(torch.as_tensor(ids, device="cuda"), q2.cuda())
     assert Hn.attn_error(out2[3:4].cpu().numpy(), out2[1:2].cpu().numpy().astype(np.float64)) <= Hn.TOL
+
+
+@pytest.mark.parametrize("fmt,bits", [((1, 1, 1), (8, 4, 2)), ((1, 0, 1), (8, 4, 2)),
+                                      ((0, 1, 1), (4, 8, 2)), ((1, 1, 0), (2, 8, 4))])
+@pytest.mark.parametrize("d,G", [(128, 64), (64, 32)])
+def test_float_code_formats(fmt, bits, d, G):
+    """The pages' own formats (FP8 E4M3, FP4 E2M1, ternary), alone and mixed
+    with integer classes: codes and params bit-exact with the oracle (the
+    hardware's E4M3/E2M1 rounding against the formats' definitions), state
+    bit-exact, attention and top-k mass within 2e-3, before and after churn."""
+    w = W.Workload(name="x", batch=3, num_q_heads=8, num_kv_heads=2, head_dim=d, group_size=G,
+                   bits=bits, fmt=fmt, lengths=("uniform", 300, 1200), segments=("geometric", 12),
+                   budget=("frac", 0.4), seed=23)
+    g, o = _pair(w, extra=10, bits=bits)
+    g.setup()
+    o.setup()
+    _check_all(g, o, topk=8)
+    for step in range(1, 3):
+        g.churn_step()
+        o.churn_step()
+        _check_all(g, o, step=step, topk=16)
+
+
+def test_float_formats_full_size_mixed_state():
+    """The r1-llama-8b history kept whole (R/E/T mix at FP8/FP4/ternary), in
+    the launch configuration the bench times; sampled sequences against the
+    oracle."""
+    from mixed_precision_paged_thinkv_b200.runner import WorkloadRun
+    w = W.get("r1-llama-8b-mixed-float")
+    g = WorkloadRun(w, extra=2)
+    g.setup()
+    osub = Hn.OracleSubset(w, [0, 7, 15], extra=2)
+    osub.setup()
+    torch.cuda.synchronize()
+    assert g.cache.status() == 0
+    snap = g.cache.snapshot()
+    ost = osub.o.state()
+    for j, s in enumerate(osub.seqs):
+        Hn.compare_seq_structure(snap, s, ost, j)
+        Hn.compare_codes_by_pos(g.cache, Hn.gpu_live_by_pos(snap, s), osub.o, osub.live_by_pos(j))
+    out, _ = g.decode(0)
+    ref, _ = osub.decode(0)
+    err = Hn.attn_error(out.cpu().numpy()[osub.seqs], ref)
+    print(f"r1-llama-8b-mixed-float: attention error {err:.3e}")
+    assert err <= Hn.TOL
