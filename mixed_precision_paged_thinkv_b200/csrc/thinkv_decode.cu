@@ -778,7 +778,9 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
               a[P * 2 + r] = vr[P][wq] & (P ? dm1 : dm0);   // raw values of dead slots: zero
             } else {
               if constexpr (F == 1) {
-                a[P * 2 + r] = unpack_float_pair<B>(vr[P][wq], e % PER);   // value(code)
+                // value(code); a dead slot's stale byte may be an E4M3 NaN,
+                // which its zero weight would not cancel: zero it here
+                a[P * 2 + r] = unpack_float_pair<B>(vr[P][wq], e % PER) & (P ? dm1 : dm0);
               } else {
                 a[P * 2 + r] = unpack_pair<B>(vr[P][wq], e % PER);   // 1024 + code
                 if constexpr (B != 8) a[P * 2 + r] = hsub2_bits(a[P * 2 + r], centre_bits<B>());
@@ -1323,21 +1325,19 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
     return false;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return false;
   // one CTA per SM: the stages take what the prefix, the per-warp scratch and
-  // the kernel's static shared memory (under 1 KB) leave.  Of the warp counts
-  // that fit at least two stages (whose ring can hold the warp's last piece
-  // record after the loop), the one with the most stages in flight per SM
-  // wins; ties go to more warps.
+  // the kernel's static shared memory (under 1 KB) leave.  The most warps
+  // that fit at least two stages each win (warps hide the page step's
+  // latency; a deeper ring at fewer warps measured far slower), with as many
+  // stages as fit; the ring must also hold the warp's last piece record
   const int64_t fixed = plan_smem_bytes(n_seqs) + 1024;
   int best_nw = 0, best_ns = 0;
-  for (int nw = kDecWarps; nw >= 4; --nw) {
+  for (int nw = kDecWarps; nw >= 4 && best_nw == 0; --nw) {
     const int64_t per_warp = (optin - fixed) / nw - 64 - kPbufBytes - topk_bytes;
     int ns = per_warp > 0 ? (int)(per_warp / stage_bytes) : 0;
     if (ns > kMaxStages) ns = kMaxStages;
     if (ns < 2 || (int64_t)ns * stage_bytes < rb) continue;
-    if (nw * ns > best_nw * best_ns) {
-      best_nw = nw;
-      best_ns = ns;
-    }
+    best_nw = nw;
+    best_ns = ns;
   }
   if (best_nw == 0) return false;
   const int warp_smem = best_ns * stage_bytes + 64 + kPbufBytes + topk_bytes;
