@@ -454,6 +454,8 @@ def measure_compaction(w, run, last, out, mass, live, K: int, flush, dev):
     import torch
     from mixed_precision_paged_thinkv_b200.binding import ThinKVCache
     c = run.cache
+    # sized from the state as it is now (the timed steps may have grown it)
+    _, live, _ = algorithmic_decode_bytes(w, c.snapshot())
     pool = [n // 16 + w.batch + 1 for n in live]
     dst = ThinKVCache(w.num_q_heads, w.num_kv_heads, w.head_dim, w.group_size, w.bits,
                       c.max_seqs, c.max_blocks, pool, device=str(dev), fmt=w.fmt)
