@@ -486,7 +486,7 @@ def measure_compaction(w, run, last, out, mass, live, K: int, flush, dev):
     torch.cuda.empty_cache()
     cm = sum(comp_ms) / K
     nbytes = compaction_bytes(w, live)
-    return {"kernels": "thinkv_compact (compact_assign_kernel + compact_copy_kernel)",
+    return {"kernels": "thinkv_compact (compact_count_kernel, compact_plan_kernel, compact_list_kernel, compact_copy_kernel)",
             "ms": cm, "bytes_moved_min": nbytes, "gbs": nbytes / (cm / 1000.0) / 1e9,
             "decode_ms_on_compacted": sum(dec_ms) / K, "live_pages_after": pages,
             "note": "what one step would add if it compacted after each eviction (the step "

@@ -333,7 +333,8 @@ THINKV_API size_t thinkv_compact_workspace_bytes(int32_t n_seqs, int32_t max_tok
  * repeated/out-of-range id -> INVALID, an exhausted dst pool -> OUT_OF_PAGES,
  * both in dst's status with nothing changed.  workspace: device, >=
  * thinkv_compact_workspace_bytes(n_seqs, max_tokens), no initialisation.
- * Two kernels: the assignment (one CTA) and the copy (a warp per page-head). */
+ * Four kernels: count (a warp per sequence and class), plan (one CTA), list
+ * (a warp per sequence and class) and copy (a warp per page-head). */
 THINKV_API int thinkv_compact(const thinkv_cache* src, const thinkv_cache* dst, int32_t n_seqs,
                               const int32_t* seq, int32_t max_tokens, void* workspace,
                               size_t workspace_bytes, void* stream);
