@@ -876,188 +876,169 @@ __device__ __forceinline__ T ld_rec(const T* ptr) {
   else return *ptr;
 }
 
-// Shared scratch of the merges, carved from the warps' p-transpose buffers
-// (idle after the loop): warp 0's holds the (weight * l) table of 32 pieces x
-// 8 heads, warp 1's the weights, the heads' M and L, flags and lists; the
-// top-k lists of a head are staged in the buffer of a warp from 2 on.
-struct MergeScratch {
-  float* wl;     // [32][8]
-  float* wt;     // [32][8]
-  int* mk;       // [8] per-head maxima as order-preserving ints
-  float* M;      // [8]
-  float* L;      // [8]
-  int* flag;     // [4]
-  int* list;     // up to 320 ints (warps or CTAs holding a segment's pieces)
-  uint8_t* pbuf0;
-  int warp_smem;
-};
-
-// a float's order-preserving int key (negative floats: magnitude bits
-// flipped); the map is its own inverse
-__device__ inline int okey(int b) { return b >= 0 ? b : b ^ 0x7FFFFFFF; }
-
-// Merges np piece records of segment `seg` with the log-sum-exp rule, every
-// thread of the CTA taking part (called by all of them, with uniform
-// arguments): per head, M = max m_j, L = sum l_j 2^(m_j - M), o = sum o_j
+// Merges np piece records of segment `seg` with the log-sum-exp rule (one
+// warp): per head, M = max m_j, L = sum l_j 2^(m_j - M), o = sum o_j
 // 2^(m_j - M), and the top-k logits of all pieces merged into one sorted
 // list.  If dst is null the result is final: O = o / L in fp16 and the top-k
-// mass are written out; otherwise the merged piece is written at dst.  The
-// (m, l) pairs of a chunk of 32 pieces are requested at once, a thread per
-// output quad streams the chunk's rows four pieces at a time, and a warp per
-// head merges its top-k lists after staging them in shared memory: a handful
-// of memory round trips in all, whatever the number of pieces.
+// mass are written out.  Otherwise the merged piece is written at dst (a
+// record, for a later merge).  `piece(j)` gives the address of record j.
+// Written for few memory round trips: the (m, l) pairs of up to 16 pieces
+// are requested at once into a shared table, every lane requests all its
+// output quads of a piece at once, and each head's top-k lists are staged in
+// shared memory with one pass of loads before the bitonic merges.
+// wb: this warp's 704-float scratch: M[8], L[8], ints [16, 176) for the
+// caller's piece list, the table at [176, 432), weights at [432, 560); the
+// top-k staging reuses [176, 704).
 template <int D, bool kL2, typename PieceFn>
-__device__ void cta_merge(const DecodeParams& p, int seg, int np, PieceFn piece, uint8_t* dst,
-                          const MergeScratch& sc) {
-  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = nt >> 5;
+__device__ void merge_pieces(const DecodeParams& p, int seg, int np, PieceFn piece, uint8_t* dst,
+                             float* wb) {
+  const int lane = threadIdx.x & 31;
   const int Gq = p.Gq, k = p.topk, kpad = (k + 3) / 4 * 4;
   const int i = seg / p.Hkv, h = seg - (seg / p.Hkv) * p.Hkv;
-  constexpr int QD = D / 4;
-  const int nquad = Gq * QD;                      // <= 256
-  if (tid < 8) {
-    sc.mk[tid] = INT_MIN;
-    sc.L[tid] = 0.f;
-  }
-  __syncthreads();
-  for (int x = tid; x < np * Gq; x += nt) {
-    const int j = x / Gq, r = x - j * Gq;
-    const float m = ld_rec<kL2>(reinterpret_cast<const float2*>(piece(j)) + r).x;
-    atomicMax(&sc.mk[r], okey(__float_as_int(m)));
-  }
-  __syncthreads();
-  if (tid < 8) sc.M[tid] = __int_as_float(okey(sc.mk[tid]));
-  __syncthreads();
-  float4 acc[2];
-  acc[0] = acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j0 = 0; j0 < np; j0 += 32) {
-    const int cnt = min(32, np - j0);
-    for (int x = tid; x < cnt * Gq; x += nt) {
+  constexpr int CH = 16;                          // pieces per table chunk
+  float* M = wb;
+  float* L = wb + 8;
+  float2* tbl = reinterpret_cast<float2*>(wb + 176);
+  float* wt = wb + 432;
+  auto load_table = [&](int j0, int cnt) {
+    for (int x = lane; x < cnt * Gq; x += 32) {
       const int j = x / Gq, r = x - j * Gq;
-      const float2 ml = ld_rec<kL2>(reinterpret_cast<const float2*>(piece(j0 + j)) + r);
-      const float w = ml.x == -INFINITY ? 0.f : exp2_approx(ml.x - sc.M[r]);
-      sc.wt[j * 8 + r] = w;
-      sc.wl[j * 8 + r] = w * ml.y;
+      tbl[j * 8 + r] = ld_rec<kL2>(reinterpret_cast<const float2*>(piece(j0 + j)) + r);
     }
-    __syncthreads();
-    if (tid < Gq) {                               // L, summed in a fixed order
-      float l = sc.L[tid];
-      for (int j = 0; j < cnt; ++j) l += sc.wl[j * 8 + tid];
-      sc.L[tid] = l;
+    __syncwarp();
+  };
+  // maxima (one chunk: the table stays for the weights)
+  if (lane < 8) {
+    M[lane] = -INFINITY;
+    L[lane] = 0.f;
+  }
+  for (int j0 = 0; j0 < np; j0 += CH) {
+    load_table(j0, min(CH, np - j0));
+    if (lane < Gq) {
+      float m = M[lane];
+      for (int j = 0; j < min(CH, np - j0); ++j) m = fmaxf(m, tbl[j * 8 + lane].x);
+      M[lane] = m;
     }
+    __syncwarp();
+  }
+  constexpr int QD = D / 4;
+  const int nquad = Gq * QD;                      // <= 256: at most 8 quads per lane
+  float4 acc[8];
 #pragma unroll
-    for (int q2 = 0; q2 < 2; ++q2) {
-      const int e = tid + q2 * nt;
-      if (e >= nquad) continue;
-      const int r = e / QD;
-      int j = 0;
-      for (; j + 4 <= cnt; j += 4) {              // four pieces' rows in flight
-        float4 v[4];
+  for (int x = 0; x < 8; ++x) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < np; j0 += CH) {
+    const int cnt = min(CH, np - j0);
+    if (np > CH) load_table(j0, cnt);             // else the table is still there
+    if (lane < Gq) {                              // weights, and L in a fixed order
+      float l = L[lane];
+      for (int j = 0; j < cnt; ++j) {
+        const float2 ml = tbl[j * 8 + lane];
+        const float w = ml.x == -INFINITY ? 0.f : exp2_approx(ml.x - M[lane]);
+        wt[j * 8 + lane] = w;
+        l = fmaf(w, ml.y, l);
+      }
+      L[lane] = l;
+    }
+    __syncwarp();
+    for (int j = 0; j < cnt; ++j) {               // a piece's quads all in flight
+      const float4* o = reinterpret_cast<const float4*>(piece(j0 + j) + 64);
+      float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          v[u] = ld_rec<kL2>(reinterpret_cast<const float4*>(piece(j0 + j + u) + 64) + e);
+      for (int x = 0; x < 8; ++x) {
+        const int e = x * 32 + lane;
+        if (e < nquad) v[x] = ld_rec<kL2>(o + e);
+      }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float w = sc.wt[(j + u) * 8 + r];
-          acc[q2].x = fmaf(w, v[u].x, acc[q2].x);
-          acc[q2].y = fmaf(w, v[u].y, acc[q2].y);
-          acc[q2].z = fmaf(w, v[u].z, acc[q2].z);
-          acc[q2].w = fmaf(w, v[u].w, acc[q2].w);
+      for (int x = 0; x < 8; ++x) {
+        const int e = x * 32 + lane;
+        if (e < nquad) {
+          const float w = wt[j * 8 + e / QD];
+          acc[x].x = fmaf(w, v[x].x, acc[x].x);
+          acc[x].y = fmaf(w, v[x].y, acc[x].y);
+          acc[x].z = fmaf(w, v[x].z, acc[x].z);
+          acc[x].w = fmaf(w, v[x].w, acc[x].w);
         }
       }
-      for (; j < cnt; ++j) {
-        const float4 v = ld_rec<kL2>(reinterpret_cast<const float4*>(piece(j0 + j) + 64) + e);
-        const float w = sc.wt[j * 8 + r];
-        acc[q2].x = fmaf(w, v.x, acc[q2].x);
-        acc[q2].y = fmaf(w, v.y, acc[q2].y);
-        acc[q2].z = fmaf(w, v.z, acc[q2].z);
-        acc[q2].w = fmaf(w, v.w, acc[q2].w);
-      }
     }
-    __syncthreads();                              // the tables are refilled by the next chunk
+    __syncwarp();                                 // the weights are refilled by the next chunk
   }
 #pragma unroll
-  for (int q2 = 0; q2 < 2; ++q2) {
-    const int e = tid + q2 * nt;
+  for (int x = 0; x < 8; ++x) {
+    const int e = x * 32 + lane;
     if (e >= nquad) continue;
     const int r = e / QD, q4 = e - r * QD;
     if (dst == nullptr) {
-      const float inv = 1.f / sc.L[r];
-      const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc[q2].x * inv)) |
-                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[q2].y * inv)) << 16);
-      const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc[q2].z * inv)) |
-                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[q2].w * inv)) << 16);
+      const float inv = 1.f / L[r];
+      const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].x * inv)) |
+                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].y * inv)) << 16);
+      const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].z * inv)) |
+                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].w * inv)) << 16);
       const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
       reinterpret_cast<uint2*>(p.out + row * D)[q4] = make_uint2(lo, hi);
     } else {
-      reinterpret_cast<float4*>(dst + 64)[e] = acc[q2];
+      reinterpret_cast<float4*>(dst + 64)[e] = acc[x];
     }
   }
-  if (dst != nullptr && tid < Gq) reinterpret_cast<float2*>(dst)[tid] = make_float2(sc.M[tid], sc.L[tid]);
+  if (dst != nullptr && lane < Gq) reinterpret_cast<float2*>(dst)[lane] = make_float2(M[lane], L[lane]);
   if (k > 0) {
-    // warps 2.. take one head each (their p-transpose buffers stage the lists)
     const bool all = dst == nullptr && p.live_count[__ldg(p.seq + i)] <= k;
-    const int tkw = nwarps - 2;
-    if (warp >= 2) {
-      float* stage = reinterpret_cast<float*>(sc.pbuf0 + (size_t)warp * sc.warp_smem);
-      const int per = (kPbufBytes / 4) / kpad;      // lists one staging pass holds
-      for (int r = warp - 2; r < Gq; r += tkw) {
-        if (all) {
-          if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + r] = 1.f;
-          continue;
-        }
-        // running list (descending) in elements 0..63, the next piece's list
-        // reversed in 64..127: a bitonic sequence
-        float tv[4];
+    float* stage = wb + 176;
+    const int per = (704 - 176) / kpad;            // lists one staging pass holds
+    for (int r = 0; r < Gq; ++r) {
+      if (all) {
+        if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + r] = 1.f;
+        continue;
+      }
+      // running list (descending) in elements 0..63, the next piece's list
+      // reversed in 64..127: a bitonic sequence
+      float tv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
-        for (int j0 = 0; j0 < np; j0 += per) {
-          const int cnt = min(per, np - j0);
-          __syncwarp();
-          for (int x = lane; x < cnt * kpad; x += 32) {
-            const int j = x / kpad, m = x - j * kpad;
-            stage[x] = ld_rec<kL2>(reinterpret_cast<const float*>(piece(j0 + j) + 64 + 4 * Gq * D) +
-                                   r * kpad + m);
+      for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
+      for (int j0 = 0; j0 < np; j0 += per) {
+        const int cnt = min(per, np - j0);
+        __syncwarp();
+        for (int x = lane; x < cnt * kpad; x += 32) {
+          const int j = x / kpad, m = x - j * kpad;
+          stage[x] = ld_rec<kL2>(reinterpret_cast<const float*>(piece(j0 + j) + 64 + 4 * Gq * D) +
+                                 r * kpad + m);
+        }
+        __syncwarp();
+        for (int j = 0; j < cnt; ++j) {
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int el = lane * 4 + e, m = 127 - el;
+            v[e] = el < 64 ? tv[e] : (m < k ? stage[j * kpad + m] : -INFINITY);
           }
-          __syncwarp();
-          for (int j = 0; j < cnt; ++j) {
-            float v[4];
+          bitonic128_merge_desc(v);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int el = lane * 4 + e, m = 127 - el;
-              v[e] = el < 64 ? tv[e] : (m < k ? stage[j * kpad + m] : -INFINITY);
-            }
-            bitonic128_merge_desc(v);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) tv[e] = v[e];
-          }
+          for (int e = 0; e < 4; ++e) tv[e] = v[e];
         }
-        if (dst == nullptr) {
-          float sum = 0.f;
+      }
+      if (dst == nullptr) {
+        float sum = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (lane * 4 + e < k) sum += exp2_approx(tv[e] - sc.M[r]);
+        for (int e = 0; e < 4; ++e)
+          if (lane * 4 + e < k) sum += exp2_approx(tv[e] - M[r]);
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-          if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + r] = sum / sc.L[r];
-        } else {
-          float* tl = reinterpret_cast<float*>(dst + 64 + 4 * Gq * D) + r * kpad;
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + r] = sum / L[r];
+      } else {
+        float* tl = reinterpret_cast<float*>(dst + 64 + 4 * Gq * D) + r * kpad;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (lane * 4 + e < kpad) tl[lane * 4 + e] = tv[e];
-        }
+        for (int e = 0; e < 4; ++e)
+          if (lane * 4 + e < kpad) tl[lane * 4 + e] = tv[e];
       }
     }
   }
-  __syncthreads();                                // scratch free for the next merge
+  __syncwarp();
 }
 
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks) decode_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int wsum[kDecWarps];
-  __shared__ int s_first[kDecWarps], s_last[kDecWarps];   // each warp's first / last segment
-  __shared__ int s_segs[2 * kDecWarps], s_nsegs;           // the CTA's split segments
+  __shared__ int s_last[kDecWarps];                // each warp's last segment
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NW = p.nw, NT = NW * 32;
   int32_t* P = reinterpret_cast<int32_t*>(smem);      // [n + 1] prefix of live pages
@@ -1246,104 +1227,72 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks) decode_kernel(Deco
       seg_end<D, G>(S, p, seg, tk, (Us >= U0 && Ue <= U1) ? nullptr : wsm);
     }
   }
-  if (lane == 0) {
-    s_first[warp] = first_seg;
-    s_last[warp] = last_seg;
-  }
+  if (lane == 0) s_last[warp] = last_seg;
   __syncthreads();
 
-  // ---- merges, the whole CTA at a time: the CTA's split segments in order
-  //      (a segment not whole in one warp); one inside the CTA is written
-  //      out, one that spans CTAs becomes the CTA's piece, and the CTA that
-  //      brings the segment's arrival count to its number of CTAs merges
-  //      those pieces ----
-  MergeScratch sc;
-  {
-    uint8_t* pb0 = smem + p.plan_smem + p.nstage * p.stage_bytes + 64;   // warp 0's p buffer
-    const int ws = p.warp_smem;
-    sc.pbuf0 = pb0;
-    sc.warp_smem = ws;
-    sc.wl = reinterpret_cast<float*>(pb0);
-    sc.wt = reinterpret_cast<float*>(pb0 + ws);
-    sc.mk = reinterpret_cast<int*>(pb0 + ws + 1024);
-    sc.M = reinterpret_cast<float*>(pb0 + ws + 1056);
-    sc.L = reinterpret_cast<float*>(pb0 + ws + 1088);
-    sc.flag = reinterpret_cast<int*>(pb0 + ws + 1120);
-    sc.list = reinterpret_cast<int*>(pb0 + ws + 1136);
-  }
-  auto whole_in_warp = [&](int S, int w) {
+  // ---- merges: the last warp of this CTA that touches a split segment merges
+  //      the warps' pieces; a segment spanning CTAs goes through the CTA records ----
+  if (U0 >= U1) return;
+  float* wbuf = pbuf;                              // the warp's 704-float merge scratch
+  int* list = reinterpret_cast<int*>(pbuf) + 16;   // up to 160 piece owners
+  for (int which = 0; which < 2; ++which) {
+    const int S = which == 0 ? first_seg : last_seg;
+    if (which == 0 && first_seg == last_seg) continue;   // one segment: handled as the last
     int64_t Us, Ue;
     seg_range(p, P, S / p.Hkv, S % p.Hkv, &Us, &Ue);
-    const int64_t a0 = U0c + w * nuc / NW, a1 = U0c + (w + 1) * nuc / NW;
-    return Us >= a0 && Ue <= a1;
-  };
-  if (tid == 0) {
-    int ns = 0, prev = -1;
-    for (int w = 0; w < NW; ++w) {
-      const int f = s_first[w], l = s_last[w];
-      if (l < 0) continue;                         // no units
-      if (f != l && !whole_in_warp(f, w) && f != prev) s_segs[ns++] = prev = f;
-      if (!whole_in_warp(l, w) && l != prev) s_segs[ns++] = prev = l;
-    }
-    s_nsegs = ns;
-  }
-  __syncthreads();
-  const int nsegs = s_nsegs;
-  for (int kseg = 0; kseg < nsegs; ++kseg) {
-    const int S = s_segs[kseg];
-    int64_t Us, Ue;
-    seg_range(p, P, S / p.Hkv, S % p.Hkv, &Us, &Ue);
-    if (tid == 0) {                                // the warps holding S's pieces
-      const int64_t wf = share_of_unit(max(Us, U0c) - U0c, nuc, NW);
-      const int64_t wl = share_of_unit(min(Ue, U1c) - 1 - U0c, nuc, NW);
-      int n = 0;
-      for (int wj = (int)wf; wj <= (int)wl; ++wj)
-        if (U0c + (int64_t)wj * nuc / NW < U0c + (int64_t)(wj + 1) * nuc / NW) sc.list[n++] = wj;
-      sc.flag[0] = n;
-    }
-    __syncthreads();
-    const int npw = sc.flag[0];
+    if (Us >= U0 && Ue <= U1) continue;            // whole in this warp: already written
+    // the last warp touching S merges: S ends in this warp, or this is the
+    // CTA's last warp with units
+    const int64_t wlast = share_of_unit(min(Ue, U1c) - 1 - U0c, nuc, NW);
+    if (wlast != warp) continue;
+    const int64_t wfirst = share_of_unit(max(Us, U0c) - U0c, nuc, NW);
+    // the warps in [wfirst, warp] that hold units (shares can be empty when
+    // the CTA has fewer units than warps)
+    int npw = 0;
+    for (int wj = (int)wfirst; wj <= warp; ++wj)
+      if (U0c + (int64_t)wj * nuc / NW < U0c + (int64_t)(wj + 1) * nuc / NW) {
+        if (lane == 0) list[npw] = wj;
+        ++npw;
+      }
+    __syncwarp();
     auto warp_piece = [&](int j) -> const uint8_t* {
-      const int wj = sc.list[j];
+      const int wj = list[j];
       // a warp's piece of S sits in its ring if S was its last segment
       return s_last[wj] == S ? smem + p.plan_smem + wj * p.warp_smem
                              : p.wrec + ((int64_t)cta * NW + wj) * p.rb;
     };
     const bool in_cta = Us >= U0c && Ue <= U1c;
-    // the CTA's piece of S: slot 0 if S holds the CTA's first unit, else slot 1
-    uint8_t* mine = in_cta ? nullptr : p.crec + ((int64_t)cta * 2 + (Us <= U0c ? 0 : 1)) * p.rb;
-    cta_merge<D, false>(p, S, npw, warp_piece, mine, sc);
-    if (in_cta) continue;
-    __threadfence();
-    __syncthreads();
-    if (warp == 0) {
-      // the CTAs holding units of S (empty shares skipped)
-      const int64_t ca = share_of_unit(Us, T, C), cb = share_of_unit(Ue - 1, T, C);
-      int ncta = 0;
-      for (int64_t c0 = ca; c0 <= cb; c0 += 32) {
-        const int64_t cj = c0 + lane;
-        const bool has = cj <= cb && cj * T / C < (cj + 1) * T / C;
-        const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
-        if (has) sc.list[ncta + __popc(bal & ((1u << lane) - 1u))] = (int)cj;
-        ncta += __popc(bal);
-      }
-      if (lane == 0) {
-        // wraps to 0 on the last arrival
-        const uint32_t old = atomicInc(p.cnt + S, (uint32_t)ncta - 1u);
-        sc.flag[1] = old == (uint32_t)ncta - 1u;
-        sc.flag[2] = ncta;
-      }
+    if (in_cta) {
+      merge_pieces<D, false>(p, S, npw, warp_piece, nullptr, wbuf);
+      continue;
     }
-    __syncthreads();
-    if (sc.flag[1] == 0) continue;
+    // the CTA's piece of S: slot 0 if S holds the CTA's first unit, else slot 1
+    uint8_t* mine = p.crec + ((int64_t)cta * 2 + (Us <= U0c ? 0 : 1)) * p.rb;
+    merge_pieces<D, false>(p, S, npw, warp_piece, mine, wbuf);
+    __threadfence();
+    __syncwarp();
+    // the CTAs holding units of S (empty shares skipped)
+    const int64_t ca = share_of_unit(Us, T, C), cb = share_of_unit(Ue - 1, T, C);
+    int ncta = 0;
+    for (int64_t c0 = ca; c0 <= cb; c0 += 32) {
+      const int64_t cj = c0 + lane;
+      const bool has = cj <= cb && cj * T / C < (cj + 1) * T / C;
+      const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
+      if (has) list[ncta + __popc(bal & ((1u << lane) - 1u))] = (int)cj;
+      ncta += __popc(bal);
+    }
+    uint32_t old = 0;
+    if (lane == 0) old = atomicInc(p.cnt + S, (uint32_t)ncta - 1u);   // wraps to 0 on the last arrival
+    old = __shfl_sync(0xFFFFFFFFu, old, 0);
+    if (old != (uint32_t)ncta - 1u) continue;
     __threadfence();                               // the other CTAs' records are visible now
-    const int ncta = sc.flag[2];
+    __syncwarp();
     auto cta_piece = [&](int j) -> const uint8_t* {
-      const int64_t cj = sc.list[j];
+      const int64_t cj = list[j];
       const int64_t u0j = cj * T / C;
       return p.crec + (cj * 2 + (Us <= u0j ? 0 : 1)) * p.rb;
     };
-    cta_merge<D, true>(p, S, ncta, cta_piece, nullptr, sc);
+    merge_pieces<D, true>(p, S, ncta, cta_piece, nullptr, wbuf);
   }
 }
 
