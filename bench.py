@@ -119,8 +119,8 @@ def traffic_per_launch(workload: str):
 
 def launches_per_step(batch: int) -> int:
     """Kernels one step launches: append (one launch up to 512 tokens, else
-    two), evict, decode (one kernel)."""
-    return (1 if batch <= 512 else 2) + 1 + 1
+    two), evict, decode (split + combine)."""
+    return (1 if batch <= 512 else 2) + 1 + 2
 
 
 def algorithmic_decode_bytes(w, snap) -> int:
@@ -598,7 +598,7 @@ def roofline_block(w, res):
             "algorithmic_bytes_per_launch": res["alg_bytes"], "live_pages": res["pages"]}
 
 
-DECODE_KERNELS = "decode call: decode_kernel (one launch)"
+DECODE_KERNELS = "decode call: decode_split_kernel + decode_combine_kernel"
 
 
 def thinkv_arm(args, w, world, rank, local):

@@ -353,14 +353,10 @@ THINKV_API size_t thinkv_decode_workspace_bytes(const thinkv_layout* L, int32_t 
  * probability held by the topk (1..64) most probable live tokens (1 when the
  * sequence has <= topk live tokens, 0 when it has none).
  * workspace: device, >= thinkv_decode_workspace_bytes(L, n_seqs, topk) bytes,
- * caller-owned scratch for the split-K partial results.  It starts with one
- * arrival counter per (sequence, kv-head): zero-fill the workspace once
- * before its first use; every call that completes leaves the counters zero
- * (after a call that set THINKV_ERR_TIMEOUT, zero-fill it again).  Calls that
- * share a workspace must not overlap on the GPU.
- * One kernel runs per call: each SM takes an equal share of the live
- * page-heads; a (sequence, kv-head) whose pages fall to several SMs is merged
- * by the last of them to finish.
+ * caller-owned scratch for the split-K partial results; its contents need no
+ * initialisation.  Calls that share a workspace must not overlap on the GPU.
+ * Two kernels run per call: the split kernel over the live page-heads and the
+ * combine of the segments it left in several pieces.
  * 1 <= n_seqs <= 16384. */
 THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs, const int32_t* seq,
                             const uint16_t* q, uint16_t* out, float* topk_mass,
@@ -379,8 +375,7 @@ THINKV_API int thinkv_decode_attention(const thinkv_cache* cache, int32_t n_seqs
  * this is an interface convenience of this library.)
  * The split-K scratch lives in one file-scope device array of
  * THINKV_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
- * until the process exits.  Each call clears the array's arrival counters on
- * `stream` (cudaMemsetAsync) before its kernel.  A call whose scratch need (what
+ * until the process exits.  A call whose scratch need (what
  * thinkv_decode_workspace_bytes reports for the same n_seqs and topk) exceeds
  * that size returns THINKV_ERR_WORKSPACE before launching anything.
  * The first call on a device looks up the array's device address (once per

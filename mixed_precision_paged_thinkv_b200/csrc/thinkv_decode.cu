@@ -7,29 +7,25 @@
 // "Implementation Systeme: Pensee Continue (CT)").  The pages print no kernel
 // design; this one is written for sm_100a:
 //
-//   One kernel per call.  The live page-heads of all decoded sequences form one
-//   ordered list of units (sequence, kv-head, live page), segment by segment.
-//   The grid has one CTA of 12 warps per SM; CTA c takes an equal contiguous
-//   share of the units (stream-K at CTA level), and its warps split that
-//   share into equal contiguous sub-ranges, so work is balanced by live pages
-//   however lengths and budgets vary.  Per warp, lane 0 streams page-head
+//   split kernel (stream-K): the live page-heads of all decoded sequences form
+//   one ordered list of units (sequence, kv-head, live page); every warp of the
+//   grid takes an equal contiguous share, so work is balanced by live pages no
+//   matter how lengths and budgets vary.  Per warp, lane 0 streams page-head
 //   blocks (K codes, V codes, params: one contiguous block per page and head)
-//   into a shared-memory ring with cp.async.bulk (TMA) + mbarriers, every
-//   stage issued at once when the warp starts; the warp unpacks codes straight
-//   into mma.sync m16n8k16 operands (byte-permute conversion to fp16 1024 +
-//   code), computes q.k for the whole GQA group at once (tokens x heads),
-//   applies the per-group scale/zero in fp32, runs the online softmax,
-//   transposes p through a small shared buffer and accumulates p*scale (fp16,
-//   exponent-shifted) times the centred V codes on the tensor cores, with the
-//   zero terms summed in fp32.
+//   into a shared-memory ring with cp.async.bulk (TMA) + mbarriers; the warp
+//   unpacks codes straight into mma.sync m16n8k16 operands (byte-permute
+//   conversion to fp16 1024 + code), computes q.k for the whole GQA group at
+//   once (tokens x heads), applies the per-group scale/zero in fp32, runs the
+//   online softmax, transposes p through a small shared buffer and accumulates
+//   p*scale (fp16, exponent-shifted) times the centred V codes on the tensor
+//   cores, with the zero terms summed in fp32.  A segment (sequence, kv-head)
+//   that lies wholly in one warp is written out at once; otherwise each warp
+//   writes one piece record (m, l, o, top-k logits) per segment it touched.
 //
-//   A segment (sequence, kv-head) that lies wholly in one warp is written out
-//   at once.  The others leave one piece (m, l, o, top-k logits) per warp;
-//   after the loop the CTA merges the pieces of each of its segments with the
-//   log-sum-exp rule (a warp per segment).  A segment that spans CTAs leaves
-//   one piece per CTA in global memory; the last CTA to finish its piece
-//   (a self-resetting arrival counter per segment) merges them and writes O
-//   and the top-k mass.  Nothing waits on another CTA.
+//   combine kernel (launched right behind, programmatic dependent launch): one
+//   CTA per segment left in several pieces merges the records with the
+//   log-sum-exp rule -- a thread per quad of each head's output row, a warp per
+//   head for the top-k lists -- and writes fp16 O and the top-k mass.
 #include <cuda_fp16.h>
 #include <limits.h>
 #include <mutex>
@@ -42,14 +38,15 @@ namespace thinkv {
 
 namespace {
 
-constexpr int kDecWarps = 12;                          // most warps per CTA (the plan may use fewer)
+constexpr int kDecWarps = 4;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecMinBlocks = 1;                       // CTAs per SM the kernel is built for
-constexpr int kPrefixPer = 4;                          // sequences per thread and prefix pass
+constexpr int kDecMinBlocks = 3;                       // CTAs per SM the kernel is built for
+constexpr int kDecRegs = 65536 / (kDecThreads * kDecMinBlocks) / 8 * 8;  // register cap (168)
 constexpr int kPbufStride = 12;                 // floats per row of the p transpose buffer
 // per-warp scratch: during pages, the p transpose (16 x 12 floats) and the
-// segment's Q fragments (lane-contiguous, up to 2 KB); during a merge, after
-// the loop, the weights of 32 pieces x 8 heads and the heads' M and L
+// segment's Q fragments (lane-contiguous, up to 2 KB); during a merge, which
+// runs between two segments, the (m, l) table of the pieces (32 x 8 float2 +
+// 16 floats) overlays both
 constexpr int kPtBytes = 16 * kPbufStride * 4;          // 768
 constexpr int kQfragOff = kPtBytes;
 constexpr int kQfragBytes = 2048;                       // (D / 16) k-steps x 32 lanes x 8 B
@@ -72,16 +69,14 @@ struct DecodeParams {
   int32_t n;
   const uint16_t* q;
   float scale_log2;
-  uint32_t* cnt;     // [n * Hkv] arrival counters of segments spanning CTAs (zero between calls)
-  uint8_t* wrec;     // [grid][nw] piece of each warp's first segment, when it is split
-  uint8_t* crec;     // [grid][2] piece of each CTA's first / last segment, when it spans CTAs
-  int32_t rb;        // bytes of one piece record
+  void* rec;         // piece records of split segments (index warp + segment)
+  int32_t* pref;      // [n + 1] prefix of live pages over the call's sequences
+  int64_t split_warps;  // warps of the split kernel's grid
   const int32_t* live_count;
   uint16_t* out;     // [n][Hq][D]
   float* mass;       // [n][Hq] or null
   int32_t topk;
   int32_t* status;
-  int32_t nw;        // warps per CTA (blockDim.x / 32)
   int32_t nstage, stage_bytes, warp_smem, plan_smem;
   int32_t q_off, q_bytes;  // Q rows of a segment ride with its first page: stage + q_off
 };
@@ -379,23 +374,22 @@ __device__ inline void seg_range(const DecodeParams& p, const int32_t* P, int i,
   *Ue = *Us + nl;
 }
 
-// Which of W equal contiguous shares of [0, T) (share w holds [w*T/W,
-// (w+1)*T/W)) holds unit u < T.
-__device__ inline int64_t share_of_unit(int64_t u, int64_t T, int64_t W) {
+// The warp of the stream-K split (warp w holds units [w*T/W, (w+1)*T/W))
+// that holds unit u.
+__device__ inline int64_t warp_of_unit(int64_t u, int64_t T, int64_t W) {
   return ((u + 1) * W - 1) / T;
 }
 
-// Ends the warp's work on segment seg = i * Hkv + h.  With piece == null the
-// whole segment was in this warp: its O rows and top-k mass are written at
-// once.  Otherwise the warp's piece record (m, l, unnormalised o, sorted top-k
-// logits) is written at `piece` (shared or global memory) for the merge.
+// Ends the warp's work on segment seg = i * Hkv + h.  If the whole segment
+// was in this warp (Us >= U0 and Ue <= U1) its O rows and top-k mass are
+// written at once; otherwise the warp's piece record goes to rec[w + seg]
+// for the merge.
 template <int D, int G>
-__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int seg,
-                               const TopkCtx& tk, uint8_t* piece) {
+__device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t w, int seg,
+                               const TopkCtx& tk, bool whole) {
   constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int i = seg / p.Hkv, h = seg - (seg / p.Hkv) * p.Hkv;
-  const bool whole = piece == nullptr;
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     S.lp[0] += __shfl_xor_sync(0xFFFFFFFFu, S.lp[0], o);
@@ -408,13 +402,15 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int seg
   }
   const int Gq = p.Gq;
   const float sinv = pow2i(-S.sigma);
-  float* po = whole ? nullptr : reinterpret_cast<float*>(piece + 64);
+  const int64_t rb = record_bytes(Gq, D, tk.topk);
+  uint8_t* rec = reinterpret_cast<uint8_t*>(p.rec) + (w + seg) * rb;
+  float* po = reinterpret_cast<float*>(rec + 64);
   const float li0 = whole ? 1.f / S.lp[0] : 1.f, li1 = whole ? 1.f / S.lp[1] : 1.f;
   if (!whole && g == 0) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int hd = 2 * t + c;
-      if (hd < Gq) reinterpret_cast<float2*>(piece)[hd] = make_float2(S.m[c], S.lp[c]);
+      if (hd < Gq) reinterpret_cast<float2*>(rec)[hd] = make_float2(S.m[c], S.lp[c]);
     }
   }
 #pragma unroll
@@ -435,8 +431,8 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int seg
   }
   if (tk.topk > 0) {
     const int kpad = (tk.topk + 3) / 4 * 4;
-    const bool all = whole && p.live_count[__ldg(p.seq + i)] <= tk.topk;
-    float* tl = whole ? nullptr : reinterpret_cast<float*>(piece + 64 + 4 * Gq * D);
+    const bool all = whole && p.live_count[p.seq[i]] <= tk.topk;
+    float* tl = reinterpret_cast<float*>(rec + 64 + 4 * Gq * D);
     for (int hd = 0; hd < Gq; ++hd) {
       float sum = 0.f;
       if (!all) {
@@ -824,23 +820,6 @@ struct UnitMeta {
   uint32_t mask;
 };
 
-// Call index i whose units hold unit u (P: prefix of live pages, n + 1 entries).
-__device__ inline int seq_of_unit(const DecodeParams& p, const int32_t* P, int64_t u) {
-  int lo = 0, hi = p.n;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if ((int64_t)P[mid] * p.Hkv <= u) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
-// Segment (i * Hkv + h) of unit u.
-__device__ inline int seg_of_unit(const DecodeParams& p, const int32_t* P, int64_t u) {
-  const int i = seq_of_unit(p, P, u);
-  const int nl = P[i + 1] - P[i];
-  return i * p.Hkv + (int)((u - (int64_t)P[i] * p.Hkv) / nl);
-}
-
 __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P, int64_t u,
                                         int64_t U1) {
   UnitMeta m;
@@ -848,11 +827,16 @@ __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P,
   m.cls_seg = 0;
   m.mask = 0;
   if (u >= U1) return m;
-  const int i = seq_of_unit(p, P, u);
+  int lo = 0, hi = p.n;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)P[mid] * p.Hkv <= u) lo = mid; else hi = mid;
+  }
+  const int i = lo;
   const int nl = P[i + 1] - P[i];
   const int rel = (int)(u - (int64_t)P[i] * p.Hkv);   // < Hkv * max_blocks_per_seq < 2^31
   const int h = rel / nl, j = rel - h * nl;
-  const int64_t row = (int64_t)__ldg(p.seq + i) * p.max_blocks;
+  const int64_t row = (int64_t)P[p.n + 1 + i] * p.max_blocks;   // the sequence id, cached
   const uint64_t desc = p.live_list[row + j];       // page | class << 32 | entry << 40
   const int cls = entry_class(desc);
   const uint64_t src = reinterpret_cast<uint64_t>(p.pool[cls]) +
@@ -864,222 +848,33 @@ __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P,
   return m;
 }
 
-// ---------------------------------------------------------------------------
-// merging the pieces of one segment (the whole CTA)
-// ---------------------------------------------------------------------------
-// Loads of piece records: records written by other CTAs are read through L2
-// (kL2); the CTA's own records (shared memory, or global memory written by
-// its warps before a __syncthreads) with ordinary loads.
-template <bool kL2, typename T>
-__device__ __forceinline__ T ld_rec(const T* ptr) {
-  if constexpr (kL2) return __ldcg(ptr);
-  else return *ptr;
-}
-
-// Merges np piece records of segment `seg` with the log-sum-exp rule (one
-// warp): per head, M = max m_j, L = sum l_j 2^(m_j - M), o = sum o_j
-// 2^(m_j - M), and the top-k logits of all pieces merged into one sorted
-// list.  If dst is null the result is final: O = o / L in fp16 and the top-k
-// mass are written out.  Otherwise the merged piece is written at dst (a
-// record, for a later merge).  `piece(j)` gives the address of record j.
-// Written for few memory round trips: the (m, l) pairs of up to 16 pieces
-// are requested at once into a shared table, every lane requests all its
-// output quads of a piece at once, and each head's top-k lists are staged in
-// shared memory with one pass of loads before the bitonic merges.
-// wb: this warp's 704-float scratch: M[8], L[8], ints [16, 176) for the
-// caller's piece list, the table at [176, 432), weights at [432, 560); the
-// top-k staging reuses [176, 704).
-template <int D, bool kL2, typename PieceFn>
-__device__ void merge_pieces(const DecodeParams& p, int seg, int np, PieceFn piece, uint8_t* dst,
-                             float* wb) {
-  const int lane = threadIdx.x & 31;
-  const int Gq = p.Gq, k = p.topk, kpad = (k + 3) / 4 * 4;
-  const int i = seg / p.Hkv, h = seg - (seg / p.Hkv) * p.Hkv;
-  constexpr int CH = 16;                          // pieces per table chunk
-  float* M = wb;
-  float* L = wb + 8;
-  float2* tbl = reinterpret_cast<float2*>(wb + 176);
-  float* wt = wb + 432;
-  auto load_table = [&](int j0, int cnt) {
-    for (int x = lane; x < cnt * Gq; x += 32) {
-      const int j = x / Gq, r = x - j * Gq;
-      tbl[j * 8 + r] = ld_rec<kL2>(reinterpret_cast<const float2*>(piece(j0 + j)) + r);
-    }
-    __syncwarp();
-  };
-  // maxima (one chunk: the table stays for the weights)
-  if (lane < 8) {
-    M[lane] = -INFINITY;
-    L[lane] = 0.f;
-  }
-  for (int j0 = 0; j0 < np; j0 += CH) {
-    load_table(j0, min(CH, np - j0));
-    if (lane < Gq) {
-      float m = M[lane];
-      for (int j = 0; j < min(CH, np - j0); ++j) m = fmaxf(m, tbl[j * 8 + lane].x);
-      M[lane] = m;
-    }
-    __syncwarp();
-  }
-  constexpr int QD = D / 4;
-  const int nquad = Gq * QD;                      // <= 256: at most 8 quads per lane
-  float4 acc[8];
-#pragma unroll
-  for (int x = 0; x < 8; ++x) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j0 = 0; j0 < np; j0 += CH) {
-    const int cnt = min(CH, np - j0);
-    if (np > CH) load_table(j0, cnt);             // else the table is still there
-    if (lane < Gq) {                              // weights, and L in a fixed order
-      float l = L[lane];
-      for (int j = 0; j < cnt; ++j) {
-        const float2 ml = tbl[j * 8 + lane];
-        const float w = ml.x == -INFINITY ? 0.f : exp2_approx(ml.x - M[lane]);
-        wt[j * 8 + lane] = w;
-        l = fmaf(w, ml.y, l);
-      }
-      L[lane] = l;
-    }
-    __syncwarp();
-    for (int j = 0; j < cnt; ++j) {               // a piece's quads all in flight
-      const float4* o = reinterpret_cast<const float4*>(piece(j0 + j) + 64);
-      float4 v[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int e = x * 32 + lane;
-        if (e < nquad) v[x] = ld_rec<kL2>(o + e);
-      }
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int e = x * 32 + lane;
-        if (e < nquad) {
-          const float w = wt[j * 8 + e / QD];
-          acc[x].x = fmaf(w, v[x].x, acc[x].x);
-          acc[x].y = fmaf(w, v[x].y, acc[x].y);
-          acc[x].z = fmaf(w, v[x].z, acc[x].z);
-          acc[x].w = fmaf(w, v[x].w, acc[x].w);
-        }
-      }
-    }
-    __syncwarp();                                 // the weights are refilled by the next chunk
-  }
-#pragma unroll
-  for (int x = 0; x < 8; ++x) {
-    const int e = x * 32 + lane;
-    if (e >= nquad) continue;
-    const int r = e / QD, q4 = e - r * QD;
-    if (dst == nullptr) {
-      const float inv = 1.f / L[r];
-      const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].x * inv)) |
-                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].y * inv)) << 16);
-      const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc[x].z * inv)) |
-                          ((uint32_t)__half_as_ushort(__float2half_rn(acc[x].w * inv)) << 16);
-      const int64_t row = (int64_t)i * p.Hq + h * Gq + r;
-      reinterpret_cast<uint2*>(p.out + row * D)[q4] = make_uint2(lo, hi);
-    } else {
-      reinterpret_cast<float4*>(dst + 64)[e] = acc[x];
-    }
-  }
-  if (dst != nullptr && lane < Gq) reinterpret_cast<float2*>(dst)[lane] = make_float2(M[lane], L[lane]);
-  if (k > 0) {
-    const bool all = dst == nullptr && p.live_count[__ldg(p.seq + i)] <= k;
-    float* stage = wb + 176;
-    const int per = (704 - 176) / kpad;            // lists one staging pass holds
-    for (int r = 0; r < Gq; ++r) {
-      if (all) {
-        if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + r] = 1.f;
-        continue;
-      }
-      // running list (descending) in elements 0..63, the next piece's list
-      // reversed in 64..127: a bitonic sequence
-      float tv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
-      for (int j0 = 0; j0 < np; j0 += per) {
-        const int cnt = min(per, np - j0);
-        __syncwarp();
-        for (int x = lane; x < cnt * kpad; x += 32) {
-          const int j = x / kpad, m = x - j * kpad;
-          stage[x] = ld_rec<kL2>(reinterpret_cast<const float*>(piece(j0 + j) + 64 + 4 * Gq * D) +
-                                 r * kpad + m);
-        }
-        __syncwarp();
-        for (int j = 0; j < cnt; ++j) {
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int el = lane * 4 + e, m = 127 - el;
-            v[e] = el < 64 ? tv[e] : (m < k ? stage[j * kpad + m] : -INFINITY);
-          }
-          bitonic128_merge_desc(v);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) tv[e] = v[e];
-        }
-      }
-      if (dst == nullptr) {
-        float sum = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (lane * 4 + e < k) sum += exp2_approx(tv[e] - M[r]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + r] = sum / L[r];
-      } else {
-        float* tl = reinterpret_cast<float*>(dst + 64 + 4 * Gq * D) + r * kpad;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (lane * 4 + e < kpad) tl[lane * 4 + e] = tv[e];
-      }
-    }
-  }
-  __syncwarp();
-}
-
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks) decode_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+    decode_split_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int wsum[kDecWarps];
-  __shared__ int s_last[kDecWarps];                // each warp's last segment
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NW = p.nw, NT = NW * 32;
   int32_t* P = reinterpret_cast<int32_t*>(smem);      // [n + 1] prefix of live pages
+  int32_t* Sq = P + (p.n + 1);                         // [n] the call's sequence ids
   pdl_launch_dependents();
   // the call's own inputs may be read before the previous kernel has finished
-  int sv[kPrefixPer];
-#pragma unroll
-  for (int e = 0; e < kPrefixPer; ++e) {
-    const int i = tid * kPrefixPer + e;
-    sv[e] = i < p.n ? __ldg(p.seq + i) : -1;
-  }
+  for (int i = tid; i < p.n; i += kDecThreads) Sq[i] = p.seq[i];
   // everything below reads cache state: wait for the previous kernel
   pdl_wait();
+  __syncthreads();
 
-  // ---- prefix of live pages over the call's sequences (per CTA; each
-  //      thread takes kPrefixPer consecutive sequences of a pass) ----
+  // ---- prefix of live pages over the call's sequences (per CTA) ----
   {
+    __shared__ int wsum[kDecWarps];
     int carry = 0;
-    for (int base = 0; base < p.n; base += NT * kPrefixPer) {
-      if (base > 0) {
-#pragma unroll
-        for (int e = 0; e < kPrefixPer; ++e) {
-          const int i = base + tid * kPrefixPer + e;
-          sv[e] = i < p.n ? __ldg(p.seq + i) : -1;
-        }
+    for (int base = 0; base < p.n; base += kDecThreads) {
+      const int i = base + tid;
+      int v = 0;
+      if (i < p.n) {
+        const int s = Sq[i];
+        if (s >= 0 && s < p.max_seqs) v = p.num_live[s];
+        else if (blockIdx.x == 0) set_status(p.status, THINKV_ERR_INVALID);  // decoded as empty
       }
-      int v[kPrefixPer];
-#pragma unroll
-      for (int e = 0; e < kPrefixPer; ++e) {
-        const int i = base + tid * kPrefixPer + e;
-        v[e] = 0;
-        if (i < p.n) {
-          const int s = sv[e];
-          if (s >= 0 && s < p.max_seqs) v[e] = p.num_live[s];
-          else if (blockIdx.x == 0) set_status(p.status, THINKV_ERR_INVALID);  // decoded as empty
-        }
-      }
-      int tsum = 0;
-#pragma unroll
-      for (int e = 0; e < kPrefixPer; ++e) tsum += v[e];
-      int x = tsum;
+      int x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
@@ -1087,31 +882,26 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks) decode_kernel(Deco
       }
       if (lane == 31) wsum[warp] = x;
       __syncthreads();
-      int before = carry, tot = 0;
-      for (int w = 0; w < NW; ++w) {
-        before += w < warp ? wsum[w] : 0;
-        tot += wsum[w];
-      }
-      int run = before + x - tsum;
-#pragma unroll
-      for (int e = 0; e < kPrefixPer; ++e) {
-        const int i = base + tid * kPrefixPer + e;
-        if (i < p.n) P[i] = run;
-        run += v[e];
-      }
+      int before = carry;
+      for (int w = 0; w < warp; ++w) before += wsum[w];
+      if (i < p.n) P[i] = before + x - v;
+      int tot = 0;
+      for (int w = 0; w < kDecWarps; ++w) tot += wsum[w];
       carry += tot;
       __syncthreads();
     }
     if (tid == 0) P[p.n] = carry;
     __syncthreads();
   }
+  if (blockIdx.x == 0)
+    for (int x = tid; x <= p.n; x += kDecThreads) p.pref[x] = P[x];   // for the combine
   write_empty_outputs(p, P, D);
 
-  // ---- this CTA's share of the units, and this warp's part of it ----
   const int64_t T = (int64_t)P[p.n] * p.Hkv;
-  const int64_t C = gridDim.x, cta = blockIdx.x;
-  const int64_t U0c = cta * T / C, U1c = (cta + 1) * T / C, nuc = U1c - U0c;
-  const int64_t U0 = U0c + warp * nuc / NW, U1 = U0c + (warp + 1) * nuc / NW;
+  const int64_t W = (int64_t)gridDim.x * kDecWarps;
+  const int64_t w = (int64_t)blockIdx.x * kDecWarps + warp;
+  const int64_t U0 = w * T / W, U1 = (w + 1) * T / W;
+  if (U0 >= U1) return;
 
   uint8_t* wsm = smem + p.plan_smem + warp * p.warp_smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + p.nstage * p.stage_bytes);
@@ -1124,180 +914,269 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks) decode_kernel(Deco
     tk.cand = reinterpret_cast<float*>(tb + kTopkHdrBytes);
     tk.topk = p.topk;
   }
-  // the piece of this warp's first segment, when that segment started in an
-  // earlier warp and ends in this one, goes to global memory (the ring is
-  // busy then); a piece left at the end of the loop goes into the idle ring
-  uint8_t* first_piece = p.wrec + ((int64_t)cta * NW + warp) * p.rb;
-  // this warp's first and last segments, from the unit ranges (whatever the
-  // loop below achieves, the merge duties stay the same)
-  const int first_seg = U0 < U1 ? seg_of_unit(p, P, U0) : -1;
-  const int last_seg = U0 < U1 ? seg_of_unit(p, P, U1 - 1) : -1;
+  if (lane == 0) {
+    for (int s = 0; s < p.nstage; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
 
-  if (U0 < U1) {
+  UnitMeta cur = resolve_unit(p, P, U0 + lane, U1);
+  UnitMeta nxt = resolve_unit(p, P, U0 + 32 + lane, U1);
+  const int nu = (int)(U1 - U0);   // units of one warp: < 2^31
+
+  // Issues unit ku (its lane in `m`) into stage st: the page-head block, plus
+  // the segment's Q rows when ku is the first unit of a segment in this warp.
+  int last_issued_seg = -1;
+  auto issue = [&](const UnitMeta& m, int ku, int st) {
+    const int srcl = ku & 31;
+    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, m.src_lo, srcl);
+    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, m.src_hi, srcl);
+    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, m.cls_seg, srcl);
+    const int useg = (int)(cs & 0xFFFFFFu);
+    const bool needq = useg != last_issued_seg;
+    last_issued_seg = useg;
     if (lane == 0) {
-      for (int s2 = 0; s2 < p.nstage; ++s2) mbar_init(&bars[s2], 1);
-      fence_mbar_init();
+      uint8_t* dst = wsm + st * p.stage_bytes;
+      const uint32_t bytes = (uint32_t)p.phb[cs >> 24];
+      mbar_arrive_expect_tx(&bars[st], bytes + (needq ? (uint32_t)p.q_bytes : 0u));
+      bulk_g2s(dst, reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[st]);
+      if (needq) {
+        const int i = useg / p.Hkv, h = useg - (useg / p.Hkv) * p.Hkv;
+        bulk_g2s(dst + p.q_off, p.q + ((int64_t)i * p.Hq + (int64_t)h * p.Gq) * D,
+                 (uint32_t)p.q_bytes, &bars[st]);
+      }
     }
-    __syncwarp();
+  };
 
-    UnitMeta cur = resolve_unit(p, P, U0 + lane, U1);
-    UnitMeta nxt = resolve_unit(p, P, U0 + 32 + lane, U1);
-    const int nu = (int)(U1 - U0);   // units of one warp: < 2^31
+  // only the first page goes out before the loop: copies issued together all
+  // land together, so the rest of the ring is filled once the first has landed
+  issue(cur, 0, 0);
 
-    // Issues unit ku (its lane in `m`) into stage st: the page-head block, plus
-    // the segment's Q rows when ku is the first unit of a segment in this warp.
-    int last_issued_seg = -1;
-    auto issue = [&](const UnitMeta& m, int ku, int st) {
-      const int srcl = ku & 31;
-      const uint32_t lo = __shfl_sync(0xFFFFFFFFu, m.src_lo, srcl);
-      const uint32_t hi = __shfl_sync(0xFFFFFFFFu, m.src_hi, srcl);
-      const uint32_t cs = __shfl_sync(0xFFFFFFFFu, m.cls_seg, srcl);
-      const int useg = (int)(cs & 0xFFFFFFu);
-      const bool needq = useg != last_issued_seg;
-      last_issued_seg = useg;
-      if (lane == 0) {
-        uint8_t* dst = wsm + st * p.stage_bytes;
-        const uint32_t bytes = (uint32_t)p.phb[cs >> 24];
-        mbar_arrive_expect_tx(&bars[st], bytes + (needq ? (uint32_t)p.q_bytes : 0u));
-        bulk_g2s(dst, reinterpret_cast<const void*>(((uint64_t)hi << 32) | lo), bytes, &bars[st]);
-        if (needq) {
-          const int i = useg / p.Hkv, h = useg - (useg / p.Hkv) * p.Hkv;
-          bulk_g2s(dst + p.q_off, p.q + ((int64_t)i * p.Hq + (int64_t)h * p.Gq) * D,
-                   (uint32_t)p.q_bytes, &bars[st]);
-        }
+  SegState<D, G> S;
+  int seg = -1;
+  int stage = 0;
+  uint32_t parity = 0;
+  bool failed = false;
+  for (int k = 0; k < nu; ++k) {
+    const int kk = k & 31;
+    if (kk == 0 && k > 0) {
+      cur = nxt;
+      nxt = resolve_unit(p, P, U0 + k + 32 + lane, U1);
+    }
+    if (!mbar_wait_bounded(&bars[stage], parity)) {
+      if (lane == 0) set_status(p.status, THINKV_ERR_TIMEOUT);
+      // drain the copies still in flight (bounded), then stop
+      const int issued = k == 0 ? 1 : min(nu, k + p.nstage);
+      for (int k2 = k + 1; k2 < issued; ++k2)
+        mbar_wait_bounded(&bars[k2 % p.nstage], (uint32_t)((k2 / p.nstage) & 1));
+      failed = true;
+      break;
+    }
+    if (k == 0)
+      for (int s2 = 1; s2 < p.nstage && s2 < nu; ++s2) issue(cur, s2, s2);
+    const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, kk);
+    const int useg = (int)(cs & 0xFFFFFFu);
+    uint8_t* blk = wsm + stage * p.stage_bytes;
+    if (useg != seg) {
+      if (seg >= 0) {
+        int64_t Us, Ue;
+        seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
+        seg_end<D, G>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
       }
-    };
-
-    // every stage of the ring goes out at once: the first pages of all warps
-    // are in flight together
-    for (int s2 = 0; s2 < p.nstage && s2 < nu; ++s2) issue(cur, s2, s2);
-
-    SegState<D, G> S;
-    int seg = -1;
-    int stage = 0;
-    uint32_t parity = 0;
-    bool failed = false;
-    for (int k = 0; k < nu; ++k) {
-      const int kk = k & 31;
-      if (kk == 0 && k > 0) {
-        cur = nxt;
-        nxt = resolve_unit(p, P, U0 + k + 32 + lane, U1);
-      }
-      if (!mbar_wait_bounded(&bars[stage], parity)) {
-        if (lane == 0) set_status(p.status, THINKV_ERR_TIMEOUT);
-        // drain the copies still in flight (bounded), then stop computing;
-        // the merges below still run (on stale pieces: the status says so)
-        const int issued = min(nu, k + p.nstage);
-        for (int k2 = k + 1; k2 < issued; ++k2)
-          mbar_wait_bounded(&bars[k2 % p.nstage], (uint32_t)((k2 / p.nstage) & 1));
-        failed = true;
-        break;
-      }
-      const uint32_t cs = __shfl_sync(0xFFFFFFFFu, cur.cls_seg, kk);
-      const int useg = (int)(cs & 0xFFFFFFu);
-      uint8_t* blk = wsm + stage * p.stage_bytes;
-      if (useg != seg) {
-        if (seg >= 0) {
-          // the previous segment ends inside this warp: whole here unless it
-          // started before U0 (then it is this warp's first segment)
-          int64_t Us, Ue;
-          seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
-          seg_end<D, G>(S, p, seg, tk, Us >= U0 ? nullptr : first_piece);
-        }
-        seg = useg;
-        seg_begin<D, G>(S, p, reinterpret_cast<const uint16_t*>(blk + p.q_off),
-                        reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(pbuf) + kQfragOff), tk);
-        __syncwarp();
-      }
-      const uint32_t mask = __shfl_sync(0xFFFFFFFFu, cur.mask, kk);
-      page_dispatch<D, G>(S, blk, p.bits[cs >> 24], mask & 0xFFFFu, p.scale_log2, pbuf, tk, p.Gq);
+      seg = useg;
+      seg_begin<D, G>(S, p, reinterpret_cast<const uint16_t*>(blk + p.q_off),
+                      reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(pbuf) + kQfragOff), tk);
       __syncwarp();
-      // refill this stage with unit k + nstage (from this batch of 32 or the next)
-      const int kn = k + p.nstage;
-      if (kn < nu) issue(((kn >> 5) == (k >> 5)) ? cur : nxt, kn, stage);
-      if (++stage == p.nstage) {
-        stage = 0;
-        parity ^= 1u;
-      }
     }
-    if (!failed) {
-      int64_t Us, Ue;
-      seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
-      // the ring is idle now: every copy issued has landed
-      seg_end<D, G>(S, p, seg, tk, (Us >= U0 && Ue <= U1) ? nullptr : wsm);
+    const uint32_t mask = __shfl_sync(0xFFFFFFFFu, cur.mask, kk);
+    page_dispatch<D, G>(S, blk, p.bits[cs >> 24], mask & 0xFFFFu, p.scale_log2, pbuf, tk, p.Gq);
+    __syncwarp();
+    // refill this stage with unit k + nstage (from this batch of 32 or the next)
+    const int kn = k + p.nstage;
+    if (kn < nu) issue(((kn >> 5) == (k >> 5)) ? cur : nxt, kn, stage);
+    if (++stage == p.nstage) {
+      stage = 0;
+      parity ^= 1u;
     }
   }
-  if (lane == 0) s_last[warp] = last_seg;
-  __syncthreads();
-
-  // ---- merges: the last warp of this CTA that touches a split segment merges
-  //      the warps' pieces; a segment spanning CTAs goes through the CTA records ----
-  if (U0 >= U1) return;
-  float* wbuf = pbuf;                              // the warp's 704-float merge scratch
-  int* list = reinterpret_cast<int*>(pbuf) + 16;   // up to 160 piece owners
-  for (int which = 0; which < 2; ++which) {
-    const int S = which == 0 ? first_seg : last_seg;
-    if (which == 0 && first_seg == last_seg) continue;   // one segment: handled as the last
+  if (failed || seg < 0) return;
+  {
     int64_t Us, Ue;
-    seg_range(p, P, S / p.Hkv, S % p.Hkv, &Us, &Ue);
-    if (Us >= U0 && Ue <= U1) continue;            // whole in this warp: already written
-    // the last warp touching S merges: S ends in this warp, or this is the
-    // CTA's last warp with units
-    const int64_t wlast = share_of_unit(min(Ue, U1c) - 1 - U0c, nuc, NW);
-    if (wlast != warp) continue;
-    const int64_t wfirst = share_of_unit(max(Us, U0c) - U0c, nuc, NW);
-    // the warps in [wfirst, warp] that hold units (shares can be empty when
-    // the CTA has fewer units than warps)
-    int npw = 0;
-    for (int wj = (int)wfirst; wj <= warp; ++wj)
-      if (U0c + (int64_t)wj * nuc / NW < U0c + (int64_t)(wj + 1) * nuc / NW) {
-        if (lane == 0) list[npw] = wj;
-        ++npw;
-      }
-    __syncwarp();
-    auto warp_piece = [&](int j) -> const uint8_t* {
-      const int wj = list[j];
-      // a warp's piece of S sits in its ring if S was its last segment
-      return s_last[wj] == S ? smem + p.plan_smem + wj * p.warp_smem
-                             : p.wrec + ((int64_t)cta * NW + wj) * p.rb;
-    };
-    const bool in_cta = Us >= U0c && Ue <= U1c;
-    if (in_cta) {
-      merge_pieces<D, false>(p, S, npw, warp_piece, nullptr, wbuf);
-      continue;
-    }
-    // the CTA's piece of S: slot 0 if S holds the CTA's first unit, else slot 1
-    uint8_t* mine = p.crec + ((int64_t)cta * 2 + (Us <= U0c ? 0 : 1)) * p.rb;
-    merge_pieces<D, false>(p, S, npw, warp_piece, mine, wbuf);
-    __threadfence();
-    __syncwarp();
-    // the CTAs holding units of S (empty shares skipped)
-    const int64_t ca = share_of_unit(Us, T, C), cb = share_of_unit(Ue - 1, T, C);
-    int ncta = 0;
-    for (int64_t c0 = ca; c0 <= cb; c0 += 32) {
-      const int64_t cj = c0 + lane;
-      const bool has = cj <= cb && cj * T / C < (cj + 1) * T / C;
-      const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
-      if (has) list[ncta + __popc(bal & ((1u << lane) - 1u))] = (int)cj;
-      ncta += __popc(bal);
-    }
-    uint32_t old = 0;
-    if (lane == 0) old = atomicInc(p.cnt + S, (uint32_t)ncta - 1u);   // wraps to 0 on the last arrival
-    old = __shfl_sync(0xFFFFFFFFu, old, 0);
-    if (old != (uint32_t)ncta - 1u) continue;
-    __threadfence();                               // the other CTAs' records are visible now
-    __syncwarp();
-    auto cta_piece = [&](int j) -> const uint8_t* {
-      const int64_t cj = list[j];
-      const int64_t u0j = cj * T / C;
-      return p.crec + (cj * 2 + (Us <= u0j ? 0 : 1)) * p.rb;
-    };
-    merge_pieces<D, true>(p, S, ncta, cta_piece, nullptr, wbuf);
+    seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
+    seg_end<D, G>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// split combine: one CTA per (sequence, kv-head) segment that the split
+// kernel left in more than one piece
+// ---------------------------------------------------------------------------
+constexpr int kCombineThreads = 256;
+constexpr int kCombinePieces = 128;             // pieces per round of the weight table
+constexpr int kCombinePre = 8;                  // pieces whose quads are requested up front
+
+// Merges the segment's piece records with the log-sum-exp rule: thread t <
+// Gq * D/4 owns one quad of one head's output row; warp r < Gq then merges
+// head r's top-k lists (bitonic merges, the next piece's list loaded while the
+// current one merges) for the top-k mass.
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(DecodeParams p) {
+  constexpr int QD = D / 4;
+  __shared__ float sM[8], sL[8];
+  __shared__ int sMk[8];
+  __shared__ float cwt[kCombinePieces * 8], lt[kCombinePieces * 8];
+  pdl_launch_dependents();
+  pdl_wait();                                   // records and prefix come from the split kernel
+  const int seg = blockIdx.x;
+  const int i = seg / p.Hkv, h = seg - (seg / p.Hkv) * p.Hkv;
+  const int nl = p.pref[i + 1] - p.pref[i];
+  if (nl == 0) return;                          // written by the split kernel
+  const int64_t T = (int64_t)p.pref[p.n] * p.Hkv, W = p.split_warps;
+  const int64_t Us = (int64_t)p.pref[i] * p.Hkv + (int64_t)h * nl, Ue = Us + nl;
+  const int64_t w0 = warp_of_unit(Us, T, W), w1 = warp_of_unit(Ue - 1, T, W);
+  const bool by_unit = T <= W;                  // one unit per warp
+  const int np = (int)(by_unit ? nl : w1 - w0 + 1);
+  if (np <= 1) return;                          // finished inside one split warp
+  const int Gq = p.Gq, k = p.topk, kpad = (k + 3) / 4 * 4;
+  // the top-k warps' live count, requested now and used after the merge
+  const int live_i = (p.mass && threadIdx.x < 32 * Gq) ? p.live_count[p.seq[i]] : 0;
+  const int64_t rb = record_bytes(Gq, D, k);
+  const uint8_t* recs = reinterpret_cast<const uint8_t*>(p.rec);
+  auto rec = [&](int j) -> const uint8_t* {
+    const int64_t pc = (by_unit ? warp_of_unit(Us + j, T, W) : w0 + j) + seg;
+    return recs + pc * rb;
+  };
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- per piece and head: the weight 2^(m - M) (M the head's max), and L ----
+  // (m, l) pairs are read once, lane-parallel; a table of weights in shared
+  // memory then lets every output thread stream its quads with many loads in
+  // flight.  Segments with more pieces than the table holds go in rounds.
+  float* wt = cwt;                                // [kCombinePieces][8]
+  // a float's order-preserving int key (negative floats: magnitude bits
+  // flipped); the map is its own inverse
+  auto okey = [](int b) { return b >= 0 ? b : b ^ 0x7FFFFFFF; };
+  const int r_o = tid / QD, q_o = tid - (tid / QD) * QD;
+  const bool out_thread = tid < Gq * QD;
+  auto quad = [&](int j) {
+    return __ldcg(reinterpret_cast<const float4*>(rec(j) + 64) + r_o * QD + q_o);
+  };
+  auto pair_ml = [&](int x) {
+    const int j = x / Gq, r = x - j * Gq;
+    return __ldcg(reinterpret_cast<const float2*>(rec(j)) + r);
+  };
+  // the first pieces' quads and (m, l) pairs do not depend on the weights:
+  // all of them are requested at once
+  float4 ov[kCombinePre];
+#pragma unroll
+  for (int j = 0; j < kCombinePre; ++j)
+    ov[j] = (out_thread && j < np) ? quad(j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float2 ml0 = tid < np * Gq ? pair_ml(tid) : make_float2(-INFINITY, 0.f);
+  if (tid < 8) { sMk[tid] = INT_MIN; sL[tid] = 0.f; }
+  __syncthreads();
+  for (int x = tid; x < np * Gq; x += kCombineThreads) {
+    const float m = x == tid ? ml0.x : pair_ml(x).x;
+    atomicMax(&sMk[x - (x / Gq) * Gq], okey(__float_as_int(m)));
+  }
+  __syncthreads();
+  if (tid < 8) sM[tid] = __int_as_float(okey(sMk[tid]));
+  __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < np; j0 += kCombinePieces) {
+    const int cnt = min(kCombinePieces, np - j0);
+    for (int x = tid; x < cnt * Gq; x += kCombineThreads) {
+      const int j = x / Gq, r = x - j * Gq;
+      const float2 ml = (j0 == 0 && x == tid) ? ml0 : pair_ml(j0 * Gq + x);
+      const float wgt = exp2_approx(ml.x - sM[r]);
+      wt[j * 8 + r] = wgt;
+      lt[j * 8 + r] = wgt * ml.y;
+    }
+    __syncthreads();
+    if (warp < Gq) {                              // L, summed in a fixed order
+      float l = 0.f;
+      for (int j = lane; j < cnt; j += 32) l += lt[j * 8 + warp];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+      if (lane == 0) sL[warp] += l;
+    }
+    if (out_thread) {
+      int jstart = 0;
+      if (j0 == 0) {
+#pragma unroll
+        for (int j = 0; j < kCombinePre; ++j) {
+          const float wgt = j < cnt ? wt[j * 8 + r_o] : 0.f;
+          acc.x = fmaf(wgt, ov[j].x, acc.x);
+          acc.y = fmaf(wgt, ov[j].y, acc.y);
+          acc.z = fmaf(wgt, ov[j].z, acc.z);
+          acc.w = fmaf(wgt, ov[j].w, acc.w);
+        }
+        jstart = kCombinePre;
+      }
+#pragma unroll 8
+      for (int j = jstart; j < cnt; ++j) {
+        const float4 v = quad(j0 + j);
+        const float wgt = wt[j * 8 + r_o];
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
+      }
+    }
+    __syncthreads();                              // the table is refilled by the next round
+  }
+  if (tid < Gq * QD) {
+    const float inv = 1.f / sL[r_o];
+    const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(acc.x * inv)) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(acc.y * inv)) << 16);
+    const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(acc.z * inv)) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(acc.w * inv)) << 16);
+    const int64_t row = (int64_t)i * p.Hq + h * Gq + r_o;
+    reinterpret_cast<uint2*>(p.out + row * D)[q_o] = make_uint2(lo, hi);
+  }
+  if (!p.mass) return;
+  if (warp >= Gq) return;
+  const int r = warp;
+  const int64_t mrow = (int64_t)i * p.Hq + h * Gq + r;
+  if (live_i <= k) {
+    if (lane == 0) p.mass[mrow] = 1.f;
+    return;
+  }
+  // running list (descending) in elements 0..63, the next piece's list
+  // reversed in 64..127: a bitonic sequence
+  float tv[4], nx[4];
+  auto load_list = [&](int j, float (&x)[4]) {
+    const float* tl = reinterpret_cast<const float*>(rec(j) + 64 + 4 * Gq * D) + r * kpad;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int el = lane * 4 + e, m = 127 - el;
+      x[e] = (el >= 64 && m < k) ? __ldcg(tl + m) : -INFINITY;
+    }
+  };
+#pragma unroll
+  for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
+  load_list(0, nx);
+  for (int j = 0; j < np; ++j) {
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = (lane * 4 + e < 64) ? tv[e] : nx[e];
+    if (j + 1 < np) load_list(j + 1, nx);
+    bitonic128_merge_desc(v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tv[e] = v[e];
+  }
+  const float M = sM[r];
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (lane * 4 + e < k) sum += exp2_approx(tv[e] - M);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  if (lane == 0) p.mass[mrow] = sum / sL[r];
+}
+
 template <int D, int G>
-cudaError_t launch_kernel(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
+cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
   // raise the dynamic shared-memory limit of this instantiation once per
   // device (and again whenever a launch needs more); host threads that decode
   // at the same time serialise on the lock, so the recorded size never runs
@@ -1311,21 +1190,21 @@ cudaError_t launch_kernel(const DecodeParams& p, const DecodeLaunch& dl, cudaStr
   {
     std::lock_guard<std::mutex> guard(lock);
     if (dl.smem_bytes > configured[dev]) {
-      e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)dl.smem_bytes);
       if (e != cudaSuccess) return e;
       configured[dev] = dl.smem_bytes;
     }
   }
-  return launch_pdl(decode_kernel<D, G>, dim3(dl.grid), dim3(dl.warps_per_cta * 32), dl.smem_bytes,
-                    stream, p);
+  e = launch_pdl(decode_split_kernel<D, G>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
+                 stream, p);
+  if (e != cudaSuccess) return e;
+  // the combine: one CTA per segment (most return at once)
+  return launch_pdl(decode_combine_kernel<D>, dim3((unsigned)(p.n * p.Hkv)),
+                    dim3(kCombineThreads), 0, stream, p);
 }
 
-int plan_smem_bytes(int32_t n) { return ((n + 1) * 4 + 127) / 128 * 128; }
-
-int64_t counters_bytes(const thinkv_layout& L, int32_t n) {
-  return ((int64_t)n * L.num_kv_heads * 4 + 255) / 256 * 256;
-}
+int plan_smem_bytes(int32_t n) { return ((2 * n + 1) * 4 + 127) / 128 * 128; }
 
 }  // namespace
 
@@ -1337,55 +1216,58 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
     int64_t b = page_head_bytes(D, G, L.bits[c]);
     if (b > maxphb) maxphb = b;
   }
-  const int Gq = L.num_q_heads / L.num_kv_heads;
-  const int q_bytes = Gq * D * 2;
+  const int Gq0 = L.num_q_heads / L.num_kv_heads;
+  const int q_bytes = Gq0 * D * 2;
   const int stage_bytes = (int)((maxphb + 127) / 128 * 128) + (q_bytes + 127) / 128 * 128;
+  // ~15 KB of page-head stages and top-k buffers per warp keeps three 4-warp
+  // CTAs per SM (at 8 warps per SM the top-k path ran 12-19 % slower)
+  const int Gq = L.num_q_heads / L.num_kv_heads;
   const int topk_bytes = topk > 0 ? kTopkHdrBytes + Gq * kCandCap * 4 : 0;
-  const int64_t rb = record_bytes(Gq, D, topk > 0 ? topk : 0);
-  int optin = 0, sms = 0;
+  int nstage = (int)((15360 - topk_bytes) / stage_bytes);
+  if (nstage < 2) nstage = 2;
+  if (nstage > kMaxStages) nstage = kMaxStages;
+  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes + topk_bytes;
+  const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)kDecWarps * warp_smem;
+  int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
     return false;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return false;
-  // one CTA per SM: the stages take what the prefix, the per-warp scratch and
-  // the kernel's static shared memory (under 1 KB) leave.  The most warps
-  // that fit at least two stages each win (warps hide the page step's
-  // latency; a deeper ring at fewer warps measured far slower), with as many
-  // stages as fit; the ring must also hold the warp's last piece record
-  const int64_t fixed = plan_smem_bytes(n_seqs) + 1024;
-  int best_nw = 0, best_ns = 0;
-  for (int nw = kDecWarps; nw >= 4 && best_nw == 0; --nw) {
-    const int64_t per_warp = (optin - fixed) / nw - 64 - kPbufBytes - topk_bytes;
-    int ns = per_warp > 0 ? (int)(per_warp / stage_bytes) : 0;
-    if (ns > kMaxStages) ns = kMaxStages;
-    if (ns < 2 || (int64_t)ns * stage_bytes < rb) continue;
-    best_nw = nw;
-    best_ns = ns;
-  }
-  if (best_nw == 0) return false;
-  const int warp_smem = best_ns * stage_bytes + 64 + kPbufBytes + topk_bytes;
-  const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)best_nw * warp_smem;
   if (smem + 1024 > (size_t)optin) return false;
-  // a segment's CTA list (merge scratch) holds up to 160 entries
-  out->grid = sms < 160 ? sms : 160;
-  out->warps_per_cta = best_nw;
-  out->nstage = best_ns;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return false;
+  int smem_per_sm = 0;
+  if (cudaDeviceGetAttribute(&smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
+      cudaSuccess)
+    return false;
+  // CTAs per SM: limited by shared memory (1 KB reserved per CTA) and by registers
+  int per_sm = smem_per_sm / (int)(smem + 1024);
+  int regs_per_sm = 0;
+  if (cudaDeviceGetAttribute(&regs_per_sm, cudaDevAttrMaxRegistersPerMultiprocessor, device) !=
+      cudaSuccess)
+    return false;
+  const int by_regs = regs_per_sm / (kDecRegs * kDecThreads);
+  if (per_sm > by_regs) per_sm = by_regs;
+  if (per_sm > 16) per_sm = 16;
+  if (per_sm < 1) per_sm = 1;
+  out->grid = sms * per_sm;
+  out->warps_per_cta = kDecWarps;
+  out->nstage = nstage;
   out->stage_bytes = stage_bytes;
   out->smem_bytes = smem;
   out->warp_smem = warp_smem;
-  out->pieces = (int64_t)out->grid * (best_nw + 2);
+  out->pieces = (int64_t)out->grid * kDecWarps + (int64_t)n_seqs * L.num_kv_heads;
+
   return true;
 }
 
 size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
                               const DecodeLaunch& dl) {
   const int Gq = L.num_q_heads / L.num_kv_heads;
-  // arrival counters, then the warps' and the CTAs' piece records
-  return (size_t)counters_bytes(L, n_seqs) +
-         (size_t)dl.pieces * (size_t)record_bytes(Gq, L.head_dim, topk > 0 ? topk : 0);
-}
-
-size_t decode_counter_bytes(const thinkv_layout& L, int32_t n_seqs) {
-  return (size_t)counters_bytes(L, n_seqs);
+  // the prefix of live pages, then one record per (split warp, segment)
+  const size_t head = (size_t)(n_seqs + 1 > n_seqs * L.num_kv_heads ? n_seqs + 1
+                                                                     : n_seqs * L.num_kv_heads);
+  size_t b = (head * 4 + 255) / 256 * 256;
+  b += (size_t)dl.pieces * (size_t)record_bytes(Gq, L.head_dim, topk > 0 ? topk : 0);
+  return b;
 }
 
 cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, const uint16_t* q,
@@ -1413,15 +1295,15 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   p.q = q;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
-  p.topk = mass ? topk : 0;
-  p.rb = (int32_t)record_bytes(p.Gq, D, p.topk);
   uint8_t* w = static_cast<uint8_t*>(ws);
-  p.cnt = reinterpret_cast<uint32_t*>(w);
-  w += counters_bytes(L, n);
-  p.wrec = w;
-  w += (int64_t)dl.grid * dl.warps_per_cta * p.rb;
-  p.crec = w;
-  p.nw = dl.warps_per_cta;
+  p.pref = reinterpret_cast<int32_t*>(w);
+  {
+    const size_t head = (size_t)(n + 1 > n * L.num_kv_heads ? n + 1 : n * L.num_kv_heads);
+    w += (head * 4 + 255) / 256 * 256;
+  }
+  p.topk = mass ? topk : 0;
+  p.rec = w;
+  p.split_warps = (int64_t)dl.grid * kDecWarps;
   p.live_count = C.live_count;
   p.out = out;
   p.mass = p.topk > 0 ? mass : nullptr;
@@ -1437,10 +1319,10 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   }
   p.plan_smem = plan_smem_bytes(n);
   cudaError_t e;
-  if (D == 128 && G == 64) e = launch_kernel<128, 64>(p, dl, stream);
-  else if (D == 128 && G == 32) e = launch_kernel<128, 32>(p, dl, stream);
-  else if (D == 64 && G == 64) e = launch_kernel<64, 64>(p, dl, stream);
-  else e = launch_kernel<64, 32>(p, dl, stream);
+  if (D == 128 && G == 64) e = launch_split<128, 64>(p, dl, stream);
+  else if (D == 128 && G == 32) e = launch_split<128, 32>(p, dl, stream);
+  else if (D == 64 && G == 64) e = launch_split<64, 64>(p, dl, stream);
+  else e = launch_split<64, 32>(p, dl, stream);
   return e;
 }
 

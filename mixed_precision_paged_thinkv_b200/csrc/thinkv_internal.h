@@ -74,15 +74,12 @@ struct DecodeLaunch {
   int stage_bytes;     // bytes per stage
   size_t smem_bytes;   // dynamic shared memory of the split kernel
   int warp_smem;       // bytes of shared memory per warp
-  int64_t pieces;      // piece records (the CTAs' warps + two per CTA)
+  int64_t pieces;      // piece records (warps + segments)
 };
 bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, int device,
                         DecodeLaunch* out);
 size_t decode_workspace_bytes(const thinkv_layout& L, int32_t n_seqs, int32_t topk,
                               const DecodeLaunch& dl);
-// leading bytes of the decode workspace that must be zero before a call
-// (segment arrival counters; every call that completes leaves them zero)
-size_t decode_counter_bytes(const thinkv_layout& L, int32_t n_seqs);
 cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, const uint16_t* q,
                           uint16_t* out, float* mass, int32_t topk, float softmax_scale,
                           void* ws, const DecodeLaunch& dl, cudaStream_t stream);

@@ -4,9 +4,8 @@
 // framework that owns all device memory and gives its plugins no allocator;
 // paths that cannot afford cudaMalloc's device-wide synchronisation).  The
 // split-K scratch of the decode kernels -- the live-page prefix and the
-// per-segment arrival counters and the per-piece partial outputs and top-k
-// lists -- is one file-scope device array of fixed size instead of a caller
-// workspace.  The ThinKV pages have no
+// per-piece partial outputs and top-k lists -- is one file-scope device array
+// of fixed size instead of a caller workspace.  The ThinKV pages have no
 // counterpart.
 #include <cuda_runtime.h>
 #include <mutex>
@@ -65,9 +64,5 @@ extern "C" int thinkv_decode_attention_noalloc(const thinkv_cache* C, int32_t n,
   const cudaError_t e = scratch_address(&ws);
   if (e != cudaSuccess) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the array keeps the last call's contents: the segment counters, which
-  // must start at zero, are cleared here (a memset, not an allocation)
-  const cudaError_t z = cudaMemsetAsync(ws, 0, decode_counter_bytes(C->L, n), s);
-  if (z != cudaSuccess) return cuda_status(z);
   return cuda_status(launch_decode(view_of(C), n, seq, q, out, topk_mass, k, softmax_scale, ws, dl, s));
 }
