@@ -26,8 +26,9 @@
 //     entry and slot position.
 //   compact_copy_kernel: one warp per (dst page, kv-head) gathers the
 //     page-head block in shared memory -- K pieces, V half-words and params of
-//     each of its source slots at the new slot, every two-byte unit a load of
-//     its own, all in flight together -- and writes it out with 16-byte stores.
+//     each of its source slots at the new slot, every two- or four-byte unit
+//     a load of its own, eight per lane in flight -- and writes it out with
+//     16-byte stores.
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
@@ -40,6 +41,7 @@ namespace {
 constexpr int kCompactThreads = 1024;
 constexpr int kCompactWarps = kCompactThreads / 32;
 constexpr int kCopyWarps = 8;
+constexpr int kCopyBatch = 8;      // gather loads in flight per lane (compact_copy_kernel)
 
 // Block-wide exclusive scan (kCompactThreads threads) of one int per thread.
 __device__ int block_scan(int v, int* sh, int* total) {
@@ -284,58 +286,110 @@ __global__ void compact_list_kernel(CacheView S, CacheView Dc, int32_t n,
   }
 }
 
-// Byte offsets of unit u (two bytes) of one slot's data inside a page-head
-// block (b-bit codes, lane portions interleaved in chunks; include/thinkv.h):
-// units [0, ku) are K pieces, [ku, ku + kv) V half-words, then params words
-// (counted as two units each).
+// Byte offsets of unit u of one slot's data inside a page-head block of
+// b-bit codes (lane portions interleaved in chunks; include/thinkv.h): units
+// [0, KU) are two-byte K pieces, [KU, KU + KVU) V half-words, then (b < 16)
+// the four-byte (scale, zero) words of K and V per group.  All shapes are
+// compile-time, so every divide is a shift.
+template <int D, int G, int B>
 struct SlotUnits {
-  int D, G, b, NG, lane_bytes, region, pb, ku, kvu, Q;
+  static constexpr int NG = D / G;
+  static constexpr int LB = D * B / 16;                 // lane portion bytes
+  static constexpr int REGION = 2 * D * B;
+  static constexpr int PB = G * B / 32;                 // K piece bytes
+  static constexpr int HW = PB / 2;                     // two-byte units per piece
+  static constexpr int KU = NG * 4 * HW;
+  static constexpr int Q = B == 16 ? D / 8 : D * B / 128;
+  static constexpr int KVU = 8 * Q;
+  static constexpr int PER = KU + KVU + (B < 16 ? 2 * NG : 0);
+  static constexpr int PHB = B == 16 ? 64 * D : 4 * D * B + 128 * NG;
+  static constexpr int CH = LB < 16 ? LB : 16;          // chunk bytes
+
+  __device__ static int lane_at(int l, int o) { return (o / CH) * 32 * CH + l * CH + (o % CH); }
+
+  // source and destination offsets of unit u of slot ss -> ds; returns the size (2 or 4)
+  __device__ static int offsets(int u, int ss, int ds, int* so, int* dof) {
+    if (u < KU) {
+      const int hw = u % HW, t = (u / HW) % 4, gr = u / HW / 4;
+      *so = lane_at(4 * (ss & 7) + t, (gr * 2 + (ss >> 3)) * PB + 2 * hw);
+      *dof = lane_at(4 * (ds & 7) + t, (gr * 2 + (ds >> 3)) * PB + 2 * hw);
+      return 2;
+    }
+    u -= KU;
+    if (u < KVU) {
+      const int g = u / Q, q = u % Q;
+      *so = REGION + lane_at(4 * g + ((ss & 7) >> 1), ((ss >> 3) * Q + q) * 4 + 2 * (ss & 1));
+      *dof = REGION + lane_at(4 * g + ((ds & 7) >> 1), ((ds >> 3) * Q + q) * 4 + 2 * (ds & 1));
+      return 2;
+    }
+    u -= KVU;                                          // params: [K|V][group][slot] words
+    const int kv = u / NG, gr = u % NG;
+    const int base = 2 * REGION + kv * 64 * NG;
+    *so = base + (gr * 16 + ss) * 4;
+    *dof = base + (gr * 16 + ds) * 4;
+    return 4;
+  }
 };
 
-__device__ inline SlotUnits slot_units(int D, int G, int b) {
-  SlotUnits m;
-  m.D = D; m.G = G; m.b = b; m.NG = D / G;
-  m.lane_bytes = D * b / 16;
-  m.region = 2 * D * b;
-  m.pb = G * b / 32;
-  m.ku = m.NG * 4 * (m.pb / 2);
-  m.Q = b == 16 ? D / 8 : D * b / 128;
-  m.kvu = 8 * m.Q;
-  return m;
+// One page-head block gathered into the warp's shared-memory image db: the
+// used slots' units, lane-strided, kCopyBatch loads in flight per lane before
+// their stores.  srcl: lane sl holds slot sl's source pool slot (page*16+slot).
+template <int D, int G, int B>
+__device__ __forceinline__ void gather_block(const uint8_t* __restrict__ pool, int H, int h, int32_t srcl, int used,
+                             uint8_t* db) {
+  using M = SlotUnits<D, G, B>;
+  const int lane = threadIdx.x & 31;
+  const int total = used * M::PER;
+  for (int x0 = 0; x0 < total; x0 += 32 * kCopyBatch) {     // warp-uniform trip count
+    uint32_t val[kCopyBatch];
+    int dst[kCopyBatch];                          // smem offset | 4-byte flag; -1: none
+#pragma unroll
+    for (int j = 0; j < kCopyBatch; ++j) {
+      const int x = x0 + j * 32 + lane;
+      const int sl = min(x / M::PER, used - 1), uu = x - sl * M::PER;
+      const int32_t src = __shfl_sync(0xFFFFFFFFu, srcl, sl);
+      val[j] = 0;
+      dst[j] = -1;
+      if (x < total) {
+        int so, dof;
+        const int sz = M::offsets(uu, src & 15, sl, &so, &dof);
+        const uint8_t* sb = pool + ((int64_t)(src >> 4) * H + h) * M::PHB;
+        val[j] = sz == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(sb + so)
+                         : *reinterpret_cast<const uint32_t*>(sb + so);
+        dst[j] = dof | (sz == 4 ? (1 << 30) : 0);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kCopyBatch; ++j) {
+      if (dst[j] < 0) continue;
+      const int dof = dst[j] & ((1 << 30) - 1);
+      if (dst[j] & (1 << 30)) *reinterpret_cast<uint32_t*>(db + dof) = val[j];
+      else *reinterpret_cast<uint16_t*>(db + dof) = (uint16_t)val[j];
+    }
+  }
 }
 
-// source and destination offsets (and size, 2 or 4) of unit u of slot ss -> ds
-__device__ inline int unit_offsets(const SlotUnits& m, int u, int ss, int ds, int* so, int* dof) {
-  if (u < m.ku) {
-    const int hw = u % (m.pb / 2), t = (u / (m.pb / 2)) % 4, gr = u / (m.pb / 2) / 4;
-    *so = lane_off(4 * (ss & 7) + t, (gr * 2 + (ss >> 3)) * m.pb + 2 * hw, m.lane_bytes);
-    *dof = lane_off(4 * (ds & 7) + t, (gr * 2 + (ds >> 3)) * m.pb + 2 * hw, m.lane_bytes);
-    return 2;
+template <int D, int G>
+__device__ inline void gather_dispatch(int b, const uint8_t* pool, int H, int h, int32_t srcl,
+                                       int used, uint8_t* db) {
+  switch (b) {
+    case 2: gather_block<D, G, 2>(pool, H, h, srcl, used, db); break;
+    case 4: gather_block<D, G, 4>(pool, H, h, srcl, used, db); break;
+    case 8: gather_block<D, G, 8>(pool, H, h, srcl, used, db); break;
+    default: gather_block<D, G, 16>(pool, H, h, srcl, used, db); break;
   }
-  u -= m.ku;
-  if (u < m.kvu) {
-    const int g = u / m.Q, q = u % m.Q;
-    *so = m.region + lane_off(4 * g + ((ss & 7) >> 1), ((ss >> 3) * m.Q + q) * 4 + 2 * (ss & 1), m.lane_bytes);
-    *dof = m.region + lane_off(4 * g + ((ds & 7) >> 1), ((ds >> 3) * m.Q + q) * 4 + 2 * (ds & 1), m.lane_bytes);
-    return 2;
-  }
-  u -= m.kvu;                                      // params: [K|V][group][slot] words
-  const int kv = u / m.NG, gr = u % m.NG;
-  const int base = 2 * m.region + kv * 64 * m.NG;
-  *so = base + (gr * 16 + ss) * 4;
-  *dof = base + (gr * 16 + ds) * 4;
-  return 4;
 }
 
 // (d) one warp per (dst page, kv-head): the page-head block is gathered into
-// shared memory -- every unit of every slot a lane load of its own, all in
-// flight together -- and written out with 16-byte stores
+// shared memory -- every unit of every slot a lane load of its own, a batch
+// of kCopyBatch per lane in flight -- and written out with 16-byte stores
+template <int D, int G>
 __global__ void __launch_bounds__(kCopyWarps * 32)
     compact_copy_kernel(CacheView S, CacheView Dc, int32_t n, CompactWs ws, int max_phb) {
   extern __shared__ __align__(16) uint8_t img[];   // kCopyWarps block images
   if (ws.totals[3] == 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int H = S.L.num_kv_heads, D = S.L.head_dim, G = S.L.group_size;
+  const int H = S.L.num_kv_heads;
   const int t0 = ws.totals[0], t1 = ws.totals[1], t2 = ws.totals[2];
   const int64_t units = (int64_t)(t0 + t1 + t2) * H;
   uint8_t* db = img + warp * max_phb;
@@ -361,25 +415,25 @@ __global__ void __launch_bounds__(kCopyWarps * 32)
     int toff = ws.tbase[c * (n + 1) + i] + j * kPage;
     for (int c2 = 0; c2 < c; ++c2) toff += ws.tbase[c2 * (n + 1) + n];
     const int32_t srcl = lane < used ? ws.src[toff + lane] : 0;   // lane sl: slot sl's source
-    const SlotUnits m = slot_units(D, G, b);
-    const int per = m.ku + m.kvu + 2 * m.NG;
-    for (int x0 = 0; x0 < used * per; x0 += 32) {     // warp-uniform trip count
-      const int x = x0 + lane;
-      const int sl = min(x / per, used - 1), uu = x - sl * per;
-      const int32_t src = __shfl_sync(0xFFFFFFFFu, srcl, sl);
-      if (x < used * per) {
-        int so, dof;
-        const int sz = unit_offsets(m, uu, src & 15, sl, &so, &dof);
-        const uint8_t* sb = S.pool[c] + ((int64_t)(src >> 4) * H + h) * phb;
-        if (sz == 2) *reinterpret_cast<uint16_t*>(db + dof) = *reinterpret_cast<const uint16_t*>(sb + so);
-        else *reinterpret_cast<uint32_t*>(db + dof) = *reinterpret_cast<const uint32_t*>(sb + so);
-      }
-    }
+    gather_dispatch<D, G>(b, S.pool[c], H, h, srcl, used, db);
     __syncwarp();
     uint4* dst = reinterpret_cast<uint4*>(Dc.pool[c] + ((int64_t)page * H + h) * phb);
     for (int x = lane; x < phb / 16; x += 32) dst[x] = reinterpret_cast<const uint4*>(db)[x];
     __syncwarp();
   }
+}
+
+template <int D, int G>
+cudaError_t launch_copy(const CacheView& S, const CacheView& Dc, int32_t n, const CompactWs& ws,
+                        int max_phb, int num_sms, cudaStream_t stream) {
+  const size_t smem = (size_t)kCopyWarps * max_phb;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(compact_copy_kernel<D, G>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  compact_copy_kernel<D, G><<<num_sms * 4, kCopyWarps * 32, smem, stream>>>(S, Dc, n, ws, max_phb);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -406,6 +460,12 @@ cudaError_t launch_compact(const CacheView& S, const CacheView& Dc, int32_t n, c
   const size_t seen_bytes = (size_t)((S.L.max_seqs + 31) / 32) * 4;
   const int64_t pairs = (int64_t)n * 3;
   const int gblocks = (int)((pairs * 32 + 255) / 256);
+  if (seen_bytes > 48 * 1024) {
+    const cudaError_t a = cudaFuncSetAttribute(compact_plan_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)seen_bytes);
+    if (a != cudaSuccess) return a;
+  }
   compact_count_kernel<<<gblocks, 256, 0, stream>>>(S, n, seq, ws);
   compact_plan_kernel<<<1, kCompactThreads, seen_bytes, stream>>>(S, Dc, n, seq, max_tokens, ws);
   compact_list_kernel<<<gblocks, 256, 0, stream>>>(S, Dc, n, seq, ws);
@@ -416,14 +476,11 @@ cudaError_t launch_compact(const CacheView& S, const CacheView& Dc, int32_t n, c
     const int b = (int)page_head_bytes(S.L.head_dim, S.L.group_size, S.L.bits[c]);
     max_phb = b > max_phb ? b : max_phb;
   }
-  const size_t smem = (size_t)kCopyWarps * max_phb;
-  if (smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(compact_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  compact_copy_kernel<<<num_sms * 4, kCopyWarps * 32, smem, stream>>>(S, Dc, n, ws, max_phb);
-  return cudaGetLastError();
+  const int D = S.L.head_dim, G = S.L.group_size;
+  if (D == 128 && G == 64) return launch_copy<128, 64>(S, Dc, n, ws, max_phb, num_sms, stream);
+  if (D == 128 && G == 32) return launch_copy<128, 32>(S, Dc, n, ws, max_phb, num_sms, stream);
+  if (D == 64 && G == 64) return launch_copy<64, 64>(S, Dc, n, ws, max_phb, num_sms, stream);
+  return launch_copy<64, 32>(S, Dc, n, ws, max_phb, num_sms, stream);
 }
 
 }  // namespace thinkv

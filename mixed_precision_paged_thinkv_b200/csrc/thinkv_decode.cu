@@ -384,7 +384,7 @@ __device__ inline int64_t warp_of_unit(int64_t u, int64_t T, int64_t W) {
 // was in this warp (Us >= U0 and Ue <= U1) its O rows and top-k mass are
 // written at once; otherwise the warp's piece record goes to rec[w + seg]
 // for the merge.
-template <int D, int G>
+template <int D, int G, bool TOPK>
 __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t w, int seg,
                                const TopkCtx& tk, bool whole) {
   constexpr int NG = SegState<D, G>::NG, MT = SegState<D, G>::MT;
@@ -429,7 +429,7 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
       }
     }
   }
-  if (tk.topk > 0) {
+  if (TOPK && tk.topk > 0) {
     const int kpad = (tk.topk + 3) / 4 * 4;
     const bool all = whole && p.live_count[p.seq[i]] <= tk.topk;
     float* tl = reinterpret_cast<float*>(rec + 64 + 4 * Gq * D);
@@ -494,7 +494,7 @@ __device__ __forceinline__ void lane_words(const uint8_t* base, int w0, uint32_t
 //   Float codes (FP8 E4M3 at b = 8, FP4 E2M1 at b = 4; F = 1) enter as their
 //   exact fp16 values with no offset and a zero of 0; ternary codes are the
 //   2-bit integer path (zero = -scale).
-template <int D, int G, int B, int F = 0>
+template <int D, int G, int B, int F, bool TOPK>
 __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t mask,
                                  float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
   const uint2* qfrag = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(pbuf) + kQfragOff);
@@ -531,7 +531,9 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
           for (int x = 0; x < NW; ++x) w[r][x] = kw[(KALL ? gr * 2 * NW : 0) + r * NW + x];
         }
       }
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      // two accumulator chains (even and odd k-steps) halve the dependent
+      // MMA latency of a group
+      float c2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int s = 0; s < KS; ++s) {
         uint32_t a[4];
@@ -554,8 +556,10 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
           }
         }
         const uint2 qb = qfrag[(gr * KS + s) * 32 + lane];
-        mma_16816(c, a, qb.x, qb.y);
+        mma_16816(c2[s & 1], a, qb.x, qb.y);
       }
+      const float c[4] = {c2[0][0] + c2[1][0], c2[0][1] + c2[1][1], c2[0][2] + c2[1][2],
+                          c2[0][3] + c2[1][3]};
       if constexpr (B == 16) {
         lg[0] += c[0]; lg[1] += c[1]; lg[2] += c[2]; lg[3] += c[3];
       } else {
@@ -577,7 +581,7 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   lg[3] = live1 ? lg[3] * scale_log2 : -INFINITY;
 
   // ---------------- top-k candidates (logits above the head's threshold) ----------------
-  if (tk.topk > 0) {
+  if (TOPK && tk.topk > 0) {
     // the thresholds are register copies; they change only when a buffer is cut
     bool ins = false;
 #pragma unroll
@@ -798,16 +802,16 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
 }
 
 // bits: the class's code width, plus 256 for the float formats at 8 and 4 bits
-template <int D, int G>
+template <int D, int G, bool TOPK>
 __device__ inline void page_dispatch(SegState<D, G>& S, const uint8_t* blk, int bits, uint32_t mask,
                                      float scale_log2, float* pbuf, const TopkCtx& tk, int Gq) {
   switch (bits) {
-    case 256 + 8: page_step<D, G, 8, 1>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
-    case 256 + 4: page_step<D, G, 4, 1>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
-    case 8: page_step<D, G, 8>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
-    case 4: page_step<D, G, 4>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
-    case 2: page_step<D, G, 2>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
-    default: page_step<D, G, 16>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 256 + 8: page_step<D, G, 8, 1, TOPK>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 256 + 4: page_step<D, G, 4, 1, TOPK>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 8: page_step<D, G, 8, 0, TOPK>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 4: page_step<D, G, 4, 0, TOPK>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    case 2: page_step<D, G, 2, 0, TOPK>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
+    default: page_step<D, G, 16, 0, TOPK>(S, blk, mask, scale_log2, pbuf, tk, Gq); break;
   }
 }
 
@@ -848,7 +852,7 @@ __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P,
   return m;
 }
 
-template <int D, int G>
+template <int D, int G, bool TOPK>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_split_kernel(DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -981,7 +985,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       if (seg >= 0) {
         int64_t Us, Ue;
         seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
-        seg_end<D, G>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
+        seg_end<D, G, TOPK>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
       }
       seg = useg;
       seg_begin<D, G>(S, p, reinterpret_cast<const uint16_t*>(blk + p.q_off),
@@ -989,7 +993,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       __syncwarp();
     }
     const uint32_t mask = __shfl_sync(0xFFFFFFFFu, cur.mask, kk);
-    page_dispatch<D, G>(S, blk, p.bits[cs >> 24], mask & 0xFFFFu, p.scale_log2, pbuf, tk, p.Gq);
+    page_dispatch<D, G, TOPK>(S, blk, p.bits[cs >> 24], mask & 0xFFFFu, p.scale_log2, pbuf, tk, p.Gq);
     __syncwarp();
     // refill this stage with unit k + nstage (from this batch of 32 or the next)
     const int kn = k + p.nstage;
@@ -1003,7 +1007,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   {
     int64_t Us, Ue;
     seg_range(p, P, seg / p.Hkv, seg % p.Hkv, &Us, &Ue);
-    seg_end<D, G>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
+    seg_end<D, G, TOPK>(S, p, w, seg, tk, Us >= U0 && Ue <= U1);
   }
 }
 
@@ -1175,8 +1179,8 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   if (lane == 0) p.mass[mrow] = sum / sL[r];
 }
 
-template <int D, int G>
-cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
+template <int D, int G, bool TOPK>
+cudaError_t launch_split_t(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
   // raise the dynamic shared-memory limit of this instantiation once per
   // device (and again whenever a launch needs more); host threads that decode
   // at the same time serialise on the lock, so the recorded size never runs
@@ -1190,18 +1194,24 @@ cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStre
   {
     std::lock_guard<std::mutex> guard(lock);
     if (dl.smem_bytes > configured[dev]) {
-      e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(decode_split_kernel<D, G, TOPK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)dl.smem_bytes);
       if (e != cudaSuccess) return e;
       configured[dev] = dl.smem_bytes;
     }
   }
-  e = launch_pdl(decode_split_kernel<D, G>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
+  e = launch_pdl(decode_split_kernel<D, G, TOPK>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
                  stream, p);
   if (e != cudaSuccess) return e;
   // the combine: one CTA per segment (most return at once)
   return launch_pdl(decode_combine_kernel<D>, dim3((unsigned)(p.n * p.Hkv)),
                     dim3(kCombineThreads), 0, stream, p);
+}
+
+// the top-k candidate code is compiled only into the instantiation that uses it
+template <int D, int G>
+cudaError_t launch_split(const DecodeParams& p, const DecodeLaunch& dl, cudaStream_t stream) {
+  return p.topk > 0 ? launch_split_t<D, G, true>(p, dl, stream) : launch_split_t<D, G, false>(p, dl, stream);
 }
 
 int plan_smem_bytes(int32_t n) { return ((2 * n + 1) * 4 + 127) / 128 * 128; }

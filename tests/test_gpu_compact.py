@@ -22,7 +22,8 @@ def _dev(a, dt):
 def test_compaction_matches_oracle(seed):
     from mixed_precision_paged_thinkv_b200.binding import ThinKVCache
     rng = np.random.default_rng(seed)
-    ns, L, H, d, G = 5, 700, 2, [64, 128][seed % 2], 32
+    # every (head_dim, group_size) instantiation of the gather: (64|128) x (32|64)
+    ns, L, H, d, G = 5, 700, 2, [64, 128][seed % 2], [32, 64][seed // 2]
     bits = [(8, 4, 2), (16, 4, 2), (2, 8, 16), (4, 4, 8)][seed]
     nb = L // 16 * 3 + 8
     pool = (ns * L // 16 + 8,) * 3
