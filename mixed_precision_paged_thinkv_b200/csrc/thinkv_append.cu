@@ -207,7 +207,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   __shared__ int s_total[3];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int max_seqs = C.L.max_seqs, nb_max = C.L.max_blocks_per_seq;
-  const int64_t cap = (int64_t)nb_max * kPage;
 
   if (tid == 0) {
     s_err = (*C.status != 0) ? -1 : 0;

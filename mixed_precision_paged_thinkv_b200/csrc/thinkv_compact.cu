@@ -25,10 +25,10 @@
 //     again and writes every moved token's source slot, destination FIFO
 //     entry and slot position.
 //   compact_copy_kernel: one warp per (dst page, kv-head) gathers the
-//     page-head block in shared memory -- K pieces, V half-words and params of
-//     each of its source slots at the new slot, every two- or four-byte unit
-//     a load of its own, eight per lane in flight -- and writes it out with
-//     16-byte stores.
+//     page-head block in shared memory -- each source slot's K pieces (whole,
+//     up to 16 bytes), V half-words and params words at the new slot, a load
+//     per unit, sixteen per lane in flight -- and writes it out with 16-byte
+//     stores.
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
@@ -41,7 +41,10 @@ namespace {
 constexpr int kCompactThreads = 1024;
 constexpr int kCompactWarps = kCompactThreads / 32;
 constexpr int kCopyWarps = 8;
-constexpr int kCopyBatch = 8;      // gather loads in flight per lane (compact_copy_kernel)
+constexpr int kCopyBlocks = 2;    // resident copy CTAs per SM (128 registers)
+// gather loads in flight per lane (compact_copy_kernel): 8 narrow units, or
+// 64 bytes of 8- and 16-byte units
+template <int N> __host__ __device__ constexpr int copy_batch() { return N >= 8 ? 64 / N : 8; }
 
 // Block-wide exclusive scan (kCompactThreads threads) of one int per thread.
 __device__ int block_scan(int v, int* sh, int* total) {
@@ -301,7 +304,6 @@ struct SlotUnits {
   static constexpr int KU = NG * 4 * HW;
   static constexpr int Q = B == 16 ? D / 8 : D * B / 128;
   static constexpr int KVU = 8 * Q;
-  static constexpr int PER = KU + KVU + (B < 16 ? 2 * NG : 0);
   static constexpr int PHB = B == 16 ? 64 * D : 4 * D * B + 128 * NG;
   static constexpr int CH = LB < 16 ? LB : 16;          // chunk bytes
 
@@ -331,41 +333,78 @@ struct SlotUnits {
   }
 };
 
-// One page-head block gathered into the warp's shared-memory image db: the
-// used slots' units, lane-strided, kCopyBatch loads in flight per lane before
-// their stores.  srcl: lane sl holds slot sl's source pool slot (page*16+slot).
+// Loads and stores of one unit of N bytes (N = 2, 4, 8 or 16).
+template <int N> struct UnitT;
+template <> struct UnitT<2> { using T = uint16_t; };
+template <> struct UnitT<4> { using T = uint32_t; };
+template <> struct UnitT<8> { using T = uint2; };
+template <> struct UnitT<16> { using T = uint4; };
+
+// Copies `total` units of N bytes into the warp's image db, lane-strided,
+// copy_batch<N>() loads in flight per lane before their stores.  at(x, &so, &dof,
+// &sb) gives unit x's source block, source offset and image offset.
+template <int N, typename At>
+__device__ __forceinline__ void gather_units(int total, uint8_t* db, At at) {
+  using T = typename UnitT<N>::T;
+  constexpr int NB = copy_batch<N>();
+  const int lane = threadIdx.x & 31;
+  for (int x0 = 0; x0 < total; x0 += 32 * NB) {     // warp-uniform trip count
+    T val[NB];
+    int dst[NB];                                  // image offset; -1: none
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      const int x = x0 + j * 32 + lane;
+      int so = 0, dof = -1;
+      const uint8_t* sb = nullptr;
+      at(x < total ? x : total - 1, &so, &dof, &sb);   // shuffles inside: every lane takes part
+      dst[j] = x < total ? dof : -1;
+      if (x < total) val[j] = *reinterpret_cast<const T*>(sb + so);
+    }
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+      if (dst[j] >= 0) *reinterpret_cast<T*>(db + dst[j]) = val[j];
+  }
+}
+
+// One page-head block gathered into the warp's shared-memory image db.  K
+// moves as whole pieces (units of up to 16 bytes: a piece never straddles a
+// chunk), then V half-words and (b < 16) the params words.  srcl: lane sl
+// holds slot sl's source pool slot (page * 16 + slot).
 template <int D, int G, int B>
 __device__ __forceinline__ void gather_block(const uint8_t* __restrict__ pool, int H, int h, int32_t srcl, int used,
                              uint8_t* db) {
   using M = SlotUnits<D, G, B>;
-  const int lane = threadIdx.x & 31;
-  const int total = used * M::PER;
-  for (int x0 = 0; x0 < total; x0 += 32 * kCopyBatch) {     // warp-uniform trip count
-    uint32_t val[kCopyBatch];
-    int dst[kCopyBatch];                          // smem offset | 4-byte flag; -1: none
-#pragma unroll
-    for (int j = 0; j < kCopyBatch; ++j) {
-      const int x = x0 + j * 32 + lane;
-      const int sl = min(x / M::PER, used - 1), uu = x - sl * M::PER;
-      const int32_t src = __shfl_sync(0xFFFFFFFFu, srcl, sl);
-      val[j] = 0;
-      dst[j] = -1;
-      if (x < total) {
-        int so, dof;
-        const int sz = M::offsets(uu, src & 15, sl, &so, &dof);
-        const uint8_t* sb = pool + ((int64_t)(src >> 4) * H + h) * M::PHB;
-        val[j] = sz == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(sb + so)
-                         : *reinterpret_cast<const uint32_t*>(sb + so);
-        dst[j] = dof | (sz == 4 ? (1 << 30) : 0);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kCopyBatch; ++j) {
-      if (dst[j] < 0) continue;
-      const int dof = dst[j] & ((1 << 30) - 1);
-      if (dst[j] & (1 << 30)) *reinterpret_cast<uint32_t*>(db + dof) = val[j];
-      else *reinterpret_cast<uint16_t*>(db + dof) = (uint16_t)val[j];
-    }
+  constexpr int KPU = M::PB < 16 ? M::PB : 16;          // K unit bytes
+  constexpr int KPN = M::PB / KPU;                      // units per piece
+  constexpr int KPER = 4 * M::NG * KPN;                 // K units per slot
+  auto src_of = [&](int sl, int* ss, const uint8_t** sb) {
+    const int32_t src = __shfl_sync(0xFFFFFFFFu, srcl, sl);
+    *ss = src & 15;
+    *sb = pool + ((int64_t)(src >> 4) * H + h) * M::PHB;
+  };
+  gather_units<KPU>(used * KPER, db, [&](int x, int* so, int* dof, const uint8_t** sb) {
+    const int sl = x / KPER, u = x - sl * KPER;
+    int ss;
+    src_of(sl, &ss, sb);
+    const int kp = u % KPN, t = (u / KPN) % 4, gr = u / KPN / 4;
+    *so = M::lane_at(4 * (ss & 7) + t, (gr * 2 + (ss >> 3)) * M::PB + kp * KPU);
+    *dof = M::lane_at(4 * (sl & 7) + t, (gr * 2 + (sl >> 3)) * M::PB + kp * KPU);
+  });
+  // V half-words (2 bytes) and params words (4 bytes): two passes of one width each
+  gather_units<2>(used * M::KVU, db, [&](int x, int* so, int* dof, const uint8_t** sb) {
+    const int sl = x / M::KVU, u = x - sl * M::KVU;
+    int ss;
+    src_of(sl, &ss, sb);
+    M::offsets(M::KU + u, ss, sl, so, dof);
+  });
+  if constexpr (B < 16) {
+    constexpr int PU = 2 * M::NG;                       // params words per slot
+    gather_units<4>(used * PU, db, [&](int x, int* so, int* dof, const uint8_t** sb) {
+      const int sl = x / PU, u = x - sl * PU;
+      int ss;
+      src_of(sl, &ss, sb);
+      M::offsets(M::KU + M::KVU + u, ss, sl, so, dof);
+    });
   }
 }
 
@@ -381,10 +420,9 @@ __device__ inline void gather_dispatch(int b, const uint8_t* pool, int H, int h,
 }
 
 // (d) one warp per (dst page, kv-head): the page-head block is gathered into
-// shared memory -- every unit of every slot a lane load of its own, a batch
-// of kCopyBatch per lane in flight -- and written out with 16-byte stores
+// shared memory (gather_block) and written out with 16-byte stores
 template <int D, int G>
-__global__ void __launch_bounds__(kCopyWarps * 32)
+__global__ void __launch_bounds__(kCopyWarps * 32, kCopyBlocks)
     compact_copy_kernel(CacheView S, CacheView Dc, int32_t n, CompactWs ws, int max_phb) {
   extern __shared__ __align__(16) uint8_t img[];   // kCopyWarps block images
   if (ws.totals[3] == 0) return;
@@ -432,7 +470,8 @@ cudaError_t launch_copy(const CacheView& S, const CacheView& Dc, int32_t n, cons
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  compact_copy_kernel<D, G><<<num_sms * 4, kCopyWarps * 32, smem, stream>>>(S, Dc, n, ws, max_phb);
+  compact_copy_kernel<D, G><<<num_sms * kCopyBlocks, kCopyWarps * 32, smem, stream>>>(S, Dc, n, ws,
+                                                                                  max_phb);
   return cudaGetLastError();
 }
 
