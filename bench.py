@@ -42,8 +42,10 @@ METRIC = "decode-attention tokens/sec and achieved HBM GB/s (% of B200 peak), 1 
 DEFAULT_WORKLOAD = "churn"
 PER_CONFIG = ["r1-llama-8b", "r1-qwen-14b", "gpt-oss-20b"]
 FLUSH_BYTES = 512 << 20
+# the sources the decode kernels are compiled from (the shared internal header
+# holds host-side declarations only)
 DECODE_SRC = [os.path.join(ROOT, "mixed_precision_paged_thinkv_b200", "csrc", f)
-              for f in ("thinkv_decode.cu", "thinkv_common.cuh", "thinkv_internal.h")]
+              for f in ("thinkv_decode.cu", "thinkv_common.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 

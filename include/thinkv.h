@@ -311,6 +311,33 @@ THINKV_API int thinkv_evict_tbe(const thinkv_cache* cache, const thinkv_tbe* tbe
                                 int32_t t_min, const int32_t* schedule, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Workspace bytes thinkv_evict_slots needs for n_victims victims. */
+THINKV_API size_t thinkv_evict_slots_workspace_bytes(int32_t n_victims);
+
+/* Explicit victims: the eviction step a policy drives when it chooses the
+ * victims itself (explainer, Methodologie, "Eviction Adaptative a la Pensee
+ * (TBE)": segment-level eviction chosen by a policy; "Implementation Systeme:
+ * Pensee Continue (CT)": an evicted slot is marked in the block table and
+ * refilled in place later).  Victim i is the token at FIFO counter
+ * fifo_index[i] of the class cls[i] FIFO of sequence seq[i]; the counters of
+ * a (sequence, class) FIFO run from fifo_head to fifo_tail - 1, in arrival
+ * order.  Victims go in call order, each like a TBE victim: live bit cleared,
+ * slot_pos -1, slot pushed onto its class's free stack, FIFO entry made a
+ * tombstone (-1) that thinkv_evict steps over.  A victim whose entry is
+ * already a tombstone (evicted before, or named earlier in the call) is
+ * skipped.  A sequence out of range, a class above 2, a counter outside
+ * [fifo_head, fifo_tail) or a sequence whose victims are not contiguous in the
+ * call -> *status = INVALID and nothing changes; while *status != 0 the call
+ * does nothing.  TBE counts a segment's live tokens as a suffix of it, so a
+ * cache driven by thinkv_evict_tbe should not also take victims from inside
+ * its segments.
+ * seq, fifo_index: device int32 [n_victims] (4-byte aligned); cls: device
+ * uint8 [n_victims].  workspace: device, >= thinkv_evict_slots_workspace_bytes
+ * (n_victims) bytes, no initialisation needed.  One kernel. */
+THINKV_API int thinkv_evict_slots(const thinkv_cache* cache, int32_t n_victims, const int32_t* seq,
+                                  const uint8_t* cls, const int32_t* fifo_index, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* Workspace bytes thinkv_compact needs for n_seqs sequences holding at most
  * max_tokens live tokens together. */
 THINKV_API size_t thinkv_compact_workspace_bytes(int32_t n_seqs, int32_t max_tokens);

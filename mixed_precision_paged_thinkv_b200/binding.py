@@ -35,6 +35,7 @@ EXPORTED = [
     "thinkv_get_status", "thinkv_clear_status", "thinkv_status_string",
     "thinkv_decode_attention_noalloc", "thinkv_classify_thoughts",
     "thinkv_tbe_buffer_bytes", "thinkv_tbe_reset", "thinkv_tbe_workspace_bytes", "thinkv_evict_tbe",
+    "thinkv_evict_slots_workspace_bytes", "thinkv_evict_slots",
     "thinkv_compact_workspace_bytes", "thinkv_compact",
 ]
 
@@ -111,6 +112,10 @@ def lib():
             L.thinkv_tbe_buffer_bytes.restype = SZ
             L.thinkv_tbe_reset.argtypes = [C.POINTER(Layout), C.POINTER(TbeStruct), P]
             L.thinkv_tbe_reset.restype = C.c_int
+            L.thinkv_evict_slots_workspace_bytes.argtypes = [I32]
+            L.thinkv_evict_slots_workspace_bytes.restype = SZ
+            L.thinkv_evict_slots.argtypes = [C.POINTER(CacheStruct), I32, P, P, P, P, SZ, P]
+            L.thinkv_evict_slots.restype = C.c_int
             L.thinkv_tbe_workspace_bytes.argtypes = [I32]
             L.thinkv_tbe_workspace_bytes.restype = SZ
             L.thinkv_evict_tbe.argtypes = [C.POINTER(CacheStruct), C.POINTER(TbeStruct), I32, P, P, P,
@@ -229,6 +234,18 @@ class ThinKVCache:
         if self.tbe is not None:
             _check(lib().thinkv_tbe_reset(C.byref(self.layout), C.byref(self.tbe), _stream(stream)),
                    "tbe_reset")
+
+    def evict_slots(self, seq: torch.Tensor, cls: torch.Tensor, fifo_index: torch.Tensor, stream=None):
+        """Explicit victims: (sequence, class, FIFO counter) each, evicted in order."""
+        n = int(seq.numel())
+        if n == 0:
+            return
+        assert seq.dtype == torch.int32 and cls.dtype == torch.uint8 and fifo_index.dtype == torch.int32
+        assert cls.numel() == n and fifo_index.numel() == n
+        nbytes = int(lib().thinkv_evict_slots_workspace_bytes(n))
+        ws = self._workspace("evict_slots", nbytes)
+        _check(lib().thinkv_evict_slots(C.byref(self.cs), n, _ptr(seq), _ptr(cls), _ptr(fifo_index),
+                                        _ptr(ws), ws.numel(), _stream(stream)), "evict_slots")
 
     def evict_tbe(self, seq: torch.Tensor, pos: torch.Tensor, tag: torch.Tensor, t_min: int = 0,
                   schedule: Optional[Sequence[int]] = None, stream=None):

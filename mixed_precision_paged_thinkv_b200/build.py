@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libthinkv.so")
 SOURCES = ["thinkv_api.cu", "thinkv_append.cu", "thinkv_evict.cu", "thinkv_decode.cu",
            "thinkv_noalloc.cu", "thinkv_classify.cu", "thinkv_tbe.cu",
-           "thinkv_compact.cu"]
+           "thinkv_compact.cu", "thinkv_victims.cu"]
 HEADERS = ["thinkv_common.cuh", "thinkv_internal.h"]
 
 NVCC_FLAGS = [

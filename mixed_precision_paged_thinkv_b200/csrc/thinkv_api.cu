@@ -273,6 +273,25 @@ int thinkv_evict_tbe(const thinkv_cache* C, const thinkv_tbe* T, int32_t n, cons
                                 static_cast<cudaStream_t>(stream)));
 }
 
+size_t thinkv_evict_slots_workspace_bytes(int32_t n_victims) {
+  if (n_victims < 0) return 0;
+  return ((size_t)(n_victims > 0 ? n_victims : 1) * 4 + 255) / 256 * 256;
+}
+
+int thinkv_evict_slots(const thinkv_cache* C, int32_t n, const int32_t* seq, const uint8_t* cls,
+                       const int32_t* fifo_index, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!cache_ok(C) || n < 0) return THINKV_ERR_INVALID;
+  if (n == 0) return THINKV_OK;
+  if (!seq || !cls || !fifo_index || !aligned(seq, 4) || !aligned(fifo_index, 4))
+    return THINKV_ERR_INVALID;
+  if (workspace && !aligned(workspace, 16)) return THINKV_ERR_INVALID;
+  if (!workspace || workspace_bytes < thinkv_evict_slots_workspace_bytes(n)) return THINKV_ERR_WORKSPACE;
+  return cuda_status(launch_evict_slots(view_of(C), n, seq, cls, fifo_index,
+                                        static_cast<int32_t*>(workspace),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 size_t thinkv_compact_workspace_bytes(int32_t n_seqs, int32_t max_tokens) {
   if (n_seqs < 0 || max_tokens < 0) return 0;
   return compact_workspace_bytes(n_seqs, max_tokens);

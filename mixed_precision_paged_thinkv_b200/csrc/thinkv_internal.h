@@ -89,6 +89,10 @@ cudaError_t launch_tbe(const CacheView& C, int4* seg, int32_t* nseg, int32_t* se
                        const int32_t* seq, const int32_t* pos, const uint8_t* tag, int32_t t_min,
                        const int32_t schedule[3], int32_t* run_start, cudaStream_t stream);
 
+// explicit victims
+cudaError_t launch_evict_slots(const CacheView& C, int32_t n, const int32_t* seq, const uint8_t* cls,
+                               const int32_t* idx, int32_t* run_start, cudaStream_t stream);
+
 // gather compaction (the step CT avoids; a baseline)
 size_t compact_workspace_bytes(int32_t n, int32_t max_tokens);
 cudaError_t launch_compact(const CacheView& S, const CacheView& Dc, int32_t n, const int32_t* seq,

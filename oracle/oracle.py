@@ -81,6 +81,7 @@ def lib():
                 getattr(L, f).restype = C.c_uint8
             L.or_classify.argtypes = [C.c_int32, C.c_int32, P, C.c_float, C.c_float, P]
             L.or_tbe.argtypes = [P, C.c_int32, P, P, P, C.c_int32, P]
+            L.or_evict_slots.argtypes = [P, C.c_int32, P, P, P]
             L.or_compact.argtypes = [P, P, C.c_int32, P]
             for f in ("or_codes", "or_params", "or_slot_pos"):
                 getattr(L, f).argtypes = [P, C.c_int]
@@ -228,6 +229,13 @@ class Oracle:
         sch = None if schedule is None else np.ascontiguousarray(schedule, dtype=np.int32)
         return int(lib().or_tbe(self._h, seq.shape[0], _ptr(seq), _ptr(pos), _ptr(tag),
                                 int(t_min), None if sch is None else _ptr(sch)))
+
+    def evict_slots(self, seq, cls, idx) -> int:
+        """Explicit victims: (sequence, class, FIFO counter) each (see or_evict_slots)."""
+        seq = np.ascontiguousarray(seq, dtype=np.int32)
+        cls = np.ascontiguousarray(cls, dtype=np.uint8)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        return int(lib().or_evict_slots(self._h, seq.shape[0], _ptr(seq), _ptr(cls), _ptr(idx)))
 
     def compact_into(self, dst: "Oracle", seq) -> int:
         """Gather the live tokens of `seq` into the empty oracle `dst` (see or_compact)."""

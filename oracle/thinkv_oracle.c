@@ -536,6 +536,48 @@ int or_evict(or_state* S, int32_t n, const int32_t* seq, const int32_t* budget,
 }
 
 /* ====================================================================== */
+/* explicit victims                                                        */
+/* ====================================================================== */
+/* The eviction step a policy drives directly (the explicit-victim call TBE
+ * needs when the policy runs on the host).  Victim i is the token at FIFO
+ * counter idx[i] of the class cls[i] FIFO of sequence seq[i]
+ * (head <= idx < tail).  Victims go in call order, each like a TBE victim:
+ * mask bit cleared, start index -1, slot pushed onto its class's free stack,
+ * FIFO entry made a tombstone (-1).  A victim whose entry is already a
+ * tombstone (evicted before, or named earlier in the call) is skipped.  The
+ * call is all-or-nothing on its arguments: a sequence out of range, a class
+ * above 2, a counter outside its FIFO window, or a sequence whose victims are
+ * not contiguous in the call make it invalid, and nothing changes. */
+int or_evict_slots(or_state* S, int32_t n, const int32_t* seq, const uint8_t* cls,
+                   const int32_t* idx) {
+  const or_layout* L = &S->L;
+  if (n < 0) return OR_ERR_INVALID;
+  char* seen = (char*)calloc((size_t)L->max_seqs, 1);
+  for (int32_t i = 0; i < n; ++i) {
+    int s = seq[i];
+    if (s < 0 || s >= L->max_seqs || cls[i] > 2) { free(seen); return OR_ERR_INVALID; }
+    int c = cls[i];
+    if (idx[i] < S->fifo_head[s * 3 + c] || idx[i] >= S->fifo_tail[s * 3 + c]) {
+      free(seen);
+      return OR_ERR_INVALID;
+    }
+    if (i == 0 || seq[i - 1] != s) {             /* a new run of victims */
+      if (seen[s]) { free(seen); return OR_ERR_INVALID; }
+      seen[s] = 1;
+    }
+  }
+  free(seen);
+  for (int32_t i = 0; i < n; ++i) {
+    int s = seq[i], c = cls[i];
+    int32_t* entry = &fifo_ring(S, s, c)[idx[i] % S->cap];
+    if (*entry < 0) continue;                    /* already a tombstone */
+    evict_token(S, s, c, *entry);
+    *entry = -1;
+  }
+  return OR_OK;
+}
+
+/* ====================================================================== */
 /* TBE: segment-level eviction on Transition thoughts                      */
 /* ====================================================================== */
 /* Explainer, Methodologie, "Eviction Adaptative a la Pensee (TBE)": when a

@@ -72,6 +72,15 @@ int or_decode(const or_state* S, int32_t n, const int32_t* seq,
 int or_tbe(or_state* S, int32_t n, const int32_t* seq, const int32_t* pos, const uint8_t* tag,
            int32_t t_min, const int32_t* schedule);
 
+/* Explicit victims: victim i is the token at FIFO counter idx[i] of the
+ * class cls[i] FIFO of sequence seq[i] (head <= idx < tail), evicted in call
+ * order (mask bit, start index -1, free-stack push, FIFO tombstone); a victim
+ * whose entry is already a tombstone is skipped.  Invalid (nothing changes): a
+ * sequence out of range, a class above 2, a counter outside the window, a
+ * sequence whose victims are not contiguous in the call. */
+int or_evict_slots(or_state* S, int32_t n, const int32_t* seq, const uint8_t* cls,
+                   const int32_t* idx);
+
 /* Gather compaction (what CT avoids): the live tokens of seq[0..n) move into
  * fresh hole-free pages of the empty cache dst (same geometry), class by
  * class, FIFO order within a class, codes copied. */

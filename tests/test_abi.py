@@ -172,3 +172,32 @@ def test_classify_host_validation(lib):
     assert f(4, 4, None, C.c_float(0.5), C.c_float(0.2), ok, None) == 1
     assert f(4, 4, C.c_void_p(4098), C.c_float(0.5), C.c_float(0.2), ok, None) == 1
     assert f(0, 4, None, C.c_float(0.5), C.c_float(0.2), None, None) == 0
+
+
+def test_evict_slots_host_validation(lib):
+    """thinkv_evict_slots refuses bad counts, missing or misaligned arrays and a
+    short workspace before any CUDA call; zero victims is a no-op."""
+    from mixed_precision_paged_thinkv_b200 import binding
+    cs = binding.CacheStruct()
+    cs.L = _layout()
+    for name, _ in binding.CacheStruct._fields_[1:]:
+        v = getattr(cs, name)
+        if isinstance(v, C.Array):
+            for i in range(3):
+                v[i] = 4096
+        else:
+            setattr(cs, name, 4096)
+    ok, odd = C.c_void_p(4096), C.c_void_p(4096 + 2)
+    f = lib.thinkv_evict_slots
+    need = lib.thinkv_evict_slots_workspace_bytes(8)
+    assert need >= 8 * 4 and lib.thinkv_evict_slots_workspace_bytes(-1) == 0
+    assert f(C.byref(cs), -1, ok, ok, ok, ok, need, None) == 1
+    assert f(C.byref(cs), 8, None, ok, ok, ok, need, None) == 1
+    assert f(C.byref(cs), 8, ok, None, ok, ok, need, None) == 1
+    assert f(C.byref(cs), 8, ok, ok, None, ok, need, None) == 1
+    assert f(C.byref(cs), 8, odd, ok, ok, ok, need, None) == 1        # seq not 4-byte aligned
+    assert f(C.byref(cs), 8, ok, ok, odd, ok, need, None) == 1        # fifo_index likewise
+    assert f(C.byref(cs), 8, ok, ok, ok, C.c_void_p(4096 + 4), need, None) == 1   # workspace
+    assert f(C.byref(cs), 8, ok, ok, ok, ok, need - 1, None) == binding.ERR_WORKSPACE
+    assert f(C.byref(cs), 8, ok, ok, ok, None, need, None) == binding.ERR_WORKSPACE
+    assert f(C.byref(cs), 0, None, None, None, None, 0, None) == 0
