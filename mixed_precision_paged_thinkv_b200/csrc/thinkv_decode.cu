@@ -16,8 +16,9 @@
 //   unpacks codes straight into mma.sync m16n8k16 operands (byte-permute
 //   conversion to fp16 1024 + code), computes q.k for the whole GQA group at
 //   once (tokens x heads), applies the per-group scale/zero in fp32, runs the
-//   online softmax, transposes p through a small shared buffer and accumulates
-//   p*scale (fp16, exponent-shifted) times the centred V codes on the tensor
+//   online softmax, forms p*scale (fp16, exponent-shifted) where the logits
+//   are and moves it into the PV operand layout with register transposes
+//   (movmatrix), and accumulates it times the centred V codes on the tensor
 //   cores, with the zero terms summed in fp32.  A segment (sequence, kv-head)
 //   that lies wholly in one warp is written out at once; otherwise each warp
 //   writes one piece record (m, l, o, top-k logits) per segment it touched.
@@ -42,15 +43,11 @@ constexpr int kDecWarps = 4;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecMinBlocks = 3;                       // CTAs per SM the kernel is built for
 constexpr int kDecRegs = 65536 / (kDecThreads * kDecMinBlocks) / 8 * 8;  // register cap (168)
-constexpr int kPbufStride = 12;                 // floats per row of the p transpose buffer
-// per-warp scratch: during pages, the p transpose (16 x 12 floats) and the
-// segment's Q fragments (lane-contiguous, up to 2 KB); during a merge, which
-// runs between two segments, the (m, l) table of the pieces (32 x 8 float2 +
-// 16 floats) overlays both
-constexpr int kPtBytes = 16 * kPbufStride * 4;          // 768
-constexpr int kQfragOff = kPtBytes;
+// per-warp scratch: the segment's Q fragments, lane-contiguous (the B
+// operands of the QK products)
+constexpr int kQfragOff = 0;
 constexpr int kQfragBytes = 2048;                       // (D / 16) k-steps x 32 lanes x 8 B
-constexpr int kPbufBytes = kPtBytes + kQfragBytes;      // >= 2 * 32 * 8 * 4 + 16 * 4
+constexpr int kPbufBytes = kQfragBytes;
 constexpr int kSigmaInit = 1 << 20;
 constexpr int kMaxStages = 8;                   // page ring stages (one mbarrier each)
 constexpr int kCandCap = 128;                   // top-k candidate slots per head
@@ -458,6 +455,15 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
   __syncwarp();
 }
 
+// Transpose of an 8x8 matrix of 16-bit elements held one register per lane
+// (lane 4r + c holds row r, columns 2c and 2c + 1): afterwards the lane holds
+// row r of the transpose, i.e. column r of the original.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 // Words [w0, w0 + NW) of this lane's portion of a code region laid out in
 // chunks of U = min(16, LB) bytes interleaved over the 32 lanes (see
 // lane_off); `base` is the region + lane * U.  w0 and NW are multiples of U/4,
@@ -638,12 +644,18 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
   S.lp[0] = fmaf(S.lp[0], a0, pr[0] + pr[2]);
   S.lp[1] = fmaf(S.lp[1], a1, pr[1] + pr[3]);
 
-  if constexpr (B != 16) {
+  // V scales of this lane's tokens g and g + 8, per group (the rows the zero term reads)
+  float s0[NG], s1[NG];
 #pragma unroll
-    for (int gr = 0; gr < NG; ++gr) {
+  for (int gr = 0; gr < NG; ++gr) {
+    if constexpr (B == 16) {
+      s0[gr] = s1[gr] = 1.f;
+    } else {
       const uint32_t p0 = vpar[gr * 16 + g], p1 = vpar[gr * 16 + g + 8];
       const float2 sz0 = __half22float2(*reinterpret_cast<const __half2*>(&p0));
       const float2 sz1 = __half22float2(*reinterpret_cast<const __half2*>(&p1));
+      s0[gr] = sz0.x;
+      s1[gr] = sz1.x;
       constexpr float voff = F == 1 ? 0.f : (float)(1 << (B - 1));
       const float zv0 = live0 ? fmaf(voff, sz0.x, sz0.y) : 0.f;
       const float zv1 = live1 ? fmaf(voff, sz1.x, sz1.y) : 0.f;
@@ -652,61 +664,41 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
     }
   }
 
-  // ---------------- p transpose: (tokens gid, gid+8 ; heads 2t, 2t+1) ->
-  //                  (tokens 2t, 2t+1, 2t+8, 2t+9 ; head gid) ----------------
-  *reinterpret_cast<float2*>(pbuf + g * kPbufStride + 2 * t) = make_float2(pr[0], pr[1]);
-  *reinterpret_cast<float2*>(pbuf + (g + 8) * kPbufStride + 2 * t) = make_float2(pr[2], pr[3]);
-  __syncwarp();
-  float pt[4];
-  pt[0] = pbuf[(2 * t) * kPbufStride + g];
-  pt[1] = pbuf[(2 * t + 1) * kPbufStride + g];
-  pt[2] = pbuf[(2 * t + 8) * kPbufStride + g];
-  pt[3] = pbuf[(2 * t + 9) * kPbufStride + g];
+  // ---------------- PV operands W = p * s_V * 2^sigma (one sigma per segment),
+  //   formed where the logits are (tokens g, g+8; heads 2t, 2t+1), packed to
+  //   fp16 and moved to the B-operand layout (tokens 2t, 2t+1, 2t+8, 2t+9;
+  //   head g) by an 8x8 register transpose per token half ----------------
+  // dead slots of the V operand (float codes, raw fp16): zeroed in the A operand
   const uint32_t tmask = mask >> (2 * t);
-  const bool tl[4] = {(tmask & 1u) != 0, (tmask & 2u) != 0, (tmask & 0x100u) != 0,
-                      (tmask & 0x200u) != 0};
-
-  // ---------------- PV operands W = p * s_V * 2^sigma (one sigma per segment) ----------------
-  float sv[NG][4];
-#pragma unroll
-  for (int gr = 0; gr < NG; ++gr) {
-    if constexpr (B == 16) {
-      sv[gr][0] = sv[gr][1] = sv[gr][2] = sv[gr][3] = 1.f;
-    } else {
-      const uint2 q0 = *reinterpret_cast<const uint2*>(vpar + gr * 16 + 2 * t);
-      const uint2 q1 = *reinterpret_cast<const uint2*>(vpar + gr * 16 + 2 * t + 8);
-      sv[gr][0] = __half2float(__ushort_as_half((uint16_t)(q0.x & 0xFFFFu)));
-      sv[gr][1] = __half2float(__ushort_as_half((uint16_t)(q0.y & 0xFFFFu)));
-      sv[gr][2] = __half2float(__ushort_as_half((uint16_t)(q1.x & 0xFFFFu)));
-      sv[gr][3] = __half2float(__ushort_as_half((uint16_t)(q1.y & 0xFFFFu)));
-    }
-  }
-  // dead slots: p is 0, their scale bytes are stale; zero the packed operand instead
-  const uint32_t dm0 = (tl[0] ? 0xFFFFu : 0u) | (tl[1] ? 0xFFFF0000u : 0u);
-  const uint32_t dm1 = (tl[2] ? 0xFFFFu : 0u) | (tl[3] ? 0xFFFF0000u : 0u);
+  const uint32_t dm0 = ((tmask & 1u) ? 0xFFFFu : 0u) | ((tmask & 2u) ? 0xFFFF0000u : 0u);
+  const uint32_t dm1 = ((tmask & 0x100u) ? 0xFFFFu : 0u) | ((tmask & 0x200u) ? 0xFFFF0000u : 0u);
   float f = S.sigma == kSigmaInit ? 0.f : pow2i(S.sigma);
   float wv[NG][4];
   float wmax = 0.f;
 #pragma unroll
-  for (int gr = 0; gr < NG; ++gr)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      wv[gr][j] = pt[j] * f * sv[gr][j];
-      wmax = tl[j] ? fmaxf(wmax, wv[gr][j]) : wmax;
-    }
+  for (int gr = 0; gr < NG; ++gr) {
+    wv[gr][0] = pr[0] * f * s0[gr];
+    wv[gr][1] = pr[1] * f * s0[gr];
+    wv[gr][2] = pr[2] * f * s1[gr];
+    wv[gr][3] = pr[3] * f * s1[gr];
+    wmax = live0 ? fmaxf(wmax, fmaxf(wv[gr][0], wv[gr][1])) : wmax;
+    wmax = live1 ? fmaxf(wmax, fmaxf(wv[gr][2], wv[gr][3])) : wmax;
+  }
   float fac = 1.f;
   // slow path: first page of the segment, or a scale large enough to overflow fp16
   if (__any_sync(0xFFFFFFFFu, S.sigma == kSigmaInit || !(wmax < 32768.f))) {
     int e5 = 1;
 #pragma unroll
-    for (int gr = 0; gr < NG; ++gr)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int ef = (__float_as_int(sv[gr][j]) >> 23) - 112;  // fp16 exponent field
-        e5 = tl[j] ? max(e5, ef) : e5;
-      }
-    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 1));
-    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 2));
+    for (int gr = 0; gr < NG; ++gr) {
+      const int ef0 = (__float_as_int(s0[gr]) >> 23) - 112;   // fp16 exponent field
+      const int ef1 = (__float_as_int(s1[gr]) >> 23) - 112;
+      e5 = live0 ? max(e5, ef0) : e5;
+      e5 = live1 ? max(e5, ef1) : e5;
+    }
+    // over the page's 16 tokens: the lanes of other g hold the other tokens
+    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 4));
+    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 8));
+    e5 = max(e5, __shfl_xor_sync(0xFFFFFFFFu, e5, 16));
     const int sp = 29 - e5;             // s * 2^sp < 2^15 for every live scale of the page
     if (sp < S.sigma) {
       if (S.sigma != kSigmaInit) fac = pow2i(sp - S.sigma);
@@ -714,15 +706,21 @@ __device__ inline void page_step(SegState<D, G>& S, const uint8_t* blk, uint32_t
     }
     f = pow2i(S.sigma);
 #pragma unroll
-    for (int gr = 0; gr < NG; ++gr)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) wv[gr][j] = pt[j] * f * sv[gr][j];
+    for (int gr = 0; gr < NG; ++gr) {
+      wv[gr][0] = pr[0] * f * s0[gr];
+      wv[gr][1] = pr[1] * f * s0[gr];
+      wv[gr][2] = pr[2] * f * s1[gr];
+      wv[gr][3] = pr[3] * f * s1[gr];
+    }
   }
   uint32_t wf[NG][2];
 #pragma unroll
   for (int gr = 0; gr < NG; ++gr) {
-    wf[gr][0] = pack_half2_rn(wv[gr][0], wv[gr][1]) & dm0;
-    wf[gr][1] = pack_half2_rn(wv[gr][2], wv[gr][3]) & dm1;
+    // dead tokens: p is 0, but their stale scales may not be finite
+    const uint32_t lo = live0 ? pack_half2_rn(wv[gr][0], wv[gr][1]) : 0u;   // token g
+    const uint32_t hi = live1 ? pack_half2_rn(wv[gr][2], wv[gr][3]) : 0u;   // token g + 8
+    wf[gr][0] = movmatrix_trans(lo);    // head g: tokens 2t, 2t+1
+    wf[gr][1] = movmatrix_trans(hi);    // head g: tokens 2t+8, 2t+9
   }
   if (__any_sync(0xFFFFFFFFu, a0 != 1.f || a1 != 1.f || fac != 1.f)) {
     const float r0 = a0 * fac, r1 = a1 * fac;
