@@ -21,12 +21,13 @@
 //   (movmatrix), and accumulates it times the centred V codes on the tensor
 //   cores, with the zero terms summed in fp32.  A segment (sequence, kv-head)
 //   that lies wholly in one warp is written out at once; otherwise each warp
-//   writes one piece record (m, l, o, top-k logits) per segment it touched.
+//   writes one piece record (m, l, o, top-k candidates) per segment it touched.
 //
 //   combine kernel (launched right behind, programmatic dependent launch): one
 //   CTA per segment left in several pieces merges the records with the
 //   log-sum-exp rule -- a thread per quad of each head's output row, a warp per
-//   head for the top-k lists -- and writes fp16 O and the top-k mass.
+//   head sorting and merging the pieces' top-k candidates -- and writes fp16 O
+//   and the top-k mass.
 #include <cuda_fp16.h>
 #include <limits.h>
 #include <mutex>
@@ -263,11 +264,11 @@ __device__ inline void cand_compact(const TopkCtx& tk, int h) {
 //   [0, 64)                 (m, l) of query heads 0..7 (m in log2 units, l the
 //                           row sum relative to m)
 //   [64, 64 + 4*Gq*D)       the unnormalised output rows o[Gq][D]
-//   then 4*Gq*kpad bytes    per head, the top-k largest logits, descending,
-//                           -inf padded (kpad = topk rounded up to 4)
+//   then (with the top-k statistic) 4*Gq*kCandCap bytes: per head, the
+//                           piece's candidate logits -- a superset of its topk
+//                           largest -- unsorted, -inf padded
 __host__ __device__ inline int64_t record_bytes(int Gq, int D, int topk) {
-  const int kpad = (topk + 3) / 4 * 4;
-  return 64 + 4LL * Gq * D + 4LL * Gq * kpad;
+  return 64 + 4LL * Gq * D + (topk > 0 ? 4LL * Gq * kCandCap : 0);
 }
 
 // Merges a bitonic sequence of 128 values held 4 per lane (element lane*4+j)
@@ -427,26 +428,33 @@ __device__ inline void seg_end(SegState<D, G>& S, const DecodeParams& p, int64_t
     }
   }
   if (TOPK && tk.topk > 0) {
-    const int kpad = (tk.topk + 3) / 4 * 4;
-    const bool all = whole && p.live_count[p.seq[i]] <= tk.topk;
-    float* tl = reinterpret_cast<float*>(rec + 64 + 4 * Gq * D);
-    for (int hd = 0; hd < Gq; ++hd) {
-      float sum = 0.f;
-      if (!all) {
-        if (tk.topk <= 32 && tk.cnt[hd] > 64) cand_prune(tk, hd);   // then the 64-wide sort
-        if (tk.cnt[hd] > 0) cand_compact(tk, hd);      // sorted, the k largest kept
+    if (!whole) {
+      // a piece hands its candidate buffers over as they are (each a superset
+      // of its head's topk largest; -inf past the count): the combine sorts
+      // them, a warp per head
+      float* tl = reinterpret_cast<float*>(rec + 64 + 4 * Gq * D);
+      for (int hd = 0; hd < Gq; ++hd) {
         const int n = tk.cnt[hd];
-        if (whole) {
+        float4 v = *reinterpret_cast<const float4*>(tk.cand + hd * kCandCap + 4 * lane);
+        if (4 * lane + 0 >= n) v.x = -INFINITY;
+        if (4 * lane + 1 >= n) v.y = -INFINITY;
+        if (4 * lane + 2 >= n) v.z = -INFINITY;
+        if (4 * lane + 3 >= n) v.w = -INFINITY;
+        *reinterpret_cast<float4*>(tl + hd * kCandCap + 4 * lane) = v;
+      }
+    } else {
+      const bool all = p.live_count[p.seq[i]] <= tk.topk;
+      for (int hd = 0; hd < Gq; ++hd) {
+        float sum = 0.f;
+        if (!all) {
+          if (tk.topk <= 32 && tk.cnt[hd] > 64) cand_prune(tk, hd);   // then the 64-wide sort
+          if (tk.cnt[hd] > 0) cand_compact(tk, hd);      // sorted, the k largest kept
+          const int n = tk.cnt[hd];
           const float m = __shfl_sync(0xFFFFFFFFu, (hd & 1) ? S.m[1] : S.m[0], hd >> 1);
           for (int j = lane; j < n; j += 32) sum += exp2_approx(tk.cand[hd * kCandCap + j] - m);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        } else {
-          for (int j = lane; j < kpad; j += 32)
-            tl[hd * kpad + j] = j < n ? tk.cand[hd * kCandCap + j] : -INFINITY;
         }
-      }
-      if (whole) {
         const float l = __shfl_sync(0xFFFFFFFFu, (hd & 1) ? S.lp[1] : S.lp[0], hd >> 1);
         if (lane == 0) p.mass[(int64_t)i * p.Hq + h * Gq + hd] = all ? 1.f : sum / l;
       }
@@ -1019,9 +1027,10 @@ constexpr int kCombinePieces = 128;             // pieces per round of the weigh
 constexpr int kCombinePre = 8;                  // pieces whose quads are requested up front
 
 // Merges the segment's piece records with the log-sum-exp rule: thread t <
-// Gq * D/4 owns one quad of one head's output row; warp r < Gq then merges
-// head r's top-k lists (bitonic merges, the next piece's list loaded while the
-// current one merges) for the top-k mass.
+// Gq * D/4 owns one quad of one head's output row; warp r < Gq then sorts each
+// piece's top-k candidates for head r and merges their largest into a running
+// list (bitonic networks, the next piece's candidates loaded while the current
+// ones are sorted) for the top-k mass.
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(DecodeParams p) {
   constexpr int QD = D / 4;
@@ -1040,7 +1049,7 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   const bool by_unit = T <= W;                  // one unit per warp
   const int np = (int)(by_unit ? nl : w1 - w0 + 1);
   if (np <= 1) return;                          // finished inside one split warp
-  const int Gq = p.Gq, k = p.topk, kpad = (k + 3) / 4 * 4;
+  const int Gq = p.Gq, k = p.topk;
   // the top-k warps' live count, requested now and used after the merge
   const int live_i = (p.mass && threadIdx.x < 32 * Gq) ? p.live_count[p.seq[i]] : 0;
   const int64_t rb = record_bytes(Gq, D, k);
@@ -1144,16 +1153,14 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
     if (lane == 0) p.mass[mrow] = 1.f;
     return;
   }
-  // running list (descending) in elements 0..63, the next piece's list
-  // reversed in 64..127: a bitonic sequence
+  // each piece's candidates (128, unsorted) sorted ascending put its 64
+  // largest in elements 64..127, rising; with the running list (descending)
+  // in elements 0..63 that is a bitonic sequence
   float tv[4], nx[4];
   auto load_list = [&](int j, float (&x)[4]) {
-    const float* tl = reinterpret_cast<const float*>(rec(j) + 64 + 4 * Gq * D) + r * kpad;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int el = lane * 4 + e, m = 127 - el;
-      x[e] = (el >= 64 && m < k) ? __ldcg(tl + m) : -INFINITY;
-    }
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(rec(j) + 64 + 4 * Gq * D) +
+                            r * (kCandCap / 4) + lane);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
   };
 #pragma unroll
   for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
@@ -1161,7 +1168,10 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   for (int j = 0; j < np; ++j) {
     float v[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = (lane * 4 + e < 64) ? tv[e] : nx[e];
+    for (int e = 0; e < 4; ++e) v[e] = -nx[e];
+    bitonic128_desc(v);                           // descending of -x: ascending of x
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = (lane * 4 + e < 64) ? tv[e] : -v[e];
     if (j + 1 < np) load_list(j + 1, nx);
     bitonic128_merge_desc(v);
 #pragma unroll
