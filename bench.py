@@ -120,9 +120,9 @@ def traffic_per_launch(workload: str):
 
 
 def launches_per_step(batch: int) -> int:
-    """Kernels one step launches: append (one launch up to 512 tokens, else
-    two), evict, decode (split + combine)."""
-    return (1 if batch <= 512 else 2) + 1 + 2
+    """Kernels one step launches: append + evict (one launch up to 512 tokens,
+    else the append's two and the evict's one), decode (split + combine)."""
+    return (1 if batch <= 512 else 3) + 2
 
 
 def algorithmic_decode_bytes(w, snap) -> int:
@@ -529,12 +529,10 @@ def measure_workload(w, K: int, Wm: int, dev, flush, e2e_steps: int = 0, clocks=
     for k in range(K):
         flush.zero_()
         inp = steps[Wm + k]
-        # no event between the three calls: each kernel may start while the
-        # previous one finishes (programmatic dependent launch)
+        # no event between the two calls (append + evict, decode): each kernel
+        # may start while the previous one finishes (programmatic dependent launch)
         ev[k][0].record()
-        run.cache.append(inp.seqs, inp.pos, inp.tags, inp.k, inp.v)
-        run.cache.evict(inp.seqs, inp.budgets)
-        run.cache.decode(inp.seqs, inp.q, topk=w.topk, out=out, mass=mass)
+        run_step(run.cache, inp, out, topk=w.topk, mass=mass)
         ev[k][1].record()
     torch.cuda.synchronize()
     t_wall = time.time() - t_wall

@@ -248,6 +248,23 @@ THINKV_API int thinkv_append_quantize(const thinkv_cache* cache, int32_t n_token
                            const uint16_t* k, const uint16_t* v,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Append + evict in one call: the tokens are appended exactly as by
+ * thinkv_append_quantize, then each sequence of the call is evicted to its
+ * budget exactly as by thinkv_evict with `order` (host array of the 3 classes
+ * in victim order, NULL for T, E, R).  budget: device int32 [n_tokens], 4-byte
+ * aligned; the value at the first token of each sequence's run is that
+ * sequence's budget (>= 0), the others are not read.  The call is
+ * all-or-nothing: bad token data or a negative budget -> *status = INVALID and
+ * nothing changes (with the other errors of thinkv_append_quantize).  Calls of
+ * up to 512 tokens take one launch: each sequence's evict runs in the CTA that
+ * assigned its slots, right after the assignment, with no second kernel.
+ * Larger calls take the append's two kernels and one evict kernel.
+ * workspace: as for thinkv_append_quantize (same size, same counter rule). */
+THINKV_API int thinkv_append_evict(const thinkv_cache* cache, int32_t n_tokens, const int32_t* seq,
+                                   const int32_t* pos, const uint8_t* tag, const uint16_t* k,
+                                   const uint16_t* v, const int32_t* budget, const uint8_t* order,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Evict to budget (TBE + CT free path).
  * For each i < n_seqs, sequence seq[i] (distinct, in range) keeps at most
  * budget[i] >= 0 live tokens: n = max(0, live_count - budget) victims are the

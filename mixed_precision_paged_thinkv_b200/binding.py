@@ -31,6 +31,7 @@ BUFFERS = ["pool_R", "pool_E", "pool_T", "slot_pos_R", "slot_pos_E", "slot_pos_T
 EXPORTED = [
     "thinkv_layout_check", "thinkv_page_head_bytes", "thinkv_buffer_bytes",
     "thinkv_cache_reset", "thinkv_append_workspace_bytes", "thinkv_append_quantize",
+    "thinkv_append_evict",
     "thinkv_evict", "thinkv_decode_workspace_bytes", "thinkv_decode_attention",
     "thinkv_get_status", "thinkv_clear_status", "thinkv_status_string",
     "thinkv_decode_attention_noalloc", "thinkv_classify_thoughts",
@@ -96,6 +97,8 @@ def lib():
             L.thinkv_append_workspace_bytes.restype = SZ
             L.thinkv_append_quantize.argtypes = [C.POINTER(CacheStruct), I32, P, P, P, P, P, P, SZ, P]
             L.thinkv_append_quantize.restype = C.c_int
+            L.thinkv_append_evict.argtypes = [C.POINTER(CacheStruct), I32, P, P, P, P, P, P, P, P, SZ, P]
+            L.thinkv_append_evict.restype = C.c_int
             L.thinkv_evict.argtypes = [C.POINTER(CacheStruct), I32, P, P, P, P]
             L.thinkv_evict.restype = C.c_int
             L.thinkv_decode_workspace_bytes.argtypes = [C.POINTER(Layout), I32, I32]
@@ -274,6 +277,27 @@ class ThinKVCache:
         _check(lib().thinkv_append_quantize(C.byref(self.cs), n, _ptr(seq), _ptr(pos), _ptr(tag),
                                             _ptr(k), _ptr(v), _ptr(ws), ws.numel(),
                                             _stream(stream)), "append")
+
+    def append_evict(self, seq: torch.Tensor, pos: torch.Tensor, tag: torch.Tensor,
+                     k: torch.Tensor, v: torch.Tensor, budget: torch.Tensor,
+                     order: Optional[Sequence[int]] = None, stream=None):
+        """Append, then evict each sequence of the call to its budget (one launch
+        for calls of up to 512 tokens).  budget: int32 per token; the value at
+        each sequence's first token counts."""
+        n = int(seq.numel())
+        if n == 0:
+            return
+        assert seq.dtype == torch.int32 and pos.dtype == torch.int32 and tag.dtype == torch.uint8
+        assert budget.dtype == torch.int32 and budget.numel() == n
+        assert k.dtype == torch.float16 and v.dtype == torch.float16
+        assert k.is_contiguous() and v.is_contiguous() and k.numel() == n * self.H * self.d
+        nbytes = int(lib().thinkv_append_workspace_bytes(C.byref(self.layout), n))
+        ws = self._workspace("append", nbytes)
+        o = None if order is None else (C.c_uint8 * 3)(*order)
+        _check(lib().thinkv_append_evict(C.byref(self.cs), n, _ptr(seq), _ptr(pos), _ptr(tag),
+                                         _ptr(k), _ptr(v), _ptr(budget),
+                                         None if o is None else C.cast(o, C.c_void_p),
+                                         _ptr(ws), ws.numel(), _stream(stream)), "append_evict")
 
     def evict(self, seq: torch.Tensor, budget: torch.Tensor, order: Optional[Sequence[int]] = None,
               stream=None):

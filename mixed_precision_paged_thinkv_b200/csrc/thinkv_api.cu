@@ -206,6 +206,33 @@ int thinkv_append_quantize(const thinkv_cache* C, int32_t n, const int32_t* seq,
                                    static_cast<cudaStream_t>(stream), sms));
 }
 
+int thinkv_append_evict(const thinkv_cache* C, int32_t n, const int32_t* seq, const int32_t* pos,
+                        const uint8_t* tag, const uint16_t* k, const uint16_t* v,
+                        const int32_t* budget, const uint8_t* order, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!cache_ok(C) || n < 0) return THINKV_ERR_INVALID;
+  uint8_t o[3] = {THINKV_T, THINKV_E, THINKV_R};
+  if (order) {
+    for (int x = 0; x < 3; ++x) {
+      if (order[x] > 2) return THINKV_ERR_INVALID;
+      o[x] = order[x];
+    }
+    if (o[0] == o[1] || o[0] == o[2] || o[1] == o[2]) return THINKV_ERR_INVALID;
+  }
+  if (n == 0) return THINKV_OK;
+  if (!seq || !pos || !tag || !k || !v || !budget) return THINKV_ERR_INVALID;
+  if (!aligned(seq, 4) || !aligned(pos, 4) || !aligned(budget, 4) || !aligned(k, 16) ||
+      !aligned(v, 16))
+    return THINKV_ERR_INVALID;
+  if (workspace && !aligned(workspace, 16)) return THINKV_ERR_INVALID;
+  if (!workspace || workspace_bytes < append_workspace_bytes(n)) return THINKV_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return THINKV_ERR_CUDA;
+  const AppendWorkspace ws = carve_append_workspace(workspace, n);
+  return cuda_status(launch_append(view_of(C), n, seq, pos, tag, k, v, ws,
+                                   static_cast<cudaStream_t>(stream), sms, budget, o));
+}
+
 int thinkv_evict(const thinkv_cache* C, int32_t n, const int32_t* seq, const int32_t* budget,
                  const uint8_t* order, void* stream) {
   if (!cache_ok(C) || n < 0) return THINKV_ERR_INVALID;

@@ -21,6 +21,7 @@
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
+#include "thinkv_evict_seq.cuh"
 #include "thinkv_internal.h"
 
 namespace thinkv {
@@ -198,7 +199,7 @@ __device__ void assign_run(const CacheView& C, int s, int start, int len, const 
 __global__ void __launch_bounds__(kAssignThreads, 1)
     append_assign_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
                          const int32_t* __restrict__ pos, const uint8_t* __restrict__ tag,
-                         AppendWorkspace ws) {
+                         AppendWorkspace ws, const int32_t* __restrict__ budget) {
   extern __shared__ uint32_t seen[];  // max_seqs bits
   __shared__ int s_err;
   __shared__ int s_blocks_bad;
@@ -227,6 +228,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       bool bad = s < 0 || s >= max_seqs || c > 2 || p < 0;
       start = (i == 0) || seq[i - 1] != s;
       if (!bad && !start && p <= pos[i - 1]) bad = true;
+      if (!bad && start && budget != nullptr && budget[i] < 0) bad = true;   // the evict that follows
       if (!bad && start) {
         uint32_t old = atomicOr(&seen[s >> 5], 1u << (s & 31));
         if (old & (1u << (s & 31))) bad = true;  // a sequence in two runs
@@ -590,7 +592,7 @@ __global__ void __launch_bounds__(kSmallThreads)
     append_small_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
                         const int32_t* __restrict__ pos, const uint8_t* __restrict__ tag,
                         const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-                        uint32_t* arrive) {
+                        uint32_t* arrive, const int32_t* __restrict__ budget, uint32_t order) {
   constexpr int NST = 9;                          // counters per run (see assign_run)
   extern __shared__ uint32_t seen[];              // max_seqs bits
   __shared__ int r_cnt[kSmallAppend * 3];         // per run: tokens of each class
@@ -604,7 +606,10 @@ __global__ void __launch_bounds__(kSmallThreads)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int max_seqs = C.L.max_seqs, nb_max = C.L.max_blocks_per_seq, H = C.L.num_kv_heads;
   const int b = blockIdx.x;                       // the run this CTA owns (if any)
-  pdl_launch_dependents();
+  // the next kernel may be scheduled at once -- unless this launch also
+  // evicts: then its CTAs live long enough that an early decode grid would
+  // find SMs short of registers, so each CTA signals once its work is done
+  if (budget == nullptr) pdl_launch_dependents();
 
   // ---- the call's own inputs (before the previous kernel has finished) ----
   // speculative prefetch: with one token per run (a decode step), run b is
@@ -648,6 +653,7 @@ __global__ void __launch_bounds__(kSmallThreads)
     const bool start = (x == 0) || sp_[e] != s;
     bool bx = s < 0 || s >= max_seqs || c > 2 || p < 0;
     if (!bx && !start && p <= pp_[e]) bx = true;
+    if (!bx && start && budget != nullptr && budget[x] < 0) bx = true;   // the evict that follows
     if (!bx && start) {
       const uint32_t old = atomicOr(&seen[s >> 5], 1u << (s & 31));
       if (old & (1u << (s & 31))) bx = true;          // a sequence in two runs
@@ -758,6 +764,10 @@ __global__ void __launch_bounds__(kSmallThreads)
       assign_run(C, s, start, len, cnt, base, pos, tag, tok_slot - start, r_st + b * NST);
     }
     __syncthreads();
+    // append + evict: warp 0 then takes the sequence down to its budget (its
+    // counters are final once the barrier has passed; the other warps store
+    // the run's codes meanwhile, into slots the evict does not read)
+    if (budget != nullptr && warp == 0) evict_seq(C, s, budget[start], order, false);
     const int64_t units = (int64_t)len * H * 2;
     for (int64_t u = warp; u < units; u += kSmallWarps) {
       const int kv = (int)(u & 1);
@@ -775,6 +785,7 @@ __global__ void __launch_bounds__(kSmallThreads)
 
   // ---- the last CTA to finish advances the page-pool counters ----
   __syncthreads();
+  if (budget != nullptr) pdl_launch_dependents();
   if (tid == 0) {
     __threadfence();
     const uint32_t old = atomicAdd(arrive, 1u);
@@ -808,18 +819,21 @@ AppendWorkspace carve_append_workspace(void* ws, int32_t n) {
 
 cudaError_t launch_append(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* pos,
                           const uint8_t* tag, const uint16_t* k, const uint16_t* v,
-                          const AppendWorkspace& ws, cudaStream_t stream, int num_sms) {
+                          const AppendWorkspace& ws, cudaStream_t stream, int num_sms,
+                          const int32_t* budget, const uint8_t* order) {
   const size_t seen_bytes = (size_t)((C.L.max_seqs + 31) / 32) * 4;
   const int D = C.L.head_dim, G = C.L.group_size;
+  const uint32_t packed =
+      order ? ((uint32_t)order[0] | ((uint32_t)order[1] << 8) | ((uint32_t)order[2] << 16)) : 0u;
   if (n <= kSmallAppend) {
     auto kern = (D == 128 && G == 64)   ? append_small_kernel<128, 64>
                 : (D == 128 && G == 32) ? append_small_kernel<128, 32>
                 : (D == 64 && G == 64)  ? append_small_kernel<64, 64>
                                         : append_small_kernel<64, 32>;
     return launch_pdl(kern, dim3(n), dim3(kSmallThreads), seen_bytes, stream, C, n, seq, pos, tag,
-                      k, v, ws.arrive);
+                      k, v, ws.arrive, budget, packed);
   }
-  append_assign_kernel<<<1, kAssignThreads, seen_bytes, stream>>>(C, n, seq, pos, tag, ws);
+  append_assign_kernel<<<1, kAssignThreads, seen_bytes, stream>>>(C, n, seq, pos, tag, ws, budget);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int64_t units = (int64_t)n * C.L.num_kv_heads * 2;
@@ -831,7 +845,10 @@ cudaError_t launch_append(const CacheView& C, int32_t n, const int32_t* seq, con
   else if (D == 128 && G == 32) append_scatter_kernel<128, 32><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
   else if (D == 64 && G == 64) append_scatter_kernel<64, 64><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
   else append_scatter_kernel<64, 32><<<(int)blocks, 256, 0, stream>>>(C, n, tag, k, v, ws);
-  return cudaGetLastError();
+  err = cudaGetLastError();
+  if (err != cudaSuccess || budget == nullptr) return err;
+  // append + evict on a large call: each run's sequence to its budget
+  return launch_evict_runs(C, n, seq, budget, order, stream);
 }
 
 }  // namespace thinkv

@@ -17,6 +17,7 @@
 #include <stdint.h>
 
 #include "thinkv_common.cuh"
+#include "thinkv_evict_seq.cuh"
 #include "thinkv_internal.h"
 
 namespace thinkv {
@@ -26,13 +27,14 @@ namespace {
 constexpr int kEvictThreads = 1024;
 constexpr int kEvictWarps = kEvictThreads / 32;
 
-__device__ void evict_seq(const CacheView& C, int s, int bud, uint32_t order, bool check_status);
 
 // Calls of any size: one CTA validates the call (all-or-nothing), then a warp
-// per sequence evicts it (evict_seq).
+// per sequence evicts it (evict_seq).  With `runs`, seq and budget are an
+// append's token arrays: only the first token of each run of a sequence names
+// it (and its budget).
 __global__ void __launch_bounds__(kEvictThreads, 1)
     evict_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
-                 const int32_t* __restrict__ budget, uint32_t order) {
+                 const int32_t* __restrict__ budget, uint32_t order, bool runs) {
   extern __shared__ uint32_t seen[];  // max_seqs bits
   __shared__ int s_err;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -43,6 +45,7 @@ __global__ void __launch_bounds__(kEvictThreads, 1)
   if (s_err != 0) return;
   for (int i = tid; i < n; i += kEvictThreads) {
     int s = seq[i];
+    if (runs && i > 0 && seq[i - 1] == s) continue;
     bool bad = s < 0 || s >= max_seqs || budget[i] < 0;
     if (!bad) {
       uint32_t old = atomicOr(&seen[s >> 5], 1u << (s & 31));
@@ -55,7 +58,8 @@ __global__ void __launch_bounds__(kEvictThreads, 1)
     if (tid == 0) set_status(C.status, s_err);
     return;
   }
-  for (int i = warp; i < n; i += kEvictWarps) evict_seq(C, seq[i], budget[i], order, false);
+  for (int i = warp; i < n; i += kEvictWarps)
+    if (!runs || i == 0 || seq[i - 1] != seq[i]) evict_seq(C, seq[i], budget[i], order, false);
 }
 
 
@@ -69,114 +73,6 @@ constexpr int kSmallEvict = 512;
 constexpr int kSmallEvictThreads = 256;
 constexpr int kSmallEvictWarps = kSmallEvictThreads / 32;
 
-// Evicts sequence s down to `bud` live tokens (one warp).  The class order is
-// packed one class per byte.  All of s's counters are loaded at once (with
-// the sticky status when check_status: a set status makes this a no-op).
-// Victims are the oldest live entries of the first class in order that has
-// one, then the next class: each class FIFO is scanned from its head 32
-// entries at a time; -1 entries are tombstones (tokens TBE evicted away from
-// the head), stepped over and consumed like the victims before them.
-__device__ void evict_seq(const CacheView& C, int s, int bud, uint32_t order,
-                          bool check_status) {
-  const int lane = threadIdx.x & 31;
-  const int nb_max = C.L.max_blocks_per_seq;
-  const int64_t cap = (int64_t)nb_max * kPage;
-  // lanes 0-2: FIFO heads, 3-5: FIFO tails, 6-8: stack tops (classes in
-  // order), 9: live_count, 10: num_live
-  int val = 0;
-  {
-    const int o = lane % 3, c = (int)((order >> (8 * o)) & 0xFFu);
-    if (lane < 3) val = C.fifo_head[s * 3 + c];
-    else if (lane < 6) val = C.fifo_tail[s * 3 + c];
-    else if (lane < 9) val = C.free_top[s * 3 + c];
-    else if (lane == 9) val = C.live_count[s];
-    else if (lane == 10) val = C.num_live[s];
-    else if (lane == 11 && check_status) val = *C.status;
-  }
-  if (check_status && __shfl_sync(0xFFFFFFFFu, val, 11) != 0) return;
-  const int live = __shfl_sync(0xFFFFFFFFu, val, 9);
-  int nlive = __shfl_sync(0xFFFFFFFFu, val, 10);
-  int remaining = live - bud;
-  if (remaining <= 0) return;
-  uint64_t* table = C.block_table + (int64_t)s * nb_max;
-  uint64_t* llist = C.live_list + (int64_t)s * nb_max;
-  int32_t* lidx = C.live_index + (int64_t)s * nb_max;
-  int total = 0;
-  int new_head = 0, new_top = 0;                     // lane o < 3 keeps class o's values
-  for (int o = 0; o < 3; ++o) {
-    const int c = (int)((order >> (8 * o)) & 0xFFu);
-    int idx = __shfl_sync(0xFFFFFFFFu, val, o);
-    const int tail = __shfl_sync(0xFFFFFFFFu, val, 3 + o);
-    int top = __shfl_sync(0xFFFFFFFFu, val, 6 + o);
-    const int32_t* ring = C.fifo + ((int64_t)s * 3 + c) * cap;
-    int32_t* stack = C.free_slots + ((int64_t)s * 3 + c) * cap;
-    while (remaining > 0 && idx < tail) {
-      const int cnt = min(32, tail - idx);
-      const int32_t ts = lane < cnt ? ring[((int64_t)idx + lane) % cap] : -1;
-      const unsigned lbal = __ballot_sync(0xFFFFFFFFu, ts >= 0);
-      const int rank = __popc(lbal & ((1u << lane) - 1u));
-      const bool valid = ts >= 0 && rank < remaining;
-      const unsigned vbal = __ballot_sync(0xFFFFFFFFu, valid);
-      const int nv = __popc(vbal);
-      // the quota reached: consumed up to the last victim; else the whole chunk
-      const int consumed = (nv == remaining) ? 32 - __clz(vbal) : cnt;
-      const int e = valid ? (ts >> 4) : -1, slot = ts & 15;
-      // merge the bits of victims that share an entry (entries are class-pure);
-      // the highest such lane writes the entry
-      const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? e : -1 - lane);
-      const uint32_t bits = __reduce_or_sync(grp, valid ? (1u << slot) : 0u);
-      const bool last = valid && (31 - __clz(grp)) == lane;
-      bool emptied = false;
-      if (valid) {
-        // through L2: an earlier batch may have rewritten this entry
-        const uint64_t ent = __ldcg(&table[e]);
-        const uint32_t page = entry_page(ent);
-        if (last) {
-          const uint32_t mask = entry_mask(ent) & ~bits;
-          table[e] = (ent & 0x0000FFFFFFFFFFFFull) | ((uint64_t)mask << 48);
-          emptied = (mask == 0);
-        }
-        C.slot_pos[c][(int64_t)page * kPage + slot] = -1;
-        stack[top + rank] = ts;
-      }
-      // entries emptied in this batch leave the live list in victim order
-      unsigned ev = __ballot_sync(0xFFFFFFFFu, emptied);
-      __syncwarp();
-      while (ev) {
-        const int src = __ffs(ev) - 1;
-        const int ee = __shfl_sync(0xFFFFFFFFu, e, src);
-        if (lane == 0) {
-          const int lastpos = nlive - 1;
-          const int at = __ldcg(&lidx[ee]);
-          const uint64_t moved = __ldcg(&llist[lastpos]);
-          llist[at] = moved;
-          lidx[live_desc_entry(moved)] = at;
-          lidx[ee] = -1;
-        }
-        --nlive;
-        __syncwarp();
-        ev &= ev - 1;
-      }
-      top += nv;
-      remaining -= nv;
-      total += nv;
-      idx += consumed;
-    }
-    if (lane == o) {
-      new_head = idx;
-      new_top = top;
-    }
-  }
-  if (lane < 3) {
-    const int c = (int)((order >> (8 * lane)) & 0xFFu);
-    C.fifo_head[s * 3 + c] = new_head;
-    C.free_top[s * 3 + c] = new_top;
-  }
-  if (lane == 0) {
-    C.live_count[s] = live - total;
-    C.num_live[s] = nlive;
-  }
-}
 
 __global__ void __launch_bounds__(kSmallEvictThreads)
     evict_small_kernel(CacheView C, int32_t n, const int32_t* __restrict__ seq,
@@ -226,7 +122,15 @@ cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, cons
     return launch_pdl(evict_small_kernel, dim3(grid), dim3(kSmallEvictThreads), seen_bytes, stream,
                       C, n, seq, budget, packed);
   }
-  evict_kernel<<<1, kEvictThreads, seen_bytes, stream>>>(C, n, seq, budget, packed);
+  evict_kernel<<<1, kEvictThreads, seen_bytes, stream>>>(C, n, seq, budget, packed, false);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_evict_runs(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
+                              const uint8_t order[3], cudaStream_t stream) {
+  const uint32_t packed = (uint32_t)order[0] | ((uint32_t)order[1] << 8) | ((uint32_t)order[2] << 16);
+  const size_t seen_bytes = (size_t)((C.L.max_seqs + 31) / 32) * 4;
+  evict_kernel<<<1, kEvictThreads, seen_bytes, stream>>>(C, n, seq, budget, packed, true);
   return cudaGetLastError();
 }
 

@@ -47,12 +47,19 @@ struct AppendWorkspace {
 
 size_t append_workspace_bytes(int32_t n);
 AppendWorkspace carve_append_workspace(void* ws, int32_t n);
+// budget (device, per token; the value at each run's first token counts) and
+// order (host, 3 classes): the append is followed by an evict of each run's
+// sequence to its budget, in one launch for calls of up to 512 tokens
 cudaError_t launch_append(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* pos,
                           const uint8_t* tag, const uint16_t* k, const uint16_t* v,
-                          const AppendWorkspace& ws, cudaStream_t stream, int num_sms);
+                          const AppendWorkspace& ws, cudaStream_t stream, int num_sms,
+                          const int32_t* budget = nullptr, const uint8_t* order = nullptr);
 
 cudaError_t launch_evict(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
                          const uint8_t order[3], cudaStream_t stream);
+// the evict of an append's runs: seq and budget are the append's token arrays
+cudaError_t launch_evict_runs(const CacheView& C, int32_t n, const int32_t* seq, const int32_t* budget,
+                              const uint8_t order[3], cudaStream_t stream);
 
 // host-side checks shared by the entry points
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }

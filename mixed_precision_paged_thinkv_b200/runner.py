@@ -164,9 +164,9 @@ def make_steps(run: "WorkloadRun", nsteps: int, first_step: int = 0, device=None
 
 def run_step(cache: ThinKVCache, inp: StepInputs, out: torch.Tensor, topk: Optional[int] = None,
              mass: Optional[torch.Tensor] = None):
-    """One step on device-resident inputs: append, evict to budget, decode."""
-    cache.append(inp.seqs, inp.pos, inp.tags, inp.k, inp.v)
-    cache.evict(inp.seqs, inp.budgets)
+    """One step on device-resident inputs: append + evict to budget (one call:
+    one token per sequence, the budgets in the same order), then decode."""
+    cache.append_evict(inp.seqs, inp.pos, inp.tags, inp.k, inp.v, inp.budgets)
     return cache.decode(inp.seqs, inp.q, topk=topk, out=out, mass=mass)
 
 
@@ -175,7 +175,7 @@ def run_step_from_host(cache: ThinKVCache, host: PackedStep, dev: PackedStep,
                        mass_dev: Optional[torch.Tensor] = None,
                        mass_host: Optional[torch.Tensor] = None):
     """One step whose inputs start in pinned host memory and whose outputs end
-    there: one host->device copy of the packed inputs, the three library
+    there: one host->device copy of the packed inputs, the two library
     calls, device->host copies, all queued on the current stream."""
     dev.buf.copy_(host.buf, non_blocking=True)
     run_step(cache, dev.inputs, out_dev, topk=topk, mass=mass_dev)

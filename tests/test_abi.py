@@ -201,3 +201,31 @@ def test_evict_slots_host_validation(lib):
     assert f(C.byref(cs), 8, ok, ok, ok, ok, need - 1, None) == binding.ERR_WORKSPACE
     assert f(C.byref(cs), 8, ok, ok, ok, None, need, None) == binding.ERR_WORKSPACE
     assert f(C.byref(cs), 0, None, None, None, None, 0, None) == 0
+
+
+def test_append_evict_host_validation(lib):
+    """thinkv_append_evict refuses a missing or misaligned budget, a bad class
+    order and the append's own bad arguments before any CUDA call."""
+    from mixed_precision_paged_thinkv_b200 import binding
+    cs = binding.CacheStruct()
+    cs.L = _layout()
+    for name, _ in binding.CacheStruct._fields_[1:]:
+        v = getattr(cs, name)
+        if isinstance(v, C.Array):
+            for i in range(3):
+                v[i] = 4096
+        else:
+            setattr(cs, name, 4096)
+    ok, odd, word = C.c_void_p(4096), C.c_void_p(4096 + 2), C.c_void_p(4096 + 4)
+    f = lib.thinkv_append_evict
+    big = 10 ** 6
+    bad_order = (C.c_uint8 * 3)(2, 2, 0)
+    far_order = (C.c_uint8 * 3)(0, 1, 3)
+    assert f(C.byref(cs), -1, ok, ok, ok, ok, ok, ok, None, ok, big, None) == 1
+    assert f(C.byref(cs), 4, ok, ok, ok, ok, ok, None, None, ok, big, None) == 1       # no budget
+    assert f(C.byref(cs), 4, ok, ok, ok, ok, ok, odd, None, ok, big, None) == 1        # budget misaligned
+    assert f(C.byref(cs), 4, ok, ok, ok, word, ok, ok, None, ok, big, None) == 1       # k misaligned
+    assert f(C.byref(cs), 4, ok, ok, ok, ok, ok, ok, C.cast(bad_order, C.c_void_p), ok, big, None) == 1
+    assert f(C.byref(cs), 4, ok, ok, ok, ok, ok, ok, C.cast(far_order, C.c_void_p), ok, big, None) == 1
+    assert f(C.byref(cs), 4, ok, ok, ok, ok, ok, ok, None, ok, 0, None) == binding.ERR_WORKSPACE
+    assert f(C.byref(cs), 0, None, None, None, None, None, None, None, None, 0, None) == 0

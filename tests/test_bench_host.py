@@ -69,8 +69,8 @@ def test_replicas_reduce_max_time_and_sum_tokens_over_two_ranks():
 
 def test_launches_per_step_counts_the_one_launch_append_path():
     import bench
-    assert bench.launches_per_step(16) == 4
-    assert bench.launches_per_step(512) == 4
+    assert bench.launches_per_step(16) == 3
+    assert bench.launches_per_step(512) == 3
     assert bench.launches_per_step(513) == 5
 
 
