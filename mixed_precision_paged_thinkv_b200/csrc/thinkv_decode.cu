@@ -1022,7 +1022,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // split combine: one CTA per (sequence, kv-head) segment that the split
 // kernel left in more than one piece
 // ---------------------------------------------------------------------------
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 256;            // the most a combine CTA takes
 constexpr int kCombinePieces = 128;             // pieces per round of the weight table
 constexpr int kCombinePre = 8;                  // pieces whose quads are requested up front
 
@@ -1086,7 +1086,7 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   const float2 ml0 = tid < np * Gq ? pair_ml(tid) : make_float2(-INFINITY, 0.f);
   if (tid < 8) { sMk[tid] = INT_MIN; sL[tid] = 0.f; }
   __syncthreads();
-  for (int x = tid; x < np * Gq; x += kCombineThreads) {
+  for (int x = tid; x < np * Gq; x += (int)blockDim.x) {
     const float m = x == tid ? ml0.x : pair_ml(x).x;
     atomicMax(&sMk[x - (x / Gq) * Gq], okey(__float_as_int(m)));
   }
@@ -1096,7 +1096,7 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j0 = 0; j0 < np; j0 += kCombinePieces) {
     const int cnt = min(kCombinePieces, np - j0);
-    for (int x = tid; x < cnt * Gq; x += kCombineThreads) {
+    for (int x = tid; x < cnt * Gq; x += (int)blockDim.x) {
       const int j = x / Gq, r = x - j * Gq;
       const float2 ml = (j0 == 0 && x == tid) ? ml0 : pair_ml(j0 * Gq + x);
       const float wgt = exp2_approx(ml.x - sM[r]);
@@ -1211,9 +1211,13 @@ cudaError_t launch_split_t(const DecodeParams& p, const DecodeLaunch& dl, cudaSt
   e = launch_pdl(decode_split_kernel<D, G, TOPK>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
                  stream, p);
   if (e != cudaSuccess) return e;
-  // the combine: one CTA per segment (most return at once)
+  // the combine: one CTA per segment (most return at once), as many threads as
+  // the segment's output quads (Gq * D/4), and a warp per head at least (the
+  // per-head sums, the top-k merges)
+  const int qt = (p.Gq * (D / 4) + 31) / 32 * 32;
+  const int ct = qt > 32 * p.Gq ? qt : 32 * p.Gq;
   return launch_pdl(decode_combine_kernel<D>, dim3((unsigned)(p.n * p.Hkv)),
-                    dim3(kCombineThreads), 0, stream, p);
+                    dim3(ct < kCombineThreads ? ct : kCombineThreads), 0, stream, p);
 }
 
 // the top-k candidate code is compiled only into the instantiation that uses it
