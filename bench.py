@@ -417,7 +417,12 @@ def _cuda_ok():
         return False
 
 
-def workload_config(w, live):
+L2_FLUSHED = "flushed between steps (512 MiB write, outside the timed events)"
+L2_LARGER = ("not flushed: the K steps run back to back, timed as one region; each step's "
+             "decode reads more than L2 holds")
+
+
+def workload_config(w, live, l2: str = L2_FLUSHED):
     cfg = {"workload": f"{w.name}: layer {w.num_q_heads}q/{w.num_kv_heads}kv heads, "
                        f"head_dim {w.head_dim}, batch {w.batch}, lengths {w.lengths}, "
                        f"R/E/T {w.bits[0]}/{w.bits[1]}/{w.bits[2]}-bit"
@@ -429,7 +434,7 @@ def workload_config(w, live):
            "batch": w.batch, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
            "head_dim": w.head_dim, "group_size": w.group_size, "page_size": w.page_size,
            "bits_RET": list(w.bits), "fmt_RET": list(w.fmt), "topk": w.topk,
-           "l2": "flushed between steps (512 MiB write, outside the timed events)",
+           "l2": l2,
            "parallelism": "replicas"}
     if live is not None:
         cfg["live_tokens_by_class"] = live
@@ -526,21 +531,35 @@ def measure_workload(w, K: int, Wm: int, dev, flush, e2e_steps: int = 0, clocks=
     if clocks is not None:
         clocks.start()
         time.sleep(0.4)
+    # a step that reads more than L2 holds cannot be helped by the previous
+    # one's cache lines: such steps run back to back, as a serving loop does,
+    # and the K steps are timed as one region; smaller ones are timed one at a
+    # time with L2 flushed between them (outside the events)
+    back_to_back = alg_bytes > L2_BYTES
     t_wall = time.time()
-    for k in range(K):
-        flush.zero_()
-        inp = steps[Wm + k]
-        # no event between the two calls (append + evict, decode): each kernel
-        # may start while the previous one finishes (programmatic dependent launch)
-        ev[k][0].record()
-        run_step(run.cache, inp, out, topk=w.topk, mass=mass)
-        ev[k][1].record()
+    if back_to_back:
+        ev[0][0].record()
+        for k in range(K):
+            run_step(run.cache, steps[Wm + k], out, topk=w.topk, mass=mass)
+        ev[0][1].record()
+    else:
+        for k in range(K):
+            flush.zero_()
+            inp = steps[Wm + k]
+            # no event between the two calls (append + evict, decode): each kernel
+            # may start while the previous one finishes (programmatic dependent launch)
+            ev[k][0].record()
+            run_step(run.cache, inp, out, topk=w.topk, mass=mass)
+            ev[k][1].record()
     torch.cuda.synchronize()
     t_wall = time.time() - t_wall
     barrier(world)
     clk = clocks.stop(str(torch.cuda.get_device_properties(dev).uuid)) if clocks is not None else None
     assert run.cache.status() == 0, "device status after the timed steps"
-    step_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    if back_to_back:
+        step_ms = [ev[0][0].elapsed_time(ev[0][1]) / K] * K
+    else:
+        step_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
     # the decode call alone, for its roofline: the same launch on the state the
     # timed steps left, L2 flushed before each
     dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -555,7 +574,8 @@ def measure_workload(w, K: int, Wm: int, dev, flush, e2e_steps: int = 0, clocks=
     dec_ms = [a.elapsed_time(b) for a, b in dev_ev]
     res = {"step_s": sum(step_ms) / 1000.0, "steps": K, "tokens": float(w.batch * K),
            "step_ms": step_ms, "dec_ms": dec_ms, "alg_bytes": alg_bytes, "live": live,
-           "pages": pages, "clocks": clk, "wall_s": t_wall}
+           "pages": pages, "clocks": clk, "wall_s": t_wall,
+           "l2": L2_LARGER if back_to_back else L2_FLUSHED}
     if compaction:
         res["compaction"] = measure_compaction(w, run, last, out, mass, live, K, flush, dev)
 
@@ -678,7 +698,7 @@ def thinkv_arm(args, w, world, rank, local):
             rc = measure_workload(wc, Kc, 3, dev, flush)
             dec = sum(rc["dec_ms"]) / len(rc["dec_ms"])
             per_config[name] = {
-                "config": workload_config(wc, rc["live"]),
+                "config": workload_config(wc, rc["live"], rc["l2"]),
                 "steps": Kc, "warmup": 3,
                 "ms_per_step": 1000.0 * rc["step_s"] / Kc,
                 "value": rc["tokens"] / rc["step_s"], "unit": "tokens/s",
@@ -704,7 +724,7 @@ def thinkv_arm(args, w, world, rank, local):
             "dtype": "f16",
             "dtype_detail": "8/4/2-bit integer codes dequantised into f16 mma operands, f32 accumulate",
             "data": "synthetic (seeded counter-hash normals, segment tags)",
-            "config": workload_config(w, res["live"]),
+            "config": workload_config(w, res["live"], res["l2"]),
             "decode_ms": dec,
             "decode_hbm_gbs": res["alg_bytes"] / (dec / 1000.0) / 1e9,
             "decode_kv_tokens_per_s": float(sum(res["live"])) / (dec / 1000.0),
