@@ -40,10 +40,17 @@ namespace thinkv {
 
 namespace {
 
-constexpr int kDecWarps = 4;
-constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecMinBlocks = 3;                       // CTAs per SM the kernel is built for
-constexpr int kDecRegs = 65536 / (kDecThreads * kDecMinBlocks) / 8 * 8;  // register cap (168)
+// Split CTA shape per head dim: warps per CTA, and CTAs per SM the kernel is
+// built for (its register cap follows).  A d = 128 page step wants up to 168
+// registers: three 4-warp CTAs.  A d = 64 one fits in 128: two 8-warp CTAs,
+// 16 warps per SM, ran 6-10 % faster than 12 warps at 168.
+template <int D>
+struct SplitShape {
+  static constexpr int warps = D == 64 ? 8 : 4;
+  static constexpr int ctas = D == 64 ? 2 : 3;
+  static constexpr int threads = warps * 32;
+  static constexpr int regs = 65536 / (threads * ctas) / 8 * 8;   // 128 | 168
+};
 // per-warp scratch: the segment's Q fragments, lane-contiguous (the B
 // operands of the QK products)
 constexpr int kQfragOff = 0;
@@ -859,8 +866,9 @@ __device__ inline UnitMeta resolve_unit(const DecodeParams& p, const int32_t* P,
 }
 
 template <int D, int G, bool TOPK>
-__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+__global__ void __launch_bounds__(SplitShape<D>::threads, SplitShape<D>::ctas)
     decode_split_kernel(DecodeParams p) {
+  constexpr int kDecWarps = SplitShape<D>::warps, kDecThreads = SplitShape<D>::threads;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int32_t* P = reinterpret_cast<int32_t*>(smem);      // [n + 1] prefix of live pages
@@ -1024,15 +1032,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kCombineThreads = 256;            // the most a combine CTA takes
 constexpr int kCombinePieces = 128;             // pieces per round of the weight table
-constexpr int kCombinePre = 8;                  // pieces whose quads are requested up front
 
 // Merges the segment's piece records with the log-sum-exp rule: thread t <
 // Gq * D/4 owns one quad of one head's output row; warp r < Gq then sorts each
 // piece's top-k candidates for head r and merges their largest into a running
 // list (bitonic networks, the next piece's candidates loaded while the current
 // ones are sorted) for the top-k mass.
-template <int D>
-__global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(DecodeParams p) {
+template <int D, bool TOPK>
+__global__ void __launch_bounds__(kCombineThreads, TOPK ? 4 : 3) decode_combine_kernel(DecodeParams p) {
   constexpr int QD = D / 4;
   __shared__ float sM[8], sL[8];
   __shared__ int sMk[8];
@@ -1059,6 +1066,9 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
     return recs + pc * rb;
   };
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // pieces whose quads are requested up front (fewer with top-k, whose CTAs
+  // are built to fit four to an SM)
+  constexpr int kCombinePre = TOPK ? 4 : 8;
 
   // ---- per piece and head: the weight 2^(m - M) (M the head's max), and L ----
   // (m, l) pairs are read once, lane-parallel; a table of weights in shared
@@ -1153,31 +1163,126 @@ __global__ void __launch_bounds__(kCombineThreads, 3) decode_combine_kernel(Deco
     if (lane == 0) p.mass[mrow] = 1.f;
     return;
   }
-  // each piece's candidates (128, unsorted) sorted ascending put its 64
-  // largest in elements 64..127, rising; with the running list (descending)
-  // in elements 0..63 that is a bitonic sequence
+  // The running list holds the 64 largest candidates so far, descending, in
+  // elements 0..63 (lane * 4 + e); its k-th element is exact, the rest of it
+  // need not be.  A piece's candidates at or below that k-th value cannot
+  // enter the top k (a tie leaves the sum unchanged) and are dropped.  Up to
+  // 32 survivors are gathered one per lane, sorted (32-wide network) and put
+  // rising in elements 96..127 (-inf in 64..95); more are sorted whole, their
+  // 64 largest rising in elements 64..127.  Either way, with the running list
+  // in 0..63 that is a bitonic sequence, which one merge puts in order.
   float tv[4], nx[4];
   auto load_list = [&](int j, float (&x)[4]) {
     const float4 v = __ldcg(reinterpret_cast<const float4*>(rec(j) + 64 + 4 * Gq * D) +
                             r * (kCandCap / 4) + lane);
     x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
   };
+  float* ys = cwt + warp * 32;                    // gather slots (the weight table is free now)
+  unsigned below;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(below));
+  // the survivors (at most 32) of this lane's candidates x, one per lane
+  // (-inf past the c-th), in descending order
+  auto gather_sorted = [&](const float (&x)[4], const unsigned (&b)[4], float th, int c) {
+    int at = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (x[e] > th) ys[at + __popc(b[e] & below)] = x[e];
+      at += __popc(b[e]);
+    }
+    __syncwarp();
+    const float y = lane < c ? ys[lane] : -INFINITY;
+    __syncwarp();                                 // the slots are rewritten by the next piece
+    return bitonic32_desc(y);
+  };
+  const float M = sM[r];
+  if (k <= 32) {
+    // k <= 32: the running list is the 32 largest so far, one per lane,
+    // descending (lane 0 the largest); its k-th element is the threshold
+    float rv = -INFINITY;
+    load_list(0, nx);
+    for (int j = 0; j < np; ++j) {
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] = nx[e];
+      if (j + 1 < np) load_list(j + 1, nx);
+      const float th = __shfl_sync(0xFFFFFFFFu, rv, k - 1);
+      unsigned b[4];
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        b[e] = __ballot_sync(0xFFFFFFFFu, x[e] > th);
+        c += __popc(b[e]);
+      }
+      if (c == 0) continue;
+      float y;
+      if (c <= 32) {
+        y = gather_sorted(x, b, th, c);
+      } else {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = -x[e];
+        bitonic128_desc(v);                       // descending of -x: ascending of x
+        // the lane-th largest is element 127 - lane: lane 31 - lane/4, slot 3 - lane%4
+        const int sl = 31 - (lane >> 2), se = 3 - (lane & 3);
+        const float t0 = __shfl_sync(0xFFFFFFFFu, v[0], sl), t1 = __shfl_sync(0xFFFFFFFFu, v[1], sl);
+        const float t2 = __shfl_sync(0xFFFFFFFFu, v[2], sl), t3 = __shfl_sync(0xFFFFFFFFu, v[3], sl);
+        y = -(se == 0 ? t0 : (se == 1 ? t1 : (se == 2 ? t2 : t3)));
+      }
+      // the 32 largest of two descending lists: each element against the
+      // other list's mirror element; the maxima form a bitonic sequence
+      float z = fmaxf(rv, __shfl_sync(0xFFFFFFFFu, y, 31 - lane));
+#pragma unroll
+      for (int stride = 16; stride > 0; stride >>= 1) {
+        const float o = __shfl_xor_sync(0xFFFFFFFFu, z, stride);
+        z = (lane & stride) == 0 ? fmaxf(z, o) : fminf(z, o);
+      }
+      rv = z;
+    }
+    float sum = lane < k ? exp2_approx(rv - M) : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane == 0) p.mass[mrow] = sum / sL[r];
+    return;
+  }
+  const int ke = (k - 1) & 3, kl = (k - 1) >> 2;  // the k-th element: lane kl, slot ke
 #pragma unroll
   for (int e = 0; e < 4; ++e) tv[e] = -INFINITY;
   load_list(0, nx);
   for (int j = 0; j < np; ++j) {
-    float v[4];
+    float x[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = -nx[e];
-    bitonic128_desc(v);                           // descending of -x: ascending of x
-#pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = (lane * 4 + e < 64) ? tv[e] : -v[e];
+    for (int e = 0; e < 4; ++e) x[e] = nx[e];
     if (j + 1 < np) load_list(j + 1, nx);
+    const float kv = ke == 0 ? tv[0] : (ke == 1 ? tv[1] : (ke == 2 ? tv[2] : tv[3]));
+    const float th = __shfl_sync(0xFFFFFFFFu, kv, kl);
+    unsigned b[4];
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      b[e] = __ballot_sync(0xFFFFFFFFu, x[e] > th);
+      c += __popc(b[e]);
+    }
+    if (c == 0) continue;
+    float v[4];
+    if (c <= 32) {
+      const float y = gather_sorted(x, b, th, c);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = (lane - 24) * 4 + e;        // rank in the rising run of lanes 24..31
+        const float ya = __shfl_sync(0xFFFFFFFFu, y, (31 - m) & 31);
+        v[e] = lane < 16 ? tv[e] : (lane >= 24 ? ya : -INFINITY);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = -x[e];
+      bitonic128_desc(v);                         // descending of -x: ascending of x
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = (lane * 4 + e < 64) ? tv[e] : -v[e];
+    }
     bitonic128_merge_desc(v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) tv[e] = v[e];
   }
-  const float M = sM[r];
   float sum = 0.f;
 #pragma unroll
   for (int e = 0; e < 4; ++e)
@@ -1208,7 +1313,7 @@ cudaError_t launch_split_t(const DecodeParams& p, const DecodeLaunch& dl, cudaSt
       configured[dev] = dl.smem_bytes;
     }
   }
-  e = launch_pdl(decode_split_kernel<D, G, TOPK>, dim3(dl.grid), dim3(kDecThreads), dl.smem_bytes,
+  e = launch_pdl(decode_split_kernel<D, G, TOPK>, dim3(dl.grid), dim3(SplitShape<D>::threads), dl.smem_bytes,
                  stream, p);
   if (e != cudaSuccess) return e;
   // the combine: one CTA per segment (most return at once), as many threads as
@@ -1216,7 +1321,7 @@ cudaError_t launch_split_t(const DecodeParams& p, const DecodeLaunch& dl, cudaSt
   // per-head sums, the top-k merges)
   const int qt = (p.Gq * (D / 4) + 31) / 32 * 32;
   const int ct = qt > 32 * p.Gq ? qt : 32 * p.Gq;
-  return launch_pdl(decode_combine_kernel<D>, dim3((unsigned)(p.n * p.Hkv)),
+  return launch_pdl(decode_combine_kernel<D, TOPK>, dim3((unsigned)(p.n * p.Hkv)),
                     dim3(ct < kCombineThreads ? ct : kCombineThreads), 0, stream, p);
 }
 
@@ -1241,42 +1346,48 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
   const int Gq0 = L.num_q_heads / L.num_kv_heads;
   const int q_bytes = Gq0 * D * 2;
   const int stage_bytes = (int)((maxphb + 127) / 128 * 128) + (q_bytes + 127) / 128 * 128;
-  // ~15 KB of page-head stages and top-k buffers per warp keeps three 4-warp
-  // CTAs per SM (at 8 warps per SM the top-k path ran 12-19 % slower)
   const int Gq = L.num_q_heads / L.num_kv_heads;
   const int topk_bytes = topk > 0 ? kTopkHdrBytes + Gq * kCandCap * 4 : 0;
-  int nstage = (int)((15360 - topk_bytes) / stage_bytes);
+  const int warps = D == 64 ? SplitShape<64>::warps : SplitShape<128>::warps;
+  const int ctas = D == 64 ? SplitShape<64>::ctas : SplitShape<128>::ctas;
+  const int regs = D == 64 ? SplitShape<64>::regs : SplitShape<128>::regs;
+  int smem_per_sm = 0;
+  if (cudaDeviceGetAttribute(&smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
+      cudaSuccess)
+    return false;
+  // page-head stages and top-k buffers: ~15 KB per warp, less where the CTA
+  // shape leaves less (1 KB of each CTA reserved); a deeper ring measured no
+  // faster: warps, not ring depth, hide the page step
+  int budget = (smem_per_sm / ctas - 1024 - plan_smem_bytes(n_seqs)) / warps - 64 - kPbufBytes;
+  if (budget > 15360) budget = 15360;
+  int nstage = (budget - topk_bytes) / stage_bytes;
   if (nstage < 2) nstage = 2;
   if (nstage > kMaxStages) nstage = kMaxStages;
   const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes + topk_bytes;
-  const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)kDecWarps * warp_smem;
+  const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)warps * warp_smem;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
     return false;
   if (smem + 1024 > (size_t)optin) return false;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return false;
-  int smem_per_sm = 0;
-  if (cudaDeviceGetAttribute(&smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
-      cudaSuccess)
-    return false;
   // CTAs per SM: limited by shared memory (1 KB reserved per CTA) and by registers
   int per_sm = smem_per_sm / (int)(smem + 1024);
   int regs_per_sm = 0;
   if (cudaDeviceGetAttribute(&regs_per_sm, cudaDevAttrMaxRegistersPerMultiprocessor, device) !=
       cudaSuccess)
     return false;
-  const int by_regs = regs_per_sm / (kDecRegs * kDecThreads);
+  const int by_regs = regs_per_sm / (regs * warps * 32);
   if (per_sm > by_regs) per_sm = by_regs;
   if (per_sm > 16) per_sm = 16;
   if (per_sm < 1) per_sm = 1;
   out->grid = sms * per_sm;
-  out->warps_per_cta = kDecWarps;
+  out->warps_per_cta = warps;
   out->nstage = nstage;
   out->stage_bytes = stage_bytes;
   out->smem_bytes = smem;
   out->warp_smem = warp_smem;
-  out->pieces = (int64_t)out->grid * kDecWarps + (int64_t)n_seqs * L.num_kv_heads;
+  out->pieces = (int64_t)out->grid * warps + (int64_t)n_seqs * L.num_kv_heads;
 
   return true;
 }
@@ -1325,7 +1436,7 @@ cudaError_t launch_decode(const CacheView& C, int32_t n, const int32_t* seq, con
   }
   p.topk = mass ? topk : 0;
   p.rec = w;
-  p.split_warps = (int64_t)dl.grid * kDecWarps;
+  p.split_warps = (int64_t)dl.grid * dl.warps_per_cta;
   p.live_count = C.live_count;
   p.out = out;
   p.mass = p.topk > 0 ? mass : nullptr;
