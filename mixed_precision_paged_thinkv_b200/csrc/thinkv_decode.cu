@@ -54,8 +54,7 @@ struct SplitShape {
 // per-warp scratch: the segment's Q fragments, lane-contiguous (the B
 // operands of the QK products)
 constexpr int kQfragOff = 0;
-constexpr int kQfragBytes = 2048;                       // (D / 16) k-steps x 32 lanes x 8 B
-constexpr int kPbufBytes = kQfragBytes;
+__host__ __device__ constexpr int pbuf_bytes(int D) { return D / 16 * 32 * 8; }  // k-steps x lanes x 8 B
 constexpr int kSigmaInit = 1 << 20;
 constexpr int kMaxStages = 8;                   // page ring stages (one mbarrier each)
 constexpr int kCandCap = 128;                   // top-k candidate slots per head
@@ -926,7 +925,7 @@ __global__ void __launch_bounds__(SplitShape<D>::threads, SplitShape<D>::ctas)
   float* pbuf = reinterpret_cast<float*>(wsm + p.nstage * p.stage_bytes + 64);
   TopkCtx tk;
   {
-    uint8_t* tb = wsm + p.nstage * p.stage_bytes + 64 + kPbufBytes;
+    uint8_t* tb = wsm + p.nstage * p.stage_bytes + 64 + pbuf_bytes(D);
     tk.cnt = reinterpret_cast<int*>(tb);
     tk.theta = reinterpret_cast<float*>(tb + 32);
     tk.cand = reinterpret_cast<float*>(tb + kTopkHdrBytes);
@@ -1358,12 +1357,12 @@ bool plan_decode_launch(const thinkv_layout& L, int32_t n_seqs, int32_t topk, in
   // page-head stages and top-k buffers: ~15 KB per warp, less where the CTA
   // shape leaves less (1 KB of each CTA reserved); a deeper ring measured no
   // faster: warps, not ring depth, hide the page step
-  int budget = (smem_per_sm / ctas - 1024 - plan_smem_bytes(n_seqs)) / warps - 64 - kPbufBytes;
+  int budget = (smem_per_sm / ctas - 1024 - plan_smem_bytes(n_seqs)) / warps - 64 - pbuf_bytes(D);
   if (budget > 15360) budget = 15360;
   int nstage = (budget - topk_bytes) / stage_bytes;
   if (nstage < 2) nstage = 2;
   if (nstage > kMaxStages) nstage = kMaxStages;
-  const int warp_smem = nstage * stage_bytes + 64 + kPbufBytes + topk_bytes;
+  const int warp_smem = nstage * stage_bytes + 64 + pbuf_bytes(D) + topk_bytes;
   const size_t smem = (size_t)plan_smem_bytes(n_seqs) + (size_t)warps * warp_smem;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
