@@ -682,7 +682,7 @@ def thinkv_arm(args, w, world, rank, local):
     # the raw nvidia-smi samples go to THINKV_CLOCK_LOG_DIR (default: the temp dir)
     clocks = ClockSampler(os.path.join(os.environ.get("THINKV_CLOCK_LOG_DIR", tempfile.gettempdir()),
                                        f"thinkv_clocks_rank{rank}.csv"))
-    e2e_steps = max(3, min(K, 20))
+    e2e_steps = max(3, min(K, 100))   # as many as the device-timed steps, up to 100
     res = measure_workload(w, K, Wm, dev, flush, e2e_steps=e2e_steps, clocks=clocks, world=world,
                            compaction=(world == 1))
     max_s, tokens = dist_max_sum(res["step_s"], res["tokens"], world, dev)
